@@ -1,0 +1,488 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused add + RMSNorm + dynamic-quant operator on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload c2] [--no-cpu-baseline]
+
+A step is one call of the operator (arnq_run, one kernel launch) over one
+batch of the workload: by default the 8192 x 4096 bf16 configuration
+(x1 ~ N(0,1), x2 ~ N(0,0.5), gamma, beta, smooth1, outputMask [True, False],
+INT8).  Inputs are seeded synthetic data resident in HBM before timing.  The
+timed region is exactly K steps between a barrier + synchronize on both
+sides, timed with CUDA events on the launching stream; three buffer sets are
+rotated so that every step reads inputs that are not in L2 (each set is
+larger than L2 by itself).  `value` is whole-job HBM GB/s of algorithmic
+bytes; with N GPUs (launched by torchrun, one process per GPU) every rank
+processes its own batch of the same size (weak scaling; rows are independent,
+so there is no data-path collective) and the time is the maximum over ranks.
+
+Also printed, on the same JSON line: rows/s, the roofline of the kernel
+(achieved GB/s from the mean per-launch CUDA-event duration against the
+measured copy bandwidth), the end-to-end figure through the public call with
+host buffers (H2D copies, the call, D2H of the outputs, all inside the timed
+region), SM clocks sampled by NVML during the timed region, and the CPU
+oracle's throughput on a bounded sample (rank 0, one GPU only).
+
+--impl reference times the CPU oracle (the only other implementation of the
+operator; there is no runnable reference library) on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import concurrent.futures as cf
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "fused add-RMSNorm-dynquant HBM GB/s and rows/s on 1 B200 (% of HBM peak)"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+DEFAULT_WORKLOAD = "c2"
+
+
+# ---------------------------------------------------------------- byte accounting
+
+def algorithmic_bytes(rows, n, dtype, qdtype, has_beta, has_s1, has_s2, on1, on2,
+                      has_x2=True, x_out=True):
+    """Bytes the operator must move: x1, x2 read and xOut written (2 B/element
+    each), codes (1 or 1/2 B/element) and one fp32 scale per row for every
+    produced output, and each parameter vector (gamma, beta, smooth1, smooth2)
+    read once per call."""
+    esz = 2
+    per_row = n * esz * (2 if has_x2 else 1)
+    if x_out and has_x2:
+        per_row += n * esz
+    code = n if qdtype == "int8" else n // 2
+    per_row += (code + 4) * (int(on1) + int(on2))
+    params = n * esz * (1 + int(has_beta) + int(has_s1) + int(has_s2))
+    return rows * per_row + params
+
+
+def workload_bytes(w, on1, on2):
+    return algorithmic_bytes(w.rows, w.n, w.dtype, w.qdtype, w.beta is not None,
+                             w.smooth1 is not None, w.smooth2 is not None, on1, on2)
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("int4_quant_b200/csrc/arnq_kernels.cuh", "int4_quant_b200/csrc/arnq_api.cu"):
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload_name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source; else None."""
+    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+    except Exception:
+        return None
+    e = d.get(workload_name)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks (NVML)
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML every `period` seconds."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, index, period=0.002):
+        self.index, self.period = index, period
+        self.samples, self.reasons = [], set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in self.REASONS.items():
+                    if r & bit and k != "gpu_idle":
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+
+    def stop(self):
+        if self._t:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def time_oracle(w, on1, on2, target_cpu_s=12.0, threads=None):
+    """Times the (unmodified, single-threaded) oracle over row chunks of the
+    workload run concurrently on `threads` host threads (ctypes releases the
+    GIL).  Returns (GB/s, rows/s, threads, sample description)."""
+    import oracle
+    oracle.build()
+    threads = threads or os.cpu_count() or 1
+    chunk = 64
+
+    def run_rows(r0, r1):
+        oracle.add_rms_norm_dynamic_quant_v2(
+            w.x1[r0:r1], w.x2[r0:r1], w.gamma, w.beta, w.smooth1, w.smooth2, eps=w.eps,
+            mask=w.mask, qdtype=w.qdtype, dtype=w.dtype)
+
+    t0 = time.perf_counter()
+    run_rows(0, chunk)
+    per_row = (time.perf_counter() - t0) / chunk
+    total_rows = int(max(threads * chunk, min(target_cpu_s / per_row, 64 * w.rows)))
+    jobs = []
+    r = 0
+    while r < total_rows:
+        a = r % w.rows
+        b = min(a + chunk, w.rows)
+        jobs.append((a, b))
+        r += b - a
+    t0 = time.perf_counter()
+    with cf.ThreadPoolExecutor(max_workers=threads) as ex:
+        list(ex.map(lambda ab: run_rows(*ab), jobs))
+    dt = time.perf_counter() - t0
+    rows_done = sum(b - a for a, b in jobs)
+    nbytes = workload_bytes(w, on1, on2) * rows_done / w.rows
+    sample = (f"{rows_done} rows of the {w.rows}x{w.n} workload (chunks of {chunk} rows, "
+              f"cycled) on {threads} host threads")
+    return nbytes / dt / 1e9, rows_done / dt, threads, sample
+
+
+# ---------------------------------------------------------------- reference arm
+
+def run_reference(args, w, on1, on2):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    import oracle
+    oracle.build()
+    threads = os.cpu_count() or 1
+    # size each step so that the whole run stays within about a minute
+    t0 = time.perf_counter()
+    oracle.add_rms_norm_dynamic_quant_v2(w.x1[:32], w.x2[:32], w.gamma, w.beta, w.smooth1,
+                                         w.smooth2, eps=w.eps, mask=w.mask, qdtype=w.qdtype,
+                                         dtype=w.dtype)
+    per_row = (time.perf_counter() - t0) / 32
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    rows = int(max(threads, min(w.rows, budget * threads / per_row)))
+    bounds = np.linspace(0, rows, threads + 1).astype(int)
+
+    def part(k):
+        a, b = bounds[k], bounds[k + 1]
+        if b > a:
+            oracle.add_rms_norm_dynamic_quant_v2(
+                w.x1[a:b], w.x2[a:b], w.gamma, w.beta, w.smooth1, w.smooth2, eps=w.eps,
+                mask=w.mask, qdtype=w.qdtype, dtype=w.dtype)
+
+    pool = cf.ThreadPoolExecutor(max_workers=threads)
+
+    def step(i):  # the first `rows` rows of the workload, split over the host threads
+        list(pool.map(part, range(threads)))
+
+    for i in range(args.warmup):
+        step(i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        step(i)
+    dt = time.perf_counter() - t0
+    pool.shutdown()
+    nbytes = workload_bytes(w, on1, on2) * rows / w.rows
+    value = nbytes * args.steps / dt / 1e9
+    sample = f"{rows} rows of the {w.rows}x{w.n} workload per step on {threads} host threads"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "rows_per_step": rows, "n": w.n, "io_dtype": w.dtype,
+                   "qdtype": w.qdtype},
+        "rows_per_s": rows * args.steps / dt,
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sets", type=int, default=3, help="rotated buffer sets")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    from int4_quant_b200 import workloads as wl
+    w = wl.CONFIGS[args.workload]()
+    on1 = w.mask is None or w.mask[0]
+    on2 = (w.mask is not None and w.mask[1]) or (w.mask is None and w.smooth1 is not None
+                                                 and w.smooth2 is not None)
+    if args.impl == "reference":
+        return run_reference(args, w, on1, on2)
+
+    import torch
+    import torch.distributed as dist
+    import int4_quant_b200 as q
+    from int4_quant_b200 import _abi as A
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        if args.gpus > 1:
+            sys.exit("for --gpus N > 1 launch with torch.distributed.run (one process per GPU)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        # every rank runs its own batch of the full workload (weak scaling)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    A.lib()
+    TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}[w.dtype]
+    dt_code = A.ARNQ_BF16 if w.dtype == "bf16" else A.ARNQ_FP16
+    q_code = A.ARNQ_INT8 if w.qdtype == "int8" else A.ARNQ_INT4
+    mc = q.mask_code(w.mask)
+
+    def to_dev(bits):
+        if bits is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+        return t.to(dev).view(TDT)
+
+    cb = w.n if w.qdtype == "int8" else w.n // 2
+    params = [to_dev(a) for a in (w.gamma, w.beta, w.smooth1, w.smooth2)]
+    x1h, x2h = w.x1, w.x2
+    sets = []
+    for _ in range(args.sets):
+        sets.append(dict(
+            x1=to_dev(x1h), x2=to_dev(x2h),
+            y1=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if on1 else None,
+            s1=torch.empty((w.rows,), dtype=torch.float32, device=dev) if on1 else None,
+            y2=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if on2 else None,
+            s2=torch.empty((w.rows,), dtype=torch.float32, device=dev) if on2 else None,
+            xo=torch.empty((w.rows, w.n), dtype=TDT, device=dev)))
+    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sptr = stream.cuda_stream
+
+    def launch(s):
+        st = A.arnq_run(s["x1"], s["x2"], params[0], params[1], params[2], params[3], w.rows, w.n,
+                        dt_code, w.eps, mc, q_code, s["y1"], s["s1"], s["y2"], s["s2"], s["xo"], ws,
+                        256, sptr)
+        if st != A.ARNQ_OK:
+            raise A.ArnqError(st, "arnq_run")
+
+    st, plan = A.arnq_make_plan(sets[0]["x1"], sets[0]["x2"], *params, w.rows, w.n, dt_code, mc,
+                                q_code, sets[0]["y1"], sets[0]["y2"], sets[0]["xo"])
+    if st != A.ARNQ_OK:
+        raise A.ArnqError(st, "arnq_make_plan")
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize(dev)
+
+    # ---- warm-up
+    for i in range(args.warmup):
+        launch(sets[i % args.sets])
+    barrier()
+
+    # ---- timed region: exactly K steps
+    K = args.steps
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier()
+    for i in range(K):
+        ev0[i].record(stream)
+        launch(sets[i % args.sets])
+        ev1[i].record(stream)
+    barrier()
+    clocks.stop()
+    total_ms = ev0[0].elapsed_time(ev1[K - 1])
+    launch_ms = [ev0[i].elapsed_time(ev1[i]) for i in range(K)]
+    wsh = ws[:16].cpu().numpy().view(np.int32)
+    if wsh[0] != 0:
+        raise RuntimeError(f"kernel reported device status {wsh[0]}")
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    nbytes = workload_bytes(w, on1, on2)
+    value = nbytes * K * world / (total_ms / 1e3) / 1e9
+    rows_per_s = w.rows * K * world / (total_ms / 1e3)
+    mean_launch_ms = statistics.fmean(launch_ms)
+    achieved = nbytes / (mean_launch_ms / 1e3) / 1e9
+    peak, peak_kind = measured_peaks()
+
+    # ---- end to end through the public call, host buffers, copies timed
+    e2e_steps = max(1, args.e2e_steps)
+    x1p = torch.from_numpy(np.ascontiguousarray(x1h).view(np.int16)).view(TDT).pin_memory()
+    x2p = torch.from_numpy(np.ascontiguousarray(x2h).view(np.int16)).view(TDT).pin_memory()
+    outs_h = {}
+    s0 = sets[0]
+    for k, t in (("y1", s0["y1"]), ("s1", s0["s1"]), ("y2", s0["y2"]), ("s2", s0["s2"]),
+                 ("xo", s0["xo"])):
+        if t is not None:
+            outs_h[k] = torch.empty(t.shape, dtype=t.dtype).pin_memory()
+    h2d = x1p.numel() * 2 * 2
+    d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
+    ge = s0
+
+    def e2e_step():
+        ge["x1"].copy_(x1p, non_blocking=True)
+        ge["x2"].copy_(x2p, non_blocking=True)
+        q.add_rms_norm_dynamic_quant(
+            ge["x1"], ge["x2"], params[0], params[1], params[2], params[3], eps=w.eps,
+            output_mask=w.mask, qdtype=w.qdtype,
+            out={"y1": ge["y1"], "scale1": ge["s1"], "y2": ge["y2"], "scale2": ge["s2"],
+                 "x_out": ge["xo"]})
+        for k, t in outs_h.items():
+            t.copy_(ge[k], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    barrier()
+    e_start = torch.cuda.Event(enable_timing=True)
+    e_end = torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e_end.record(stream)
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e_value = nbytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        gbs, rps, cores, sample = time_oracle(w, on1, on2)
+        cpu = {"value": gbs, "unit": "GB/s", "cores": cores, "kind": "oracle", "sample": sample,
+               "rows_per_s": rps}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": total_ms / K,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f32",
+        "data": "synthetic (seeded numpy PCG64, rounded to the input dtype; no dataset exists)",
+        "config": {
+            "workload": w.name, "rows": w.rows, "n": w.n, "io_dtype": w.dtype,
+            "qdtype": w.qdtype, "output_mask": w.mask, "beta": w.beta is not None,
+            "smooth1": w.smooth1 is not None, "smooth2": w.smooth2 is not None, "eps": w.eps,
+            "l2": f"{args.sets} rotated buffer sets, inputs {2 * w.rows * w.n * 2 / 1e6:.0f} MB "
+                  f"per set (> 126 MB L2)",
+            "plan": plan.as_dict(),
+            "parallelism": f"replicas x{world} (rows independent; no collective)",
+        },
+        "rows_per_s": rows_per_s,
+        "bytes_per_step": nbytes,
+        "frac_of_nominal_hbm": value / world / NOMINAL_HBM_GBS,
+        "roofline": {
+            "bound": "hbm",
+            "achieved": achieved,
+            "peak": peak,
+            "unit": "GB/s",
+            "frac": achieved / peak,
+            "traffic": recorded_traffic(w.name),
+            "peak_kind": peak_kind,
+            "kernel": "arnq::rows_kernel",
+            "mean_launch_us": mean_launch_ms * 1e3,
+            "median_launch_us": statistics.median(launch_ms) * 1e3,
+        },
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                "ms_per_step": e2e_ms / e2e_steps},
+        "gpu_launches": K,
+        "clocks": clocks.summary(),
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

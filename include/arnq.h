@@ -1,0 +1,215 @@
+/*
+ * arnq.h -- C ABI of a B200 (sm_100a) library for the fused residual add +
+ * RMSNorm + per-row symmetric dynamic quantization operator.
+ *
+ * The operator is the one defined on the CANN page
+ * "aclnnAddRmsNormDynamicQuantV2", section "Formula":
+ *
+ *     x        = x1 + x2                                (written out as xOut)
+ *     Rms(x)   = sqrt( (1/n) * sum_i x_i^2 + epsilon )  (over the last dim, n)
+ *     y        = x / Rms(x) * gamma + beta
+ *     input_k  = y * smoothScale_k   if smoothScale_k is given, else y
+ *     scale_k  = row_max(|input_k|) / Q                 (Q = 127 INT8, 7 INT4)
+ *     y_k      = round(input_k / scale_k)
+ *
+ * with one or two quantized outputs selected by outputMask and the smooth
+ * scales as that page states (see arnq_selected_outputs), and the argument
+ * rules of its "Constraints" section.  The no-add form is the page
+ * "aclnnRmsNormDynamicQuant", formula section.
+ *
+ * Numerical conventions (the pages leave these open; the library fixes them):
+ *   - x1 + x2 is a binary32 add rounded once more, to nearest even, to the
+ *     input dtype; that rounded x is written as xOut AND is the x that is
+ *     normalised.
+ *   - y and input_k are kept in binary32 and never rounded to 16 bits.
+ *   - scale_k is a binary32 value; the codes are the quotient input_k/scale_k
+ *     rounded half-to-even and clamped to [-Q, Q].  A row whose scale is 0
+ *     (all inputs 0) gets scale 0 and all codes 0.
+ *   - INT4 codes are two's-complement nibbles packed two per byte, the even
+ *     column in the low nibble; an INT4 row of n codes occupies n/2 bytes.
+ *   - Results are deterministic: the same inputs and the same plan give the
+ *     same bits on every run ("Deterministic compute" in the Constraints
+ *     section).  Sums are fixed-order trees; there are no float atomics.
+ *
+ * Layout: every tensor is dense row-major ("ND" in the Constraints section).
+ *   x1, x2, xOut : [rows, n] of dtype (bf16 or fp16)
+ *   gamma, beta, smooth1, smooth2 : [n] of dtype
+ *   y1, y2 : [rows, n] int8, or [rows, n/2] bytes of packed INT4
+ *   scale1, scale2 : [rows] binary32
+ *
+ * Ownership: the caller owns every buffer.  All tensor pointers are DEVICE
+ * pointers on the current CUDA device.  The library allocates nothing, never
+ * synchronizes, and launches only on the given stream (a cudaStream_t passed
+ * as void *; NULL is the legacy default stream).  Outputs that are not
+ * selected are never written and may be NULL.  xOut may be the same pointer
+ * as x1 or x2 (in-place residual update); any other overlap between an
+ * output and an input is undefined.
+ *
+ * Errors: every argument check happens on the host before anything is
+ * launched; a failing call writes nothing and returns the status.  A launch
+ * failure returns ARNQ_ERR_CUDA (cudaGetLastError() holds the CUDA error).
+ * Kernels that wait on asynchronous copies do so with a time limit; if a wait
+ * expires the kernel stops early and records ARNQ_ERR_DEVICE_TIMEOUT in the
+ * workspace's status block (see arnq_workspace_status).
+ */
+#ifndef ARNQ_H
+#define ARNQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ARNQ_API __attribute__((visibility("default")))
+#else
+#define ARNQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum arnq_status {
+  ARNQ_OK = 0,
+  ARNQ_ERR_NULL_PTR = 1,        /* a required input, or a selected output, is NULL        */
+  ARNQ_ERR_EMPTY = 2,           /* rows == 0 or n == 0: empty tensors are not supported    */
+  ARNQ_ERR_SHAPE = 3,           /* INT4 with odd n; n above ARNQ_MAX_N; negative sizes     */
+  ARNQ_ERR_DTYPE = 4,           /* unknown dtype or qdtype                                 */
+  ARNQ_ERR_MASK = 5,            /* outputMask / smooth-scale combination the page forbids  */
+  ARNQ_ERR_EPS = 6,             /* epsilon negative or not finite                          */
+  ARNQ_ERR_ALIGN = 7,           /* a 16-bit tensor not 2-byte aligned, a scale not 4-byte  */
+  ARNQ_ERR_WORKSPACE = 8,       /* workspace NULL or smaller than arnq_workspace_size()    */
+  ARNQ_ERR_CUDA = 9,            /* a CUDA call failed (launch, attribute, device query)    */
+  ARNQ_ERR_PLAN = 10,           /* an explicit plan that cannot run this problem           */
+  ARNQ_ERR_DEVICE_TIMEOUT = 11  /* reported through the workspace status block only        */
+} arnq_status;
+
+typedef enum arnq_dtype { ARNQ_BF16 = 0, ARNQ_FP16 = 1 } arnq_dtype;
+typedef enum arnq_qdtype { ARNQ_INT8 = 0, ARNQ_INT4 = 1 } arnq_qdtype;
+
+/* outputMask encoding: ARNQ_MASK_ABSENT means "outputMaskOptional not given";
+ * otherwise bit 0 is outputMask[0] (y1) and bit 1 is outputMask[1] (y2). */
+#define ARNQ_MASK_ABSENT (-1)
+#define ARNQ_MASK_Y1 1
+#define ARNQ_MASK_Y2 2
+
+/* Largest supported row length n (elements). */
+#define ARNQ_MAX_N 131072
+
+/* Human-readable name of a status code (static storage; never NULL). */
+ARNQ_API const char *arnq_status_string(arnq_status s);
+
+/* Which outputs a call produces ("aclnnAddRmsNormDynamicQuantV2", Formula:
+ * the valid / invalid cases of scale1Out, y1Out, scale2Out, y2Out) and
+ * whether the combination is allowed (Constraints section):
+ *   y1/scale1 are produced  iff  mask absent, or mask[0];
+ *   y2/scale2 are produced  iff  mask[1], or (mask absent and both smooth
+ *                                 scales given);
+ *   ARNQ_ERR_MASK if the mask is given with smooth1 and !mask[0], or with
+ *   smooth2 and !mask[1], or with both entries false; or if the mask is absent
+ *   and smooth2 is given without smooth1.
+ * y1_on / y2_on may be NULL.  Host only; touches no device. */
+ARNQ_API arnq_status arnq_selected_outputs(int out_mask, int has_smooth1, int has_smooth2, int *y1_on,
+                                  int *y2_on);
+
+/* Workspace bytes arnq_run needs for this problem (first phase of the pages'
+ * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize").  The
+ * workspace holds a status block the kernels write only on error; the caller
+ * allocates it on the device, zero-fills it once, and may reuse it for any
+ * number of calls on one stream.  Validates the same arguments as arnq_run
+ * (except pointers).  Host only. */
+ARNQ_API arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdtype qdt,
+                                int out_mask, int has_smooth1, int has_smooth2, size_t *bytes);
+
+/* The fused operator ("aclnnAddRmsNormDynamicQuantV2", Formula).
+ *   x1, x2         [rows, n] dtype   required
+ *   gamma          [n] dtype         required
+ *   beta           [n] dtype         optional (NULL = no beta)
+ *   smooth1/2      [n] dtype         optional (NULL = not given)
+ *   eps            epsilon, finite and >= 0
+ *   out_mask       ARNQ_MASK_ABSENT or ARNQ_MASK_Y1 | ARNQ_MASK_Y2 bits
+ *   qdt            code type of y1 and y2
+ *   y1, scale1     written iff selected (see arnq_selected_outputs)
+ *   y2, scale2     written iff selected
+ *   x_out          [rows, n] dtype, optional (NULL = not written)
+ *   workspace      device buffer of at least arnq_workspace_size() bytes
+ *   stream         cudaStream_t (as void *) to launch on
+ * Returns ARNQ_OK once the work is enqueued; see the file header for errors. */
+ARNQ_API arnq_status arnq_run(const void *x1, const void *x2, const void *gamma, const void *beta,
+                     const void *smooth1, const void *smooth2, int64_t rows, int64_t n,
+                     arnq_dtype dt, float eps, int out_mask, arnq_qdtype qdt, void *y1,
+                     float *scale1, void *y2, float *scale2, void *x_out, void *workspace,
+                     size_t workspace_bytes, void *stream);
+
+/* The earlier interface "aclnnAddRmsNormDynamicQuant" (the V2 page: V2 adds
+ * betaOptional and outputMaskOptional to it): arnq_run with beta = NULL and
+ * the mask absent. */
+ARNQ_API arnq_status arnq_run_v1(const void *x1, const void *x2, const void *gamma, const void *smooth1,
+                        const void *smooth2, int64_t rows, int64_t n, arnq_dtype dt, float eps,
+                        arnq_qdtype qdt, void *y1, float *scale1, void *y2, float *scale2,
+                        void *x_out, void *workspace, size_t workspace_bytes, void *stream);
+
+/* The no-add operator ("aclnnRmsNormDynamicQuant", formula section): x is
+ * normalised as given, one optional smooth scale, one output.
+ *   x [rows, n] dtype; gamma [n]; beta, smooth [n] optional;
+ *   y [rows, n] int8 or [rows, n/2] packed INT4; scale [rows] binary32. */
+ARNQ_API arnq_status arnq_rms_norm_dynamic_quant(const void *x, const void *gamma, const void *beta,
+                                        const void *smooth, int64_t rows, int64_t n,
+                                        arnq_dtype dt, float eps, arnq_qdtype qdt, void *y,
+                                        float *scale, void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
+/* Status block at the start of the workspace.  code is 0 (ARNQ_OK) until a
+ * kernel records an error; the library never clears it.  row is the first
+ * row the failing kernel did not finish.  Read it with a device-to-host copy
+ * after synchronizing the stream; zero it to re-arm. */
+typedef struct arnq_workspace_status {
+  int32_t code;
+  int32_t reserved;
+  int64_t row;
+} arnq_workspace_status;
+
+/* ---- launch plans (tuning and testing) --------------------------------- */
+
+typedef enum arnq_kernel {
+  ARNQ_KERNEL_AUTO = 0,    /* let the library choose                                   */
+  ARNQ_KERNEL_DIRECT = 1,  /* rows loaded straight into registers (any alignment)      */
+  ARNQ_KERNEL_STAGED = 2   /* rows staged in shared memory by bulk async copies        */
+} arnq_kernel;
+
+/* How a call is launched.  Zero fields mean "choose".  Every plan computes
+ * the same operator; plans may differ in the last bits of the scales and, at
+ * rare rounding ties, by one in a code, because the fp32 reduction tree
+ * follows the plan.  One plan always gives the same bits. */
+typedef struct arnq_plan {
+  int32_t kernel;        /* arnq_kernel                                        */
+  int32_t cluster;       /* CTAs sharing one row: 1, 2, 4, 8 or 16             */
+  int32_t threads;       /* threads per CTA (multiple of 32, <= 1024)          */
+  int32_t units;         /* units per thread: 1, 2 (16-byte units) or 1..8 (pairs) */
+  int32_t stages;        /* staged kernel: rows in flight per CTA              */
+  int32_t ctas_per_sm;   /* resident CTAs per SM the grid is sized for         */
+  int32_t grid;          /* CTAs launched (output; multiple of cluster)        */
+  int32_t vector;        /* output: 1 if 16-byte vector loads are used         */
+} arnq_plan;
+
+/* Fills *plan with the plan arnq_run would use for these arguments (pointers
+ * are only inspected for alignment).  Fields of *plan that are nonzero on
+ * entry are kept as requested.  Queries the current device. */
+ARNQ_API arnq_status arnq_make_plan(const void *x1, const void *x2, const void *gamma, const void *beta,
+                           const void *smooth1, const void *smooth2, int64_t rows, int64_t n,
+                           arnq_dtype dt, int out_mask, arnq_qdtype qdt, const void *y1,
+                           const void *y2, const void *x_out, arnq_plan *plan);
+
+/* arnq_run with an explicit plan (from arnq_make_plan, possibly edited).
+ * ARNQ_ERR_PLAN if the plan cannot run this problem. */
+ARNQ_API arnq_status arnq_run_planned(const void *x1, const void *x2, const void *gamma,
+                             const void *beta, const void *smooth1, const void *smooth2,
+                             int64_t rows, int64_t n, arnq_dtype dt, float eps, int out_mask,
+                             arnq_qdtype qdt, void *y1, float *scale1, void *y2, float *scale2,
+                             void *x_out, void *workspace, size_t workspace_bytes, void *stream,
+                             const arnq_plan *plan);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ARNQ_H */

@@ -1,0 +1,371 @@
+"""GPU parity: the CUDA path (called through the C ABI) against the CPU oracle,
+element by element, on the same seeded inputs.
+
+Acceptance (the operator's stated tolerance): xOut bit-exact; INT4 packing
+bit-exact (codes are compared after unpacking both sides with the same
+reader, and hand-worked rows compare raw bytes); scales within relative 1e-5;
+codes within +-1 with at most 1e-4 of them off by one.  Every run also checks
+that the workspace status block stayed clear and that outputs the call must
+not write kept their canary bytes.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from int4_quant_b200 import _abi as A
+from int4_quant_b200 import build as B
+from int4_quant_b200 import workloads as wl
+from tests._util import codes, golden
+
+pytestmark = pytest.mark.gpu
+
+SCALE_RTOL = 1e-5
+OFF_BY_ONE_RATE = 1e-4
+CANARY = 0xA5
+
+DT = {"bf16": A.ARNQ_BF16, "fp16": A.ARNQ_FP16}
+QDT = {"int8": A.ARNQ_INT8, "int4": A.ARNQ_INT4}
+TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    B.build()
+    A.lib()
+    torch.cuda.set_device(0)
+
+
+def dev_bits(bits, dtype, offset=0):
+    """uint16 bit patterns -> CUDA tensor of the 16-bit dtype; with offset > 0
+    the tensor starts `offset` elements into a larger buffer (misaligned)."""
+    if bits is None:
+        return None
+    flat = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16).ravel())
+    buf = torch.empty(flat.numel() + offset, dtype=torch.int16, device="cuda")
+    buf[offset:].copy_(flat)
+    return buf[offset:].view(TDT[dtype]).view(bits.shape)
+
+
+def canary_bytes(nbytes, offset=0):
+    buf = torch.full((nbytes + offset,), CANARY, dtype=torch.uint8, device="cuda")
+    return buf[offset:]
+
+
+def run_gpu(w, plan=None, offset=0, inplace=False, mask="use", smooth="use", stream=None):
+    """Runs arnq_run (or arnq_run_planned) on workload w; returns numpy outputs."""
+    rows, n = w.rows, w.n
+    m = w.mask if mask == "use" else mask
+    s1 = w.smooth1 if smooth == "use" else smooth[0]
+    s2 = w.smooth2 if smooth == "use" else smooth[1]
+    mc = oracle.mask_code(m)
+    x1 = dev_bits(w.x1, w.dtype, offset)
+    x2 = dev_bits(w.x2, w.dtype, offset)
+    g = dev_bits(w.gamma, w.dtype, offset)
+    b = dev_bits(w.beta, w.dtype, offset)
+    d1 = dev_bits(s1, w.dtype, offset)
+    d2 = dev_bits(s2, w.dtype, offset)
+    cb = n if w.qdtype == "int8" else n // 2
+    y1 = canary_bytes(rows * cb, offset)
+    y2 = canary_bytes(rows * cb, offset)
+    sc1 = canary_bytes(rows * 4).view(torch.float32)  # scales must be 4-byte aligned
+    sc2 = canary_bytes(rows * 4).view(torch.float32)
+    xo = x1 if inplace else canary_bytes(rows * n * 2, 2 * offset).view(torch.int16)
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    args = (x1, x2, g, b, d1, d2, rows, n, DT[w.dtype], w.eps, mc, QDT[w.qdtype], y1, sc1, y2,
+            sc2, xo, ws, 256, stream)
+    if plan is None:
+        st = A.arnq_run(*args)
+    else:
+        st = A.arnq_run_planned(*args, plan)
+    assert st == A.ARNQ_OK, A.arnq_status_string(st)
+    torch.cuda.synchronize()
+    wsh = ws[:16].cpu().numpy().view(np.int32)
+    assert wsh[0] == 0, f"device status {wsh[0]}"
+    out = {
+        "y1": y1.cpu().numpy().reshape(rows, cb),
+        "y2": y2.cpu().numpy().reshape(rows, cb),
+        "scale1": sc1.cpu().numpy()[:rows].copy(),
+        "scale2": sc2.cpu().numpy()[:rows].copy(),
+        "x_out": xo.contiguous().view(torch.int16).cpu().numpy().view(np.uint16).reshape(rows, n),
+    }
+    return out, mc
+
+
+def run_oracle(w, mask="use", smooth="use"):
+    m = w.mask if mask == "use" else mask
+    s1 = w.smooth1 if smooth == "use" else smooth[0]
+    s2 = w.smooth2 if smooth == "use" else smooth[1]
+    r = oracle.add_rms_norm_dynamic_quant_v2(w.x1, w.x2, w.gamma, w.beta, s1, s2, eps=w.eps,
+                                             mask=m, qdtype=w.qdtype, dtype=w.dtype)
+    assert r["status"] == oracle.ORC_OK and r["clamp_hits"] == 0
+    return r
+
+
+def compare(g, o, qdtype, label="", xout=True):
+    """Asserts parity of one GPU run `g` with oracle result `o`; returns stats."""
+    stats = {}
+    if xout:
+        assert np.array_equal(g["x_out"], o["x_out"]), f"{label}: xOut not bit-exact"
+    for k in ("1", "2"):
+        if o["y" + k] is None:
+            # not selected: must still hold the canary
+            assert (g["y" + k] == CANARY).all(), f"{label}: y{k} written though not selected"
+            assert (g["scale" + k].view(np.uint8) == CANARY).all(), f"{label}: scale{k} written"
+            continue
+        gs, os_ = g["scale" + k].astype(np.float64), o["scale" + k].astype(np.float64)
+        zero = os_ == 0
+        assert np.array_equal(gs[zero], os_[zero]), f"{label}: zero scales differ"
+        rel = np.abs(gs[~zero] / os_[~zero] - 1.0) if (~zero).any() else np.zeros(1)
+        assert rel.max() <= SCALE_RTOL, f"{label}: scale{k} rel err {rel.max():.3g}"
+        qg = codes(g["y" + k], qdtype).astype(np.int32)
+        qo = codes(o["y" + k], qdtype).astype(np.int32)
+        d = np.abs(qg - qo)
+        assert d.max() <= 1, f"{label}: y{k} code off by {d.max()}"
+        rate = float((d == 1).mean())
+        allowed = int(np.floor(OFF_BY_ONE_RATE * d.size))
+        assert int((d == 1).sum()) <= allowed, f"{label}: y{k} off-by-one rate {rate:.3g}"
+        stats["y" + k] = dict(off_by_one=int((d == 1).sum()), rate=rate,
+                              scale_rel_max=float(rel.max()))
+    return stats
+
+
+# ------------------------------------------------------------------ full-size configurations
+
+@pytest.mark.parametrize("cfg", list(wl.CONFIGS))
+def test_config_full_size(cfg):
+    w = wl.CONFIGS[cfg]()
+    g, _ = run_gpu(w)
+    o = run_oracle(w)
+    stats = compare(g, o, w.qdtype, cfg)
+    print(cfg, stats)
+
+
+# ------------------------------------------------------------------ hand-worked rows
+
+@pytest.mark.parametrize("case", golden("tie_rows.json")["cases"], ids=lambda c: c["name"])
+def test_hand_worked_rows_on_gpu(case):
+    dt = case["dtype"]
+    bits = lambda v: wl.to_bits(np.asarray(v, np.float32), dt)  # noqa: E731
+    w = wl.Workload(name=case["name"], rows=1, n=len(case["x1"]), dtype=dt,
+                    qdtype=case["qdtype"], eps=case["eps"], mask=None, x1=bits([case["x1"]]),
+                    x2=bits([case["x2"]]), gamma=bits(case["gamma"]),
+                    beta=bits(case["beta"]) if "beta" in case else None)
+    g, _ = run_gpu(w)
+    o = run_oracle(w)
+    assert np.array_equal(g["x_out"][0], bits(case["expect_x_out"]))
+    if "gpu_tolerance" in case:
+        # binary32 cannot resolve a quotient this close to a tie: +-1 allowed here
+        assert g["scale1"][0] == o["scale1"][0]
+        d = np.abs(codes(g["y1"], w.qdtype).astype(int) - codes(o["y1"], w.qdtype).astype(int))
+        assert d.max() <= 1
+        return
+    # every intermediate is exact: bit-exact scale and codes
+    assert g["scale1"][0] == o["scale1"][0]
+    assert np.array_equal(g["y1"], o["y1"].view(np.uint8))
+
+
+# ------------------------------------------------------------------ output selection
+
+MASK_CASES = [(tuple(m) if m is not None else None, s1, s2)
+              for m, s1, s2, ok, _, _ in golden("mask_truth_table.json")["rows"] if ok]
+
+
+@pytest.mark.parametrize("mask,h1,h2", MASK_CASES)
+@pytest.mark.parametrize("qdtype", ["int8", "int4"])
+def test_mask_truth_table_on_gpu(mask, h1, h2, qdtype):
+    w = wl.random_case(37, 264, seed=17, qdtype=qdtype, beta=True, smooth1=True, smooth2=True)
+    sm = (w.smooth1 if h1 else None, w.smooth2 if h2 else None)
+    g, _ = run_gpu(w, mask=mask, smooth=sm)
+    o = run_oracle(w, mask=mask, smooth=sm)
+    compare(g, o, qdtype, f"mask={mask} s1={h1} s2={h2}")
+
+
+# ------------------------------------------------------------------ every launch plan
+
+def plan(**kw):
+    p = A.arnq_plan()
+    for k, v in kw.items():
+        setattr(p, k, v)
+    return p
+
+
+PLAN_CASES = [
+    dict(kernel=A.ARNQ_KERNEL_DIRECT),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, units=2),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=2),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=16),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=2, units=2),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=3, cluster=4),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=2, cluster=8, units=2),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=4, cluster=16),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=5, ctas_per_sm=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=2, ctas_per_sm=1, threads=1024),
+]
+
+
+@pytest.mark.parametrize("pk", PLAN_CASES, ids=lambda d: "-".join(f"{k}{v}" for k, v in d.items()))
+@pytest.mark.parametrize("shape", [(300, 4096, "bf16", "int8"), (97, 7168, "bf16", "int8"),
+                                   (211, 5120, "fp16", "int4"), (19, 16384, "bf16", "int4")])
+def test_plans(pk, shape):
+    rows, n, dt, qdt = shape
+    w = wl.random_case(rows, n, dtype=dt, qdtype=qdt, seed=rows + n, beta=True, smooth1=True,
+                       smooth2=True, mask=(True, True), outlier_frac=0.01)
+    p = plan(**pk)
+    g, _ = run_gpu(w, plan=p)
+    o = run_oracle(w)
+    compare(g, o, qdt, str(pk))
+
+
+@pytest.mark.parametrize("units", [1, 2, 4, 8])
+@pytest.mark.parametrize("cluster", [1, 4])
+def test_scalar_plans(units, cluster):
+    # n not a multiple of 8 forces 2-element units
+    w = wl.random_case(53, 3002, seed=units * 10 + cluster, beta=True, smooth1=True)
+    g, _ = run_gpu(w, plan=plan(kernel=A.ARNQ_KERNEL_DIRECT, units=units, cluster=cluster))
+    compare(g, run_oracle(w), "int8", f"scalar u{units} c{cluster}")
+
+
+def test_bad_plans_are_rejected():
+    w = wl.random_case(8, 1000, seed=1)
+    x = dev_bits(w.x1, "bf16")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    y = torch.empty(8 * 1000, dtype=torch.int8, device="cuda")
+    s = torch.empty(8, dtype=torch.float32, device="cuda")
+    gm = dev_bits(w.gamma, "bf16")
+    for bad in (dict(kernel=A.ARNQ_KERNEL_STAGED),   # n % 8 != 0 cannot be staged
+                dict(cluster=3), dict(threads=100), dict(units=3), dict(kernel=9),
+                dict(threads=32, units=1)):
+        st = A.arnq_run_planned(x, x, gm, None, None, None, 8, 1000, 0, 1e-6, -1, 0, y, s, None,
+                                None, None, ws, 256, None, plan(**bad))
+        assert st == A.ARNQ_ERR_PLAN, bad
+
+
+# ------------------------------------------------------------------ ragged, misaligned, edges
+
+@pytest.mark.parametrize("rows,n,dt,qdt", [
+    (1, 1, "bf16", "int8"), (1, 2, "fp16", "int4"), (3, 8, "bf16", "int4"), (5, 24, "fp16", "int8"),
+    (37, 1000, "bf16", "int8"), (37, 1000, "fp16", "int4"), (41, 1032, "bf16", "int8"),
+    (17, 4104, "fp16", "int8"), (9, 8200, "bf16", "int4"), (2, 65538, "bf16", "int8"),
+    (3, 131072, "bf16", "int8"), (2, 131072, "fp16", "int4"), (1000, 64, "bf16", "int8"),
+    (4097, 128, "fp16", "int4"),
+])
+def test_ragged_shapes(rows, n, dt, qdt):
+    w = wl.random_case(rows, n, dtype=dt, qdtype=qdt, seed=rows * 7 + n, beta=True, smooth1=True)
+    g, _ = run_gpu(w)
+    compare(g, run_oracle(w), qdt, f"{rows}x{n}")
+
+
+@pytest.mark.parametrize("offset", [1, 3])
+@pytest.mark.parametrize("qdt", ["int8", "int4"])
+def test_misaligned_pointers_use_the_scalar_path(offset, qdt):
+    w = wl.random_case(29, 2048, seed=offset, qdtype=qdt, beta=True, smooth1=True,
+                       smooth2=True, mask=(True, True))
+    g, _ = run_gpu(w, offset=offset)
+    compare(g, run_oracle(w), qdt, f"offset {offset}")
+
+
+def test_in_place_residual_update():
+    w = wl.random_case(300, 4096, seed=5, beta=True, smooth1=True, mask=(True, False))
+    g, _ = run_gpu(w, inplace=True)
+    compare(g, run_oracle(w), "int8", "in place")
+
+
+def test_deterministic_rerun():
+    w = wl.random_case(2048, 4096, seed=1, x_sigma=(1.0, 0.5), beta=True, smooth1=True,
+                       mask=(True, False))
+    a, _ = run_gpu(w)
+    b, _ = run_gpu(w)
+    for k in ("y1", "scale1", "x_out"):
+        assert np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)), k
+
+
+def test_zero_and_constant_rows():
+    n = 4096
+    x1 = np.zeros((4, n), np.float32)
+    x1[1] = 0.75
+    x1[2, 123] = 3.0
+    x1[3] = -2.0
+    w = wl.Workload(name="special", rows=4, n=n, dtype="bf16", qdtype="int8", eps=1e-6,
+                    mask=None, x1=wl.to_bits(x1, "bf16"), x2=wl.to_bits(np.zeros_like(x1), "bf16"),
+                    gamma=wl.to_bits(np.ones(n, np.float32), "bf16"))
+    g, _ = run_gpu(w)
+    o = run_oracle(w)
+    compare(g, o, "int8", "special rows")
+    assert g["scale1"][0] == 0.0 and not g["y1"][0].any()
+    assert (g["y1"][1].view(np.int8) == 127).all() and (g["y1"][3].view(np.int8) == -127).all()
+    q2 = g["y1"][2].view(np.int8)
+    assert q2[123] == 127 and np.count_nonzero(q2) == 1
+
+
+# ------------------------------------------------------------------ the other entry points
+
+@pytest.mark.parametrize("dt,qdt", [("bf16", "int8"), ("fp16", "int4")])
+@pytest.mark.parametrize("smooth", [False, True])
+def test_rms_norm_dynamic_quant_no_add(dt, qdt, smooth):
+    w = wl.random_case(333, 2560, dtype=dt, qdtype=qdt, seed=3, beta=True, smooth1=smooth)
+    x = dev_bits(w.x1, dt)
+    cb = w.n if qdt == "int8" else w.n // 2
+    y = torch.empty(w.rows * cb, dtype=torch.uint8, device="cuda")
+    s = torch.empty(w.rows, dtype=torch.float32, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    st = A.arnq_rms_norm_dynamic_quant(x, dev_bits(w.gamma, dt), dev_bits(w.beta, dt),
+                                       dev_bits(w.smooth1, dt), w.rows, w.n, DT[dt], w.eps,
+                                       QDT[qdt], y, s, ws, 256, None)
+    assert st == A.ARNQ_OK
+    torch.cuda.synchronize()
+    o = oracle.rms_norm_dynamic_quant(w.x1, w.gamma, w.beta, w.smooth1, eps=w.eps, qdtype=qdt,
+                                      dtype=dt)
+    g = {"y1": y.cpu().numpy().reshape(w.rows, cb), "scale1": s.cpu().numpy()}
+    oo = {"y1": o["y"], "scale1": o["scale"], "y2": None}
+    g["y2"] = np.full_like(g["y1"], CANARY)  # the single-output call has no y2
+    g["scale2"] = np.full(w.rows * 4, CANARY, np.uint8).view(np.float32)
+    compare(g, oo, qdt, "no-add", xout=False)
+
+
+def test_v1_entry_point():
+    w = wl.random_case(100, 3072, seed=8, smooth1=True, smooth2=True)
+    dt = "bf16"
+    x1, x2 = dev_bits(w.x1, dt), dev_bits(w.x2, dt)
+    y1 = torch.empty(w.rows * w.n, dtype=torch.uint8, device="cuda")
+    y2 = torch.empty(w.rows * w.n, dtype=torch.uint8, device="cuda")
+    s1 = torch.empty(w.rows, dtype=torch.float32, device="cuda")
+    s2 = torch.empty(w.rows, dtype=torch.float32, device="cuda")
+    xo = torch.empty(w.rows * w.n, dtype=torch.int16, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    st = A.arnq_run_v1(x1, x2, dev_bits(w.gamma, dt), dev_bits(w.smooth1, dt),
+                       dev_bits(w.smooth2, dt), w.rows, w.n, A.ARNQ_BF16, w.eps, A.ARNQ_INT8, y1,
+                       s1, y2, s2, xo, ws, 256, None)
+    assert st == A.ARNQ_OK
+    torch.cuda.synchronize()
+    o = oracle.add_rms_norm_dynamic_quant_v2(w.x1, w.x2, w.gamma, None, w.smooth1, w.smooth2,
+                                             eps=w.eps, mask=None)
+    g = {"x_out": xo.cpu().numpy().view(np.uint16).reshape(w.rows, w.n),
+         "y1": y1.cpu().numpy().reshape(w.rows, w.n), "scale1": s1.cpu().numpy(),
+         "y2": y2.cpu().numpy().reshape(w.rows, w.n), "scale2": s2.cpu().numpy()}
+    compare(g, o, "int8", "v1")
+
+
+def test_torch_facing_call_matches_the_abi():
+    import int4_quant_b200 as q
+    w = wl.random_case(64, 1024, seed=0)
+    x1 = dev_bits(w.x1, "bf16")
+    x2 = dev_bits(w.x2, "bf16")
+    y1, s1, y2, s2, xo = q.add_rms_norm_dynamic_quant(x1, x2, dev_bits(w.gamma, "bf16"),
+                                                      eps=w.eps)
+    assert y2 is None and s2 is None
+    torch.cuda.synchronize()
+    g, _ = run_gpu(w)
+    assert np.array_equal(y1.cpu().numpy().view(np.uint8), g["y1"])
+    assert np.array_equal(s1.cpu().numpy(), g["scale1"])
+    assert np.array_equal(xo.view(torch.int16).cpu().numpy().view(np.uint16), g["x_out"])
+
+
+def test_non_default_stream():
+    w = wl.random_case(500, 2048, seed=12, beta=True, smooth1=True)
+    s = torch.cuda.Stream()
+    g, _ = run_gpu(w, stream=s)
+    compare(g, run_oracle(w), "int8", "side stream")
