@@ -18,37 +18,44 @@ namespace {
 using arnq::KParams;
 typedef void (*KernelFn)(KParams);
 
-constexpr int kHeaderSmem = 16 * 32 * 12 + 128 + 8 * 16;  // slots, abort flag, mbarriers
-constexpr size_t kWorkspaceBytes = 256;                     // status block, padded
-constexpr int kMaxStages = 16;
+constexpr int kHeaderSmem = arnq::kRingOff;  // reduction slots, abort flag, mbarriers
+constexpr size_t kWorkspaceBytes = 256;      // status block, padded
+constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
+constexpr int kMaxSegElems = 8192;           // elements of a row one CTA holds in registers
 
 // ---------------------------------------------------------------- kernel table
 
-constexpr int kUptSlots = 4;  // units per thread 1, 2, 4, 8
-int upt_slot(int upt) { return upt == 1 ? 0 : upt == 2 ? 1 : upt == 4 ? 2 : upt == 8 ? 3 : -1; }
+// units per thread: 16-byte units 1 or 2; element pairs 1, 4 or 8
+constexpr int kUptSlots = 3;
+int upt_slot(int mode, int upt) {
+  if (mode == arnq::LOAD_SCALAR) return upt == 1 ? 0 : upt == 4 ? 1 : upt == 8 ? 2 : -1;
+  return upt == 1 ? 0 : upt == 2 ? 1 : -1;
+}
 
-template <class T, bool I4, int M>
-void fill_mode(KernelFn *t) {
-  t[0] = arnq::rows_kernel<T, I4, M, 1>;
-  t[1] = arnq::rows_kernel<T, I4, M, 2>;
-  if (M == arnq::LOAD_SCALAR) {
-    t[2] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 4>;
-    t[3] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 8>;
-  } else {
-    t[2] = t[3] = nullptr;  // vector units: at most 2 per thread (register budget)
-  }
+template <class T, bool I4, int NOUT, bool ADD>
+void fill(KernelFn *t) {
+  t[0 * kUptSlots + 0] = arnq::rows_kernel<T, I4, arnq::LOAD_VEC, 1, NOUT, ADD>;
+  t[0 * kUptSlots + 1] = arnq::rows_kernel<T, I4, arnq::LOAD_VEC, 2, NOUT, ADD>;
+  t[0 * kUptSlots + 2] = nullptr;
+  t[1 * kUptSlots + 0] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 1, NOUT, ADD>;
+  t[1 * kUptSlots + 1] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 4, NOUT, ADD>;
+  t[1 * kUptSlots + 2] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 8, NOUT, ADD>;
+  t[2 * kUptSlots + 0] = arnq::rows_kernel<T, I4, arnq::LOAD_STAGED, 1, NOUT, ADD>;
+  t[2 * kUptSlots + 1] = arnq::rows_kernel<T, I4, arnq::LOAD_STAGED, 2, NOUT, ADD>;
+  t[2 * kUptSlots + 2] = nullptr;
 }
 
 template <class T, bool I4>
-void fill_q(KernelFn *t) {
-  fill_mode<T, I4, arnq::LOAD_VEC>(t + 0 * kUptSlots);
-  fill_mode<T, I4, arnq::LOAD_SCALAR>(t + 1 * kUptSlots);
-  fill_mode<T, I4, arnq::LOAD_STAGED>(t + 2 * kUptSlots);
+void fill_q(KernelFn (*t)[2][3 * kUptSlots]) {
+  fill<T, I4, 1, false>(t[0][0]);
+  fill<T, I4, 1, true>(t[0][1]);
+  fill<T, I4, 2, false>(t[1][0]);
+  fill<T, I4, 2, true>(t[1][1]);
 }
 
 struct KernelTable {
-  KernelFn fn[2][2][3 * kUptSlots];
+  KernelFn fn[2][2][2][2][3 * kUptSlots];  // [dtype][qdtype][nout-1][add][mode*slots+upt]
   KernelTable() {
     fill_q<arnq::Bf16, false>(fn[0][0]);
     fill_q<arnq::Bf16, true>(fn[0][1]);
@@ -57,11 +64,17 @@ struct KernelTable {
   }
 };
 
-KernelFn lookup(int dt, int qdt, int mode, int upt) {
+KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt) {
   static const KernelTable table;
-  const int s = upt_slot(upt);
-  if (s < 0) return nullptr;
-  return table.fn[dt][qdt][mode * kUptSlots + s];
+  const int s = upt_slot(mode, upt);
+  if (s < 0 || nout < 1 || nout > 2) return nullptr;
+  return table.fn[dt][qdt][nout - 1][add ? 1 : 0][mode * kUptSlots + s];
+}
+
+// mirrors arnq::MaxThreads
+int max_threads(int mode, int upt, int nout) {
+  const int elems = upt * (mode == arnq::LOAD_SCALAR ? 2 : 8);
+  return elems <= 8 ? (nout == 1 ? 1024 : 768) : 512;
 }
 
 // ---------------------------------------------------------------- device info
@@ -138,7 +151,8 @@ struct Problem {
   int64_t rows, n;
   int dt, qdt;
   float eps;
-  int flags;
+  bool add;       // x = x1 + x2 (else x = x1: the no-add operator)
+  bool on1, on2;  // selected outputs
 };
 
 arnq_status selected(int out_mask, int has_s1, int has_s2, int *on1, int *on2) {
@@ -170,68 +184,67 @@ arnq_status check_shape(int64_t rows, int64_t n, int dt, int qdt, float eps) {
   return ARNQ_OK;
 }
 
-// Validates a problem; `has_add` false for the no-add operator (x2 unused).
-arnq_status validate(const Problem &P, bool has_add, int out_mask, const void *workspace,
-                     size_t workspace_bytes, int *flags_out) {
+// Decides the selected outputs and drops the pointers of the others.
+arnq_status select_outputs(Problem &P, int out_mask) {
+  int on1 = 0, on2 = 0;
+  arnq_status st = selected(out_mask, P.s1 != nullptr, P.s2 != nullptr, &on1, &on2);
+  if (st != ARNQ_OK) return st;
+  P.on1 = on1 != 0;
+  P.on2 = on2 != 0;
+  if (!P.on1) { P.y1 = nullptr; P.scale1 = nullptr; }
+  if (!P.on2) { P.y2 = nullptr; P.scale2 = nullptr; }
+  if (!P.add) { P.x2 = nullptr; P.x_out = nullptr; }
+  return ARNQ_OK;
+}
+
+arnq_status validate(Problem &P, int out_mask, const void *workspace, size_t workspace_bytes) {
   arnq_status st = check_shape(P.rows, P.n, P.dt, P.qdt, P.eps);
   if (st != ARNQ_OK) return st;
-  int on1 = 0, on2 = 0;
-  st = selected(out_mask, P.s1 != nullptr, P.s2 != nullptr, &on1, &on2);
+  st = select_outputs(P, out_mask);
   if (st != ARNQ_OK) return st;
-  if (!P.x1 || (has_add && !P.x2) || !P.gamma) return ARNQ_ERR_NULL_PTR;
-  if (on1 && (!P.y1 || !P.scale1)) return ARNQ_ERR_NULL_PTR;
-  if (on2 && (!P.y2 || !P.scale2)) return ARNQ_ERR_NULL_PTR;
-  const void *h16[] = {P.x1, has_add ? P.x2 : nullptr, P.gamma, P.beta, P.s1, P.s2, P.x_out};
+  if (!P.x1 || (P.add && !P.x2) || !P.gamma) return ARNQ_ERR_NULL_PTR;
+  if (P.on1 && (!P.y1 || !P.scale1)) return ARNQ_ERR_NULL_PTR;
+  if (P.on2 && (!P.y2 || !P.scale2)) return ARNQ_ERR_NULL_PTR;
+  const void *h16[] = {P.x1, P.x2, P.gamma, P.beta, P.s1, P.s2, P.x_out};
   for (const void *q : h16)
     if (q && !aligned(q, 2)) return ARNQ_ERR_ALIGN;
-  if ((on1 && !aligned(P.scale1, 4)) || (on2 && !aligned(P.scale2, 4))) return ARNQ_ERR_ALIGN;
+  if ((P.on1 && !aligned(P.scale1, 4)) || (P.on2 && !aligned(P.scale2, 4))) return ARNQ_ERR_ALIGN;
   if (!workspace || workspace_bytes < kWorkspaceBytes) return ARNQ_ERR_WORKSPACE;
   if (!aligned(workspace, 8)) return ARNQ_ERR_ALIGN;
-  int f = 0;
-  if (has_add) f |= arnq::F_X2;
-  if (P.beta) f |= arnq::F_BETA;
-  if (P.s1) f |= arnq::F_S1;
-  if (P.s2) f |= arnq::F_S2;
-  if (on1) f |= arnq::F_OUT1;
-  if (on2) f |= arnq::F_OUT2;
-  if (has_add && P.x_out) f |= arnq::F_XOUT;
-  *flags_out = f;
   return ARNQ_OK;
 }
 
 // ---------------------------------------------------------------- planning
 
 int round_up(int v, int m) { return (v + m - 1) / m * m; }
-int max_threads(int mode, int upt) {
-  return upt * (mode == arnq::LOAD_SCALAR ? 2 : 8) <= 8 ? 1024 : 512;
-}
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
+// 16-byte units need every 16-bit tensor 16-byte aligned with n % 8 == 0 (so
+// each row starts aligned), and the code outputs aligned to their 8 (INT8) or
+// 4 (INT4) bytes per unit.
 bool vector_ok(const Problem &P) {
   if (P.n % 8 != 0) return false;
-  const bool x2 = (P.flags & arnq::F_X2) != 0;
-  const void *v16[] = {P.x1, x2 ? P.x2 : nullptr, P.gamma, P.beta, P.s1, P.s2,
-                       (P.flags & arnq::F_XOUT) ? P.x_out : nullptr};
+  const void *v16[] = {P.x1, P.x2, P.gamma, P.beta, P.s1, P.s2, P.x_out};
   for (const void *q : v16)
     if (q && !aligned(q, 16)) return false;
   const uintptr_t ya = (P.qdt == ARNQ_INT8) ? 8 : 4;
-  if ((P.flags & arnq::F_OUT1) && !aligned(P.y1, ya)) return false;
-  if ((P.flags & arnq::F_OUT2) && !aligned(P.y2, ya)) return false;
+  if (P.on1 && !aligned(P.y1, ya)) return false;
+  if (P.on2 && !aligned(P.y2, ya)) return false;
   return true;
 }
 
-int stage_smem(const arnq_plan &pl, int seg_units, bool x2) {
-  return kHeaderSmem + pl.stages * seg_units * 16 * (x2 ? 2 : 1);
-}
+struct Launch {
+  KernelFn fn;
+  int smem, seg, units;
+};
 
-arnq_status make_plan(const Problem &P, arnq_plan *pl, KernelFn *fn_out, int *smem_out,
-                      int *seg_out, int *units_out) {
+arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   DeviceInfo di;
   int dev = 0;
   arnq_status st = device_info(&di, &dev);
   if (st != ARNQ_OK) return st;
   const bool vec = vector_ok(P);
-  const bool x2 = (P.flags & arnq::F_X2) != 0;
+  const int nout = (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0);
   if (pl->kernel == ARNQ_KERNEL_AUTO) pl->kernel = vec ? ARNQ_KERNEL_STAGED : ARNQ_KERNEL_DIRECT;
   if (pl->kernel == ARNQ_KERNEL_STAGED && !vec) return ARNQ_ERR_PLAN;
   if (pl->kernel != ARNQ_KERNEL_DIRECT && pl->kernel != ARNQ_KERNEL_STAGED) return ARNQ_ERR_PLAN;
@@ -241,12 +254,10 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, KernelFn *fn_out, int *sm
   pl->vector = (mode != arnq::LOAD_SCALAR) ? 1 : 0;
   const int U = (mode == arnq::LOAD_SCALAR) ? 2 : 8;
   const int units = static_cast<int>(ceil_div(P.n, U));
-  const int max_upt = (mode == arnq::LOAD_SCALAR) ? 8 : 2;
+  const int max_seg = kMaxSegElems / U;
 
-  // cluster: enough CTAs per row that one CTA's slice fits, then spread rows
-  // that are too few to fill the SMs over more CTAs
-  // a CTA holds at most 8192 elements of a row in registers (see MaxThreads)
-  const int max_seg = 8192 / U;
+  // cluster: enough CTAs per row that one CTA's slice fits in registers, then
+  // more CTAs per row while the rows are too few to fill the SMs
   if (pl->cluster == 0) {
     int cl = 1;
     while (cl < kMaxCluster && ceil_div(units, cl) > max_seg) cl *= 2;
@@ -256,49 +267,63 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, KernelFn *fn_out, int *sm
   const int cl = pl->cluster;
   if (cl != 1 && cl != 2 && cl != 4 && cl != 8 && cl != 16) return ARNQ_ERR_PLAN;
   const int seg = static_cast<int>(ceil_div(units, cl));
-
   if (seg > max_seg) return ARNQ_ERR_PLAN;
+
   if (pl->units == 0) {
-    int upt = 1;
-    while (upt < max_upt && ceil_div(seg, upt) > max_threads(mode, upt)) upt *= 2;
-    while (upt < max_upt && ceil_div(seg, upt) > 512 && U * upt * 2 <= 8) upt *= 2;
-    pl->units = upt;
+    if (mode == arnq::LOAD_SCALAR) {
+      pl->units = seg <= max_threads(mode, 1, nout) ? 1
+                  : seg <= 4 * max_threads(mode, 4, nout) ? 4 : 8;
+    } else {
+      pl->units = (seg >= 256 || seg > max_threads(mode, 1, nout)) ? 2 : 1;
+    }
   }
-  if (pl->units > max_upt || upt_slot(pl->units) < 0) return ARNQ_ERR_PLAN;
+  if (upt_slot(mode, pl->units) < 0) return ARNQ_ERR_PLAN;
   if (pl->threads == 0) {
     pl->threads = round_up(static_cast<int>(ceil_div(seg, pl->units)), 32);
     if (pl->threads < 32) pl->threads = 32;
   }
-  if (pl->threads % 32 != 0 || pl->threads > max_threads(mode, pl->units) ||
+  if (pl->threads % 32 != 0 || pl->threads > max_threads(mode, pl->units, nout) ||
       static_cast<int64_t>(pl->threads) * pl->units < seg)
     return ARNQ_ERR_PLAN;
 
-  KernelFn fn = lookup(P.dt, P.qdt, mode, pl->units);
+  KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units);
   if (!fn) return ARNQ_ERR_PLAN;
+  st = prepare_kernel(fn, dev, kHeaderSmem);
+  if (st != ARNQ_OK) return st;
+  int occ = 0;  // resident CTAs per SM allowed by threads and registers
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, pl->threads, kHeaderSmem) !=
+      cudaSuccess)
+    return ARNQ_ERR_CUDA;
+  if (occ < 1) return ARNQ_ERR_PLAN;
 
   int smem = kHeaderSmem;
   if (mode == arnq::LOAD_STAGED) {
-    if (pl->ctas_per_sm == 0) pl->ctas_per_sm = 2;
+    const int per_stage = seg * 16 * (P.add ? 2 : 1);
+    int ctas = pl->ctas_per_sm != 0 ? pl->ctas_per_sm : (occ < 4 ? occ : 4);
     if (pl->stages == 0) {
-      const int budget = di.smem_per_sm / pl->ctas_per_sm - 1024;  // 1 KB reserved per CTA
-      const int cap = budget < di.smem_per_block_optin ? budget : di.smem_per_block_optin;
-      const int per_stage = seg * 16 * (x2 ? 2 : 1);
-      int s = (cap - kHeaderSmem) / per_stage;
+      int s = 0;
+      while (true) {
+        int cap = di.smem_per_sm / ctas - 1024;  // 1 KB reserved per CTA
+        if (cap > di.smem_per_block_optin) cap = di.smem_per_block_optin;
+        s = (cap - kHeaderSmem) / per_stage;
+        if (s >= 2 || ctas == 1 || pl->ctas_per_sm != 0) break;
+        --ctas;
+      }
       if (s > kMaxStages) s = kMaxStages;
       if (s < 1) s = 1;
       pl->stages = s;
     }
+    pl->ctas_per_sm = ctas;
     if (pl->stages < 1 || pl->stages > kMaxStages) return ARNQ_ERR_PLAN;
-    smem = stage_smem(*pl, seg, x2);
+    smem = kHeaderSmem + pl->stages * per_stage;
     if (smem > di.smem_per_block_optin) return ARNQ_ERR_PLAN;
+    st = prepare_kernel(fn, dev, smem);
+    if (st != ARNQ_OK) return st;
   } else {
     pl->stages = 0;
   }
-  st = prepare_kernel(fn, dev, smem);
-  if (st != ARNQ_OK) return st;
 
   // grid: persistent, as many clusters as fit at once (or one per row)
-  int64_t clusters_needed = P.rows;
   int64_t clusters_fit = 0;
   if (cl == 1) {
     int per_sm = 0;
@@ -307,7 +332,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, KernelFn *fn_out, int *sm
       return ARNQ_ERR_CUDA;
     if (per_sm < 1) return ARNQ_ERR_PLAN;
     if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
-    if (pl->ctas_per_sm == 0) pl->ctas_per_sm = per_sm;
+    pl->ctas_per_sm = per_sm;
     clusters_fit = static_cast<int64_t>(per_sm) * di.sms;
   } else {
     cudaLaunchConfig_t cfg = {};
@@ -327,40 +352,48 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, KernelFn *fn_out, int *sm
     int64_t want = pl->ctas_per_sm != 0 ? static_cast<int64_t>(pl->ctas_per_sm) * di.sms / cl : nc;
     if (want < 1) want = 1;
     clusters_fit = want < nc ? want : nc;
-    if (pl->ctas_per_sm == 0) pl->ctas_per_sm = static_cast<int32_t>(ceil_div(nc * cl, di.sms));
+    pl->ctas_per_sm = static_cast<int32_t>(ceil_div(clusters_fit * cl, di.sms));
   }
-  const int64_t nclusters = clusters_needed < clusters_fit ? clusters_needed : clusters_fit;
+  const int64_t nclusters = P.rows < clusters_fit ? P.rows : clusters_fit;
   pl->grid = static_cast<int32_t>(nclusters * cl);
-  *fn_out = fn;
-  *smem_out = smem;
-  *seg_out = seg;
-  *units_out = units;
+  L->fn = fn;
+  L->smem = smem;
+  L->seg = seg;
+  L->units = units;
   return ARNQ_OK;
 }
 
 arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream_t stream) {
-  KernelFn fn = nullptr;
-  int smem = 0, seg = 0, units = 0;
-  arnq_status st = make_plan(P, &plan, &fn, &smem, &seg, &units);
+  Launch L;
+  arnq_status st = make_plan(P, &plan, &L);
   if (st != ARNQ_OK) return st;
   KParams k;
+  std::memset(&k, 0, sizeof k);
   k.x1 = static_cast<const uint16_t *>(P.x1);
   k.x2 = static_cast<const uint16_t *>(P.x2);
   k.gamma = static_cast<const uint16_t *>(P.gamma);
   k.beta = static_cast<const uint16_t *>(P.beta);
-  k.s1 = static_cast<const uint16_t *>(P.s1);
-  k.s2 = static_cast<const uint16_t *>(P.s2);
-  k.y1 = static_cast<uint8_t *>(P.y1);
-  k.y2 = static_cast<uint8_t *>(P.y2);
-  k.scale1 = P.scale1;
-  k.scale2 = P.scale2;
+  // output slots: the selected outputs in order, each with its own smooth scale
+  int slot = 0;
+  if (P.on1) {
+    k.smooth[slot] = static_cast<const uint16_t *>(P.s1);
+    k.y[slot] = static_cast<uint8_t *>(P.y1);
+    k.scale[slot] = P.scale1;
+    ++slot;
+  }
+  if (P.on2) {
+    k.smooth[slot] = static_cast<const uint16_t *>(P.s2);
+    k.y[slot] = static_cast<uint8_t *>(P.y2);
+    k.scale[slot] = P.scale2;
+    ++slot;
+  }
   k.x_out = static_cast<uint16_t *>(P.x_out);
   k.status = static_cast<int32_t *>(workspace);
   k.rows = P.rows;
   k.n = static_cast<int32_t>(P.n);
-  k.units = units;
-  k.seg_units = seg;
-  k.flags = P.flags;
+  k.units = L.units;
+  k.seg_units = L.seg;
+  k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0);
   k.stages = plan.stages;
   k.eps = P.eps;
 
@@ -368,7 +401,7 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(plan.grid, 1, 1);
   cfg.blockDim = dim3(plan.threads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   if (plan.cluster > 1) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -378,31 +411,26 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
     cfg.attrs = attr;
     cfg.numAttrs = 1;
   }
-  if (cudaLaunchKernelEx(&cfg, fn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
+  if (cudaLaunchKernelEx(&cfg, L.fn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
   return ARNQ_OK;
 }
 
 Problem problem(const void *x1, const void *x2, const void *gamma, const void *beta,
                 const void *s1, const void *s2, int64_t rows, int64_t n, arnq_dtype dt,
                 float eps, arnq_qdtype qdt, void *y1, float *scale1, void *y2, float *scale2,
-                void *x_out) {
+                void *x_out, bool add) {
   Problem P;
   P.x1 = x1; P.x2 = x2; P.gamma = gamma; P.beta = beta; P.s1 = s1; P.s2 = s2;
   P.y1 = y1; P.y2 = y2; P.x_out = x_out; P.scale1 = scale1; P.scale2 = scale2;
   P.rows = rows; P.n = n; P.dt = static_cast<int>(dt); P.qdt = static_cast<int>(qdt);
-  P.eps = eps; P.flags = 0;
+  P.eps = eps; P.add = add; P.on1 = P.on2 = false;
   return P;
 }
 
-arnq_status run_common(Problem P, bool has_add, int out_mask, void *workspace,
-                       size_t workspace_bytes, void *stream, const arnq_plan *plan) {
-  int flags = 0;
-  arnq_status st = validate(P, has_add, out_mask, workspace, workspace_bytes, &flags);
+arnq_status run_common(Problem P, int out_mask, void *workspace, size_t workspace_bytes,
+                       void *stream, const arnq_plan *plan) {
+  arnq_status st = validate(P, out_mask, workspace, workspace_bytes);
   if (st != ARNQ_OK) return st;
-  P.flags = flags;
-  if (!(flags & arnq::F_OUT1)) { P.y1 = nullptr; P.scale1 = nullptr; }
-  if (!(flags & arnq::F_OUT2)) { P.y2 = nullptr; P.scale2 = nullptr; }
-  if (!has_add) { P.x2 = nullptr; P.x_out = nullptr; }
   arnq_plan pl;
   std::memset(&pl, 0, sizeof pl);
   if (plan) pl = *plan;
@@ -455,8 +483,8 @@ arnq_status arnq_run(const void *x1, const void *x2, const void *gamma, const vo
                      float *scale1, void *y2, float *scale2, void *x_out, void *workspace,
                      size_t workspace_bytes, void *stream) {
   return run_common(problem(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, eps, qdt, y1,
-                            scale1, y2, scale2, x_out),
-                    true, out_mask, workspace, workspace_bytes, stream, nullptr);
+                            scale1, y2, scale2, x_out, true),
+                    out_mask, workspace, workspace_bytes, stream, nullptr);
 }
 
 arnq_status arnq_run_planned(const void *x1, const void *x2, const void *gamma,
@@ -467,8 +495,8 @@ arnq_status arnq_run_planned(const void *x1, const void *x2, const void *gamma,
                              const arnq_plan *plan) {
   if (!plan) return ARNQ_ERR_NULL_PTR;
   return run_common(problem(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, eps, qdt, y1,
-                            scale1, y2, scale2, x_out),
-                    true, out_mask, workspace, workspace_bytes, stream, plan);
+                            scale1, y2, scale2, x_out, true),
+                    out_mask, workspace, workspace_bytes, stream, plan);
 }
 
 arnq_status arnq_run_v1(const void *x1, const void *x2, const void *gamma, const void *smooth1,
@@ -486,8 +514,8 @@ arnq_status arnq_rms_norm_dynamic_quant(const void *x, const void *gamma, const 
                                         void *stream) {
   // one output, selected as with the mask absent and only smoothScale1 given
   return run_common(problem(x, nullptr, gamma, beta, smooth, nullptr, rows, n, dt, eps, qdt, y,
-                            scale, nullptr, nullptr, nullptr),
-                    false, ARNQ_MASK_ABSENT, workspace, workspace_bytes, stream, nullptr);
+                            scale, nullptr, nullptr, nullptr, false),
+                    ARNQ_MASK_ABSENT, workspace, workspace_bytes, stream, nullptr);
 }
 
 arnq_status arnq_make_plan(const void *x1, const void *x2, const void *gamma, const void *beta,
@@ -497,24 +525,13 @@ arnq_status arnq_make_plan(const void *x1, const void *x2, const void *gamma, co
   if (!plan) return ARNQ_ERR_NULL_PTR;
   Problem P = problem(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, 0.0f, qdt,
                       const_cast<void *>(y1), nullptr, const_cast<void *>(y2), nullptr,
-                      const_cast<void *>(x_out));
+                      const_cast<void *>(x_out), x2 != nullptr);
   arnq_status st = check_shape(rows, n, dt, qdt, 0.0f);
   if (st != ARNQ_OK) return st;
-  int on1 = 0, on2 = 0;
-  st = selected(out_mask, smooth1 != nullptr, smooth2 != nullptr, &on1, &on2);
+  st = select_outputs(P, out_mask);
   if (st != ARNQ_OK) return st;
-  int f = 0;
-  if (x2) f |= arnq::F_X2;
-  if (beta) f |= arnq::F_BETA;
-  if (smooth1) f |= arnq::F_S1;
-  if (smooth2) f |= arnq::F_S2;
-  if (on1) f |= arnq::F_OUT1;
-  if (on2) f |= arnq::F_OUT2;
-  if (x2 && x_out) f |= arnq::F_XOUT;
-  P.flags = f;
-  KernelFn fn = nullptr;
-  int smem = 0, seg = 0, units = 0;
-  return make_plan(P, plan, &fn, &smem, &seg, &units);
+  Launch L;
+  return make_plan(P, plan, &L);
 }
 
 }  // extern "C"

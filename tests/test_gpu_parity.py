@@ -203,7 +203,7 @@ PLAN_CASES = [
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=2, cluster=8, units=2),
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=4, cluster=16),
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=5, ctas_per_sm=1),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=2, ctas_per_sm=1, threads=1024),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4, ctas_per_sm=1, units=1),
 ]
 
 
@@ -220,7 +220,7 @@ def test_plans(pk, shape):
     compare(g, o, qdt, str(pk))
 
 
-@pytest.mark.parametrize("units", [1, 2, 4, 8])
+@pytest.mark.parametrize("units", [1, 4, 8])
 @pytest.mark.parametrize("cluster", [1, 4])
 def test_scalar_plans(units, cluster):
     # n not a multiple of 8 forces 2-element units
@@ -230,16 +230,16 @@ def test_scalar_plans(units, cluster):
 
 
 def test_bad_plans_are_rejected():
-    w = wl.random_case(8, 1000, seed=1)
+    w = wl.random_case(8, 1002, seed=1)
     x = dev_bits(w.x1, "bf16")
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-    y = torch.empty(8 * 1000, dtype=torch.int8, device="cuda")
+    y = torch.empty(8 * 1002, dtype=torch.int8, device="cuda")
     s = torch.empty(8, dtype=torch.float32, device="cuda")
     gm = dev_bits(w.gamma, "bf16")
     for bad in (dict(kernel=A.ARNQ_KERNEL_STAGED),   # n % 8 != 0 cannot be staged
                 dict(cluster=3), dict(threads=100), dict(units=3), dict(kernel=9),
-                dict(threads=32, units=1)):
-        st = A.arnq_run_planned(x, x, gm, None, None, None, 8, 1000, 0, 1e-6, -1, 0, y, s, None,
+                dict(threads=32, units=1), dict(units=2)):
+        st = A.arnq_run_planned(x, x, gm, None, None, None, 8, 1002, 0, 1e-6, -1, 0, y, s, None,
                                 None, None, ws, 256, None, plan(**bad))
         assert st == A.ARNQ_ERR_PLAN, bad
 
