@@ -16,14 +16,17 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC_DIR = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(SRC_DIR, "arnq_api.cu")]
-DEPS = SOURCES + [os.path.join(SRC_DIR, "arnq_kernels.cuh"), os.path.join(ROOT, "include", "arnq.h")]
+SOURCES = [os.path.join(SRC_DIR, f) for f in (
+    "arnq_api.cu", "arnq_k_bf16_int8.cu", "arnq_k_bf16_int4.cu", "arnq_k_fp16_int8.cu",
+    "arnq_k_fp16_int4.cu")]
+DEPS = SOURCES + [os.path.join(SRC_DIR, "arnq_kernels.cuh"), os.path.join(SRC_DIR, "arnq_table.h"),
+                  os.path.join(ROOT, "include", "arnq.h")]
 LIB = os.path.join(PKG, "libarnq.so")
+OBJ_DIR = os.path.join(ROOT, "_build")
 
 NVCC_FLAGS = [
     "-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-    "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "-shared",
-    "--expt-relaxed-constexpr", "-cudart", "static",
+    "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden", "--expt-relaxed-constexpr",
 ]
 
 
@@ -43,17 +46,33 @@ def up_to_date() -> bool:
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compiles every translation unit in parallel, then links the library."""
     if not force and up_to_date():
         return LIB
-    cmd = [nvcc(), *NVCC_FLAGS, "-I", os.path.join(ROOT, "include"), "-o", LIB, *SOURCES]
-    if verbose:
-        cmd.insert(1, "-Xptxas=-v")
-    res = subprocess.run(cmd, capture_output=True, text=True)
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    inc = ["-I", os.path.join(ROOT, "include")]
+    procs = []
+    for src in SOURCES:
+        obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
+        cmd = [nvcc(), *NVCC_FLAGS, *(["-Xptxas=-v"] if verbose else []), *inc, "-c", "-o", obj,
+               src]
+        procs.append((obj, subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.STDOUT,
+                                            text=True)))
+    objs, failed = [], False
+    for obj, p in procs:
+        out, _ = p.communicate()
+        if p.returncode != 0 or verbose:
+            sys.stderr.write(out)
+        failed |= p.returncode != 0
+        objs.append(obj)
+    if failed:
+        raise RuntimeError("nvcc failed compiling libarnq")
+    link = [nvcc(), "-shared", "-cudart", "static", "-gencode", "arch=compute_100a,code=sm_100a",
+            "-o", LIB, *objs]
+    res = subprocess.run(link, capture_output=True, text=True)
     if res.returncode != 0:
         sys.stderr.write(res.stdout + res.stderr)
-        raise RuntimeError("nvcc failed building libarnq.so")
-    if verbose:
-        sys.stderr.write(res.stdout + res.stderr)
+        raise RuntimeError("nvcc failed linking libarnq.so")
     return LIB
 
 

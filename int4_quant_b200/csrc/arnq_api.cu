@@ -11,70 +11,44 @@
 #include <mutex>
 
 #include "arnq.h"
-#include "arnq_kernels.cuh"
+#include "arnq_table.h"
 
 namespace {
 
 using arnq::KParams;
-typedef void (*KernelFn)(KParams);
+using arnq::KernelFn;
 
-constexpr int kHeaderSmem = arnq::kRingOff;  // reduction slots, abort flag, mbarriers
 constexpr size_t kWorkspaceBytes = 256;      // status block, padded
 constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
-constexpr int kMaxSegElems = 8192;           // elements of a row one CTA holds in registers
+constexpr int kMaxSegElems = 16384;          // elements of a row one CTA holds in registers
+constexpr int kMaxGroups = 15;               // named barriers 1..15
 
 // ---------------------------------------------------------------- kernel table
 
-// units per thread: 16-byte units 1 or 2; element pairs 1, 4 or 8
-constexpr int kUptSlots = 3;
-int upt_slot(int mode, int upt) {
-  if (mode == arnq::LOAD_SCALAR) return upt == 1 ? 0 : upt == 4 ? 1 : upt == 8 ? 2 : -1;
-  return upt == 1 ? 0 : upt == 2 ? 1 : -1;
-}
-
-template <class T, bool I4, int NOUT, bool ADD>
-void fill(KernelFn *t) {
-  t[0 * kUptSlots + 0] = arnq::rows_kernel<T, I4, arnq::LOAD_VEC, 1, NOUT, ADD>;
-  t[0 * kUptSlots + 1] = arnq::rows_kernel<T, I4, arnq::LOAD_VEC, 2, NOUT, ADD>;
-  t[0 * kUptSlots + 2] = nullptr;
-  t[1 * kUptSlots + 0] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 1, NOUT, ADD>;
-  t[1 * kUptSlots + 1] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 4, NOUT, ADD>;
-  t[1 * kUptSlots + 2] = arnq::rows_kernel<T, I4, arnq::LOAD_SCALAR, 8, NOUT, ADD>;
-  t[2 * kUptSlots + 0] = arnq::rows_kernel<T, I4, arnq::LOAD_STAGED, 1, NOUT, ADD>;
-  t[2 * kUptSlots + 1] = arnq::rows_kernel<T, I4, arnq::LOAD_STAGED, 2, NOUT, ADD>;
-  t[2 * kUptSlots + 2] = nullptr;
-}
-
-template <class T, bool I4>
-void fill_q(KernelFn (*t)[2][3 * kUptSlots]) {
-  fill<T, I4, 1, false>(t[0][0]);
-  fill<T, I4, 1, true>(t[0][1]);
-  fill<T, I4, 2, false>(t[1][0]);
-  fill<T, I4, 2, true>(t[1][1]);
-}
-
 struct KernelTable {
-  KernelFn fn[2][2][2][2][3 * kUptSlots];  // [dtype][qdtype][nout-1][add][mode*slots+upt]
+  KernelFn fn[2][2][arnq::kTableSize];  // [dtype][qdtype][...]
   KernelTable() {
-    fill_q<arnq::Bf16, false>(fn[0][0]);
-    fill_q<arnq::Bf16, true>(fn[0][1]);
-    fill_q<arnq::Fp16, false>(fn[1][0]);
-    fill_q<arnq::Fp16, true>(fn[1][1]);
+    std::memset(fn, 0, sizeof fn);
+    arnq::fill_table_bf16_int8(fn[0][0]);
+    arnq::fill_table_bf16_int4(fn[0][1]);
+    arnq::fill_table_fp16_int8(fn[1][0]);
+    arnq::fill_table_fp16_int4(fn[1][1]);
   }
 };
 
 KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt) {
   static const KernelTable table;
-  const int s = upt_slot(mode, upt);
+  const int s = arnq::upt_slot(mode, upt);
   if (s < 0 || nout < 1 || nout > 2) return nullptr;
-  return table.fn[dt][qdt][nout - 1][add ? 1 : 0][mode * kUptSlots + s];
+  return table.fn[dt][qdt][arnq::table_index(nout, add, mode, s)];
 }
 
 // mirrors arnq::MaxThreads
-int max_threads(int mode, int upt, int nout) {
-  const int elems = upt * (mode == arnq::LOAD_SCALAR ? 2 : 8);
-  return elems <= 8 ? (nout == 1 ? 1024 : 768) : 512;
+int max_threads(int mode, int upt) {
+  (void)mode;
+  (void)upt;
+  return 512;
 }
 
 // ---------------------------------------------------------------- device info
@@ -269,65 +243,70 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   const int seg = static_cast<int>(ceil_div(units, cl));
   if (seg > max_seg) return ARNQ_ERR_PLAN;
 
+  // units per thread: as many as keep at least two warps per row group
   if (pl->units == 0) {
-    if (mode == arnq::LOAD_SCALAR) {
-      pl->units = seg <= max_threads(mode, 1, nout) ? 1
-                  : seg <= 4 * max_threads(mode, 4, nout) ? 4 : 8;
-    } else {
-      pl->units = (seg >= 256 || seg > max_threads(mode, 1, nout)) ? 2 : 1;
+    const int cands[3] = {mode == arnq::LOAD_SCALAR ? 8 : 4, mode == arnq::LOAD_SCALAR ? 4 : 2, 1};
+    pl->units = 1;
+    for (int c : cands) {
+      const int64_t t = ceil_div(seg, c);
+      if (t >= 64 && t <= max_threads(mode, c)) { pl->units = c; break; }
     }
+    if (ceil_div(seg, pl->units) > max_threads(mode, pl->units))
+      pl->units = mode == arnq::LOAD_SCALAR ? 8 : 4;
   }
-  if (upt_slot(mode, pl->units) < 0) return ARNQ_ERR_PLAN;
+  if (arnq::upt_slot(mode, pl->units) < 0) return ARNQ_ERR_PLAN;
   if (pl->threads == 0) {
     pl->threads = round_up(static_cast<int>(ceil_div(seg, pl->units)), 32);
     if (pl->threads < 32) pl->threads = 32;
   }
-  if (pl->threads % 32 != 0 || pl->threads > max_threads(mode, pl->units, nout) ||
+  const int tmax = max_threads(mode, pl->units);
+  if (pl->threads % 32 != 0 || pl->threads > tmax ||
       static_cast<int64_t>(pl->threads) * pl->units < seg)
     return ARNQ_ERR_PLAN;
+  // row groups per CTA: fill the CTA's thread budget, one group per cluster CTA
+  if (pl->groups == 0) {
+    int g = cl > 1 ? 1 : tmax / pl->threads;
+    if (g > kMaxGroups) g = kMaxGroups;
+    const int64_t per_sm_rows = ceil_div(P.rows, di.sms);
+    if (g > per_sm_rows) g = static_cast<int>(per_sm_rows);
+    pl->groups = g < 1 ? 1 : g;
+  }
+  if (pl->groups < 1 || pl->groups > kMaxGroups || (cl > 1 && pl->groups != 1) ||
+      pl->groups * pl->threads > tmax)
+    return ARNQ_ERR_PLAN;
+  const int cta_threads = pl->groups * pl->threads;
+  const int pairs = pl->units * (mode == arnq::LOAD_SCALAR ? 1 : 4);
 
   KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units);
   if (!fn) return ARNQ_ERR_PLAN;
-  st = prepare_kernel(fn, dev, kHeaderSmem);
-  if (st != ARNQ_OK) return st;
-  int occ = 0;  // resident CTAs per SM allowed by threads and registers
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, fn, pl->threads, kHeaderSmem) !=
-      cudaSuccess)
-    return ARNQ_ERR_CUDA;
-  if (occ < 1) return ARNQ_ERR_PLAN;
-
-  int smem = kHeaderSmem;
+  const int stage_bytes = (P.add ? 2 : 1) * seg * 16;
+  int smem = arnq::layout_bytes(
+      arnq::make_layout(pl->groups, pl->threads, pairs, nout, cl, 0, 0), pl->groups);
   if (mode == arnq::LOAD_STAGED) {
-    const int per_stage = seg * 16 * (P.add ? 2 : 1);
-    int ctas = pl->ctas_per_sm != 0 ? pl->ctas_per_sm : (occ < 4 ? occ : 4);
-    if (pl->stages == 0) {
-      int s = 0;
-      while (true) {
-        int cap = di.smem_per_sm / ctas - 1024;  // 1 KB reserved per CTA
-        if (cap > di.smem_per_block_optin) cap = di.smem_per_block_optin;
-        s = (cap - kHeaderSmem) / per_stage;
-        if (s >= 2 || ctas == 1 || pl->ctas_per_sm != 0) break;
-        --ctas;
-      }
-      if (s > kMaxStages) s = kMaxStages;
-      if (s < 1) s = 1;
+    if (pl->stages == 0) {  // as deep a ring as the shared memory of one CTA per SM allows
+      int s = kMaxStages;
+      while (s > 1 && arnq::layout_bytes(arnq::make_layout(pl->groups, pl->threads, pairs, nout,
+                                                           cl, s, stage_bytes),
+                                         pl->groups) > di.smem_per_block_optin)
+        --s;
       pl->stages = s;
     }
-    pl->ctas_per_sm = ctas;
     if (pl->stages < 1 || pl->stages > kMaxStages) return ARNQ_ERR_PLAN;
-    smem = kHeaderSmem + pl->stages * per_stage;
-    if (smem > di.smem_per_block_optin) return ARNQ_ERR_PLAN;
-    st = prepare_kernel(fn, dev, smem);
-    if (st != ARNQ_OK) return st;
+    smem = arnq::layout_bytes(
+        arnq::make_layout(pl->groups, pl->threads, pairs, nout, cl, pl->stages, stage_bytes),
+        pl->groups);
   } else {
     pl->stages = 0;
   }
+  if (smem > di.smem_per_block_optin) return ARNQ_ERR_PLAN;
+  st = prepare_kernel(fn, dev, smem);
+  if (st != ARNQ_OK) return st;
 
   // grid: persistent, as many clusters as fit at once (or one per row)
   int64_t clusters_fit = 0;
   if (cl == 1) {
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, pl->threads, smem) !=
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, cta_threads, smem) !=
         cudaSuccess)
       return ARNQ_ERR_CUDA;
     if (per_sm < 1) return ARNQ_ERR_PLAN;
@@ -342,7 +321,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(cl * 1024, 1, 1);
-    cfg.blockDim = dim3(pl->threads, 1, 1);
+    cfg.blockDim = dim3(cta_threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -354,7 +333,8 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
     clusters_fit = want < nc ? want : nc;
     pl->ctas_per_sm = static_cast<int32_t>(ceil_div(clusters_fit * cl, di.sms));
   }
-  const int64_t nclusters = P.rows < clusters_fit ? P.rows : clusters_fit;
+  const int64_t clusters_needed = ceil_div(P.rows, pl->groups);
+  const int64_t nclusters = clusters_needed < clusters_fit ? clusters_needed : clusters_fit;
   pl->grid = static_cast<int32_t>(nclusters * cl);
   L->fn = fn;
   L->smem = smem;
@@ -395,12 +375,14 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   k.seg_units = L.seg;
   k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0);
   k.stages = plan.stages;
+  k.groups = plan.groups;
   k.eps = P.eps;
+  k.inv_n = 1.0 / static_cast<double>(P.n);
 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(plan.grid, 1, 1);
-  cfg.blockDim = dim3(plan.threads, 1, 1);
+  cfg.blockDim = dim3(plan.threads * plan.groups, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   if (plan.cluster > 1) {

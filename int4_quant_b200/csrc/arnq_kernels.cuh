@@ -15,22 +15,28 @@
 // exchanged through distributed shared memory.  Persistent grid: cluster c
 // handles rows c, c + nclusters, ...
 //
+// A CTA is split into row groups that each work on their own rows and meet
+// only at their own named barrier; the folded parameters live once per CTA in
+// shared memory, so a thread's registers hold just its elements of x.
+//
 // Arithmetic.  The bulk of the work is binary32, two lanes at a time with the
 // sm_100 packed instructions (add/mul/fma.rn.f32x2):
 //   x = RNE16(x1 + x2)                    -> xOut, kept as fp32 in registers
 //   ss = sum x^2                          fp64 (x^2 is exact; the sum agrees with
 //                                         an fp64 evaluation of the definition)
-//   rinv = 1/sqrt(ss/n + eps)             fp64 per row, rounded once to fp32
-//   input_k = x*rinv*G_k + B_k            G_k = gamma*smooth_k, B_k = beta*smooth_k
-//   amax_k = max |input_k|                fp32 to find candidates; the candidates
-//                                         are re-evaluated in fp64, so
-//   scale_k = fp32(amax_k / Q)            matches an fp64 evaluation bit for bit
+//   rinv = 1/sqrt(ss/n + eps)             binary32, within 3 ulp
+//   input_k = x*rinv*G_k + B_k            G_k = gamma*smooth_k, B_k = beta*smooth_k,
+//                                         exact products of two 16-bit values
+//   amax_k = max |input_k|                binary32 scan; the elements within the
+//                                         error bound of the row maximum are
+//                                         re-evaluated in fp64, so
+//   scale_k = fp32(amax_k / Q)            equals the fp64 evaluation's scale
 //   t = input_k * (1/scale_k)             rounded half-to-even by adding 1.5*2^23
-// A code whose binary32 quotient t lies within the proven error bound tau of a
-// half-way point is recomputed in fp64 in the definition's order
-// (x / Rms * gamma + beta) * smooth / scale, so every rounding decision is the
-// one an fp64 evaluation of the definition makes.  Nothing here is a
-// contraction: no tensor cores.
+// |t - t_exact| <= 7u|t| + 4u|B_k|/scale_k (u = 2^-24).  A code whose binary32
+// quotient lies within that bound of a half-way point is recomputed in fp64 in
+// the definition's order, (x / Rms * gamma + beta) * smooth / scale, so every
+// rounding decision is the one an fp64 evaluation of the definition makes.
+// Nothing here is a contraction: no tensor cores.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -54,15 +60,44 @@ enum : int { DEV_TIMEOUT = 11 };
 // A bounded wait gives up after this long (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
-// Shared-memory header: per-warp slots for the two row reductions (fp64, up to
-// 16 CTAs x 32 warps, two outputs), an abort flag, up to 16 mbarriers.
-constexpr int kMaxStagesDev = 16;
-constexpr int kSlotsSS = 0;                        // 512 doubles
-constexpr int kSlotsMax = kSlotsSS + 512 * 8;      // 512 x 2 doubles
-constexpr int kAbortOff = kSlotsMax + 512 * 16;    // int
-constexpr int kBarsOff = kAbortOff + 128;          // 16 x uint64
-constexpr int kRingOff = kBarsOff + 8 * kMaxStagesDev;
-static_assert(kRingOff % 128 == 0, "ring must stay 128-byte aligned");
+// Shared-memory layout, sized by the launch (the host computes the same):
+//   params   [NOUT][UPT][W][TG] float4 {G.x, G.y, B.x, B.y}: the folded
+//            parameters of the CTA's columns, one copy shared by all groups
+//   maxb     [NOUT][cl * warps per CTA] floats: set-up reduction of |B|
+//   per row group g (stride `group`):
+//     ss     [cl * warps per group] doubles: partial sums of squares
+//     mx     [NOUT][cl * warps per group] floats: partial binary32 maxima
+//     sc     [2][NOUT] binary32 bit patterns: the scales of the last two rows
+//     abort  int; bars [stages] mbarriers; ring [stages] rows of staged input
+constexpr int kMaxStagesDev = 8;
+struct Layout {
+  int params, maxb, group0, group;       // offsets and the per-group stride
+  int ss, mx, sc, abort, bars, ring;     // offsets within a group
+};
+__host__ __device__ inline Layout make_layout(int groups, int tg, int pairs_per_thread, int nout,
+                                              int cl, int stages, int stage_bytes) {
+  Layout L;
+  const int nwarps_cta = groups * tg / 32;
+  const int nslots = cl * (tg / 32);
+  int off = 0;
+  L.params = off; off += nout * pairs_per_thread * tg * 16;
+  L.maxb = off;   off += nout * cl * nwarps_cta * 4;
+  L.group0 = (off + 127) & ~127;
+  int g = 0;
+  L.ss = g;    g += nslots * 8;
+  L.mx = g;    g += nout * nslots * 4;
+  L.sc = g;    g += 2 * nout * 4;
+  g = (g + 7) & ~7;
+  L.abort = g; g += 8;
+  L.bars = g;  g += stages * 8;
+  L.ring = (g + 127) & ~127;
+  g = L.ring + stages * stage_bytes;
+  L.group = (g + 127) & ~127;
+  return L;
+}
+__host__ __device__ inline int layout_bytes(const Layout &L, int groups) {
+  return L.group0 + groups * L.group;
+}
 
 struct KParams {
   const uint16_t *x1, *x2, *gamma, *beta;
@@ -76,8 +111,10 @@ struct KParams {
   int32_t units;              // units per row: ceil(n / U)
   int32_t seg_units;          // units per CTA of a cluster
   int32_t flags;
-  int32_t stages;             // staged kernel: ring depth
+  int32_t stages;             // staged kernel: ring depth per row group
+  int32_t groups;             // row groups per CTA (1 when cl > 1)
   float eps;
+  double inv_n;               // 1 / n
 };
 
 struct Bf16 {};
@@ -140,14 +177,17 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// One try of an mbarrier phase wait; the thread may sleep in hardware for up
+// to kSuspendHintNs while the phase is incomplete.
+constexpr uint32_t kSuspendHintNs = 100000u;
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(kSuspendHintNs)
       : "memory");
   return ok != 0;
 }
@@ -194,74 +234,138 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
-__device__ __forceinline__ double warp_max_d(double v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
-
-// Threads per CTA the register budget allows: a thread keeps x (fp32) and the
-// folded parameters (fp32) of its elements for every output across rows.
-template <int MODE, int UPT, int NOUT>
+// Threads per CTA: 512, so a thread may use 128 registers -- x for up to 32
+// elements plus the fp64 paths, without spilling.
+template <int MODE, int UPT>
 struct MaxThreads {
-  static constexpr int elems = UPT * (MODE == LOAD_SCALAR ? 2 : 8);
-  static constexpr int value = (elems <= 8) ? (NOUT == 1 ? 1024 : 768) : 512;
+  static constexpr int value = 512;
 };
 
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: v + kMagic = RNE(v) + kMagic
 constexpr uint32_t kMagicBits = 0x4B400000u;  // its bit pattern; low bits then hold RNE(v)
 constexpr float kUnit = 5.9604644775390625e-08f;  // 2^-24, binary32 unit roundoff
 
+// Rms(x) = sqrt(ss/n + eps) in fp64, IEEE-rounded operations in the
+// definition's order.
+static __device__ __forceinline__ double rms_exact(double ss, int n, float eps) {
+  return __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(n)), static_cast<double>(eps)));
+}
+
+// |input| of one element in fp64 from the folded parameters, which are exact
+// products (G = gamma*smooth, B = beta*smooth fit in binary32): |x/Rms*G + B|.
+static __device__ __forceinline__ double input_abs_folded(float x, float g, float b, double rms) {
+  return fabs(__fma_rn(__ddiv_rn(static_cast<double>(x), rms), static_cast<double>(g),
+                       static_cast<double>(b)));
+}
+
+// The code of one element decided in fp64 exactly as the definition orders it:
+// round_half_even((x / Rms * gamma + beta) * smooth / scale), clamped to
+// [-Q, Q]; returned as kMagicBits + code so its low bits pack like the fast path.
+template <class T>
+__device__ __forceinline__ uint32_t code_exact(const uint16_t *gamma, const uint16_t *beta,
+                                            const uint16_t *smooth, int c, float x, double rms,
+                                            float scale, int qmax) {
+  int q = 0;
+  if (scale != 0.f) {
+    double y = __dmul_rn(__ddiv_rn(static_cast<double>(x), rms),
+                         static_cast<double>(Cvt<T>::f1(gamma[c])));
+    if (beta) y = __dadd_rn(y, static_cast<double>(Cvt<T>::f1(beta[c])));
+    if (smooth) y = __dmul_rn(y, static_cast<double>(Cvt<T>::f1(smooth[c])));
+    q = __double2int_rn(__ddiv_rn(y, static_cast<double>(scale)));
+    q = min(max(q, -qmax), qmax);
+  }
+  return kMagicBits + static_cast<uint32_t>(q);
+}
+
+// 1/sqrt(v) in binary32: the hardware estimate refined by one Newton-Raphson
+// step, r' = r (3 - v r^2) / 2; within 3 ulp.
+__device__ __forceinline__ float rsqrt_refined(float v) {
+  const float r = rsqrtf(v);
+  const float h = 0.5f * v;
+  return r * __fmaf_rn(-h * r, r, 1.5f);
+}
+
+// max over lanes of non-negative floats (their bit patterns order as integers)
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+  return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(v)));
+}
+
 // ---------------------------------------------------------------- row kernel
 
+// A CTA holds `groups` row groups of TG = blockDim / groups threads.  Each group
+// works on its own rows (group id g of cluster c takes rows c*groups + g,
+// + nclusters*groups, ...) and synchronizes only its own threads, with the
+// named barrier 1 + g; a cluster (cl > 1) has one group per CTA and uses the
+// cluster barrier.
 template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD>
-__global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
-    rows_kernel(const KParams p) {
+__global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(const KParams p) {
   using C = Cvt<T>;
   constexpr int U = (MODE == LOAD_SCALAR) ? 2 : 8;  // elements per unit
   constexpr int W = U / 2;                          // element pairs per unit
   constexpr int QI = INT4 ? 7 : 127;
   constexpr float QF = static_cast<float>(QI);
+  constexpr int NIN = ADD ? 2 : 1;                  // staged inputs per row
 
-  const int tid = threadIdx.x;
-  const int lane = tid & 31;
-  const int warp = tid >> 5;
-  const int nwarps = blockDim.x >> 5;
   cg::cluster_group cluster = cg::this_cluster();
   const int cl = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int64_t cluster_id = blockIdx.x / cl;
   const int64_t nclusters = gridDim.x / cl;
+  const int groups = p.groups;
+  const int TG = static_cast<int>(blockDim.x) / groups;
+  const int tid = threadIdx.x;
+  const int gid = tid / TG;           // row group
+  const int gt = tid - gid * TG;      // thread within the group
+  const int lane = tid & 31;
+  const int gwarp = gt >> 5;
+  const int nwg = TG >> 5;            // warps per group
+  const int nslots = cl * nwg;
+  const int my_slot = rank * nwg + gwarp;
+  const int64_t group_id = cluster_id * groups + gid;
+  const int64_t ngroups = nclusters * groups;
   const int n = p.n;
   const bool has_beta = (p.flags & F_BETA) != 0;
-
-  extern __shared__ __align__(128) unsigned char smem[];
-  double *ss_slots = reinterpret_cast<double *>(smem + kSlotsSS);    // [cl * nwarps]
-  double *max_slots = reinterpret_cast<double *>(smem + kSlotsMax);  // [NOUT][cl * nwarps]
-  int *abort_any = reinterpret_cast<int *>(smem + kAbortOff);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kBarsOff);
-  unsigned char *ring = smem + kRingOff;
+  const int ring_depth = (MODE == LOAD_STAGED) ? p.stages : 0;  // stages in the layout
+  const int stages = (MODE == LOAD_STAGED) ? p.stages : 1;      // ring arithmetic
 
   const int seg_begin = rank * p.seg_units;
   const int seg_end = min(seg_begin + p.seg_units, p.units);
   const int seg_len = max(seg_end - seg_begin, 0);
   const uint32_t seg_bytes = static_cast<uint32_t>(seg_len) * 16u;  // staged: bytes per input
-  const int nslots = cl * nwarps;
+  const uint32_t stage_bytes = NIN * static_cast<uint32_t>(p.seg_units) * 16u;
 
-  // column of element h (0/1) of pair i of this thread's k-th unit
-  auto col = [&](int k, int i, int h) -> int {
-    const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
-    return u * U + 2 * i + h;
+  extern __shared__ __align__(128) unsigned char smem[];
+  const Layout lay = make_layout(groups, TG, UPT * W, NOUT, cl, ring_depth, stage_bytes);
+  float4 *params = reinterpret_cast<float4 *>(smem + lay.params);
+  float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);
+  unsigned char *gb = smem + lay.group0 + gid * lay.group;
+  double *ss_slots = reinterpret_cast<double *>(gb + lay.ss);   // [nslots]
+  float *mx_slots = reinterpret_cast<float *>(gb + lay.mx);     // [NOUT][nslots]
+  unsigned *sc_slot = reinterpret_cast<unsigned *>(gb + lay.sc);  // [2][NOUT]
+  int *abort_flag = reinterpret_cast<int *>(gb + lay.abort);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(gb + lay.bars);
+  unsigned char *ring = gb + lay.ring;
+
+  auto group_sync = [&]() {
+    if (cl > 1) {
+      cluster.sync();
+    } else {
+      asm volatile("bar.sync %0, %1;" ::"r"(1 + gid), "r"(TG) : "memory");
+    }
+  };
+  // the folded parameters of pair i of this thread's k-th unit, output o
+  auto par = [&](int o, int k, int i) -> float4 {
+    return params[((o * UPT + k) * W + i) * TG + gt];
   };
 
-  // ---- folded parameters for this thread's units: input_k = a * G_k + B_k
-  float2 G[NOUT][UPT][W], B[NOUT][UPT][W];
+  // ---- set-up: fold gamma, beta, smooth into G, B (group 0 writes the shared
+  // copy); every thread keeps the bound on |B| over its own elements
   float maxB[NOUT];
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) maxB[o] = 0.f;
 #pragma unroll
   for (int k = 0; k < UPT; ++k) {
-    const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
+    const int u = seg_begin + gt + k * TG;
     const bool ok = u < seg_end;
     uint32_t gw[W], bw[W], sw[NOUT][W];
 #pragma unroll
@@ -288,16 +392,16 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
       } else {
         const int j = 2 * u;
         const bool two = j + 1 < n;
-        auto pair = [&](const uint16_t *a) -> uint32_t {
-          const uint32_t lo = __ldg(a + j);
-          const uint32_t hi = two ? __ldg(a + j + 1) : 0u;
-          return lo | (hi << 16);
-        };
-        gw[0] = pair(p.gamma);
-        if (has_beta) bw[0] = pair(p.beta);
+        gw[0] = static_cast<uint32_t>(__ldg(p.gamma + j)) |
+                (two ? static_cast<uint32_t>(__ldg(p.gamma + j + 1)) << 16 : 0u);
+        if (has_beta)
+          bw[0] = static_cast<uint32_t>(__ldg(p.beta + j)) |
+                  (two ? static_cast<uint32_t>(__ldg(p.beta + j + 1)) << 16 : 0u);
 #pragma unroll
         for (int o = 0; o < NOUT; ++o)
-          if (p.smooth[o]) sw[o][0] = pair(p.smooth[o]);
+          if (p.smooth[o])
+            sw[o][0] = static_cast<uint32_t>(__ldg(p.smooth[o] + j)) |
+                       (two ? static_cast<uint32_t>(__ldg(p.smooth[o] + j + 1)) << 16 : 0u);
       }
     }
 #pragma unroll
@@ -307,55 +411,65 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
 #pragma unroll
       for (int o = 0; o < NOUT; ++o) {
         const float2 s2 = p.smooth[o] ? C::f2(sw[o][i]) : make_float2(1.f, 1.f);
-        G[o][k][i] = __fmul2_rn(g2, s2);
-        B[o][k][i] = __fmul2_rn(b2, s2);
-        maxB[o] = fmaxf(maxB[o], fmaxf(fabsf(B[o][k][i].x), fabsf(B[o][k][i].y)));
+        const float2 G = __fmul2_rn(g2, s2);  // exact: two 8- (or 11-) bit significands
+        const float2 B = __fmul2_rn(b2, s2);
+        maxB[o] = fmaxf(maxB[o], fmaxf(fabsf(B.x), fabsf(B.y)));
+        if (gid == 0) params[((o * UPT + k) * W + i) * TG + gt] = make_float4(G.x, G.y, B.x, B.y);
       }
     }
   }
-
-  // ---- staged ring set-up
-  uint64_t policy = 0;
-  const int stages = (MODE == LOAD_STAGED) ? p.stages : 1;
-  const uint32_t stage_stride = ADD ? 2u * seg_bytes : seg_bytes;
-  if (tid == 0) {
-    *abort_any = 0;
+  const int nwarps_cta = static_cast<int>(blockDim.x) >> 5;
+#pragma unroll
+  for (int o = 0; o < NOUT; ++o) {
+    const float v = warp_max_nonneg(maxB[o]);
+    if (lane == 0) {
+      const int slot = o * cl * nwarps_cta + rank * nwarps_cta + (tid >> 5);
+      if (cl == 1) {
+        maxb_slots[slot] = v;
+      } else {
+        for (int r = 0; r < cl; ++r) cluster.map_shared_rank(maxb_slots, r)[slot] = v;
+      }
+    }
+  }
+  if (gt == 0) {
+    *abort_flag = 0;
+    for (int q = 0; q < 2 * NOUT; ++q) sc_slot[q] = 0u;
     if (MODE == LOAD_STAGED) {
       for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
   }
   if (cl > 1) cluster.sync(); else __syncthreads();
+  float maxBg[NOUT];  // bound on |B| over the whole row
+#pragma unroll
+  for (int o = 0; o < NOUT; ++o) {
+    float m = 0.f;
+    for (int i = lane; i < cl * nwarps_cta; i += 32) m = fmaxf(m, maxb_slots[o * cl * nwarps_cta + i]);
+    maxBg[o] = warp_max_nonneg(m);
+  }
 
+  // staged: row `row` goes to stage s, x1 then x2
+  uint64_t policy = 0;
   auto issue = [&](int64_t row, int s) {
     const uint32_t bar = smem_addr(&bars[s]);
-    const uint32_t dst = smem_addr(ring + static_cast<size_t>(s) * stage_stride);
+    const uint32_t dst = smem_addr(ring + static_cast<size_t>(s) * stage_bytes);
     const int64_t off = row * n + static_cast<int64_t>(seg_begin) * 8;
-    mbar_arrive_expect_tx(bar, stage_stride);
+    mbar_arrive_expect_tx(bar, NIN * seg_bytes);
     bulk_g2s(dst, p.x1 + off, seg_bytes, bar, policy);
     if (ADD) bulk_g2s(dst + seg_bytes, p.x2 + off, seg_bytes, bar, policy);
   };
-  if (MODE == LOAD_STAGED && tid == 0 && seg_len > 0) {
+  if (MODE == LOAD_STAGED && gt == 0 && seg_len > 0) {
     policy = policy_evict_first();
     for (int s = 0; s < stages; ++s) {
-      const int64_t row = cluster_id + s * nclusters;
+      const int64_t row = group_id + s * ngroups;
       if (row < p.rows) issue(row, s);
     }
   }
 
-  // fp64 re-evaluation of input_k at one column, in the definition's order:
-  // (x / Rms * gamma + beta) * smooth_k, with Rms = sqrt(ss/n + eps).
-  auto input64 = [&](int o, int c, float x, double rms) -> double {
-    double y = __dmul_rn(__ddiv_rn(static_cast<double>(x), rms),
-                         static_cast<double>(C::f1(p.gamma[c])));
-    if (has_beta) y = __dadd_rn(y, static_cast<double>(C::f1(p.beta[c])));
-    if (p.smooth[o]) y = __dmul_rn(y, static_cast<double>(C::f1(p.smooth[o][c])));
-    return y;
-  };
-
   int64_t it = 0;
-  for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
+  for (int64_t row = group_id; row < p.rows; row += ngroups, ++it) {
     const int stage = (MODE == LOAD_STAGED) ? static_cast<int>(it % stages) : 0;
+    const int par2 = static_cast<int>(it & 1);
     bool timed_out = false;
     if (MODE == LOAD_STAGED && seg_len > 0) {
       const uint32_t parity = static_cast<uint32_t>((it / stages) & 1);
@@ -367,7 +481,7 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
     double ss = 0.0;
 #pragma unroll
     for (int k = 0; k < UPT; ++k) {
-      const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
+      const int u = seg_begin + gt + k * TG;
       const bool ok = u < seg_end;
       uint32_t a[W], b[W];
 #pragma unroll
@@ -382,7 +496,7 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
             b[0] = vb.x; b[1] = vb.y; b[2] = vb.z; b[3] = vb.w;
           }
         } else if (MODE == LOAD_STAGED) {
-          const unsigned char *st = ring + static_cast<size_t>(stage) * stage_stride;
+          const unsigned char *st = ring + static_cast<size_t>(stage) * stage_bytes;
           const uint4 va = *reinterpret_cast<const uint4 *>(st + (u - seg_begin) * 16);
           a[0] = va.x; a[1] = va.y; a[2] = va.z; a[3] = va.w;
           if (ADD) {
@@ -404,8 +518,8 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
 #pragma unroll
       for (int i = 0; i < W; ++i) {
         if (ADD) {
-          const float2 s = __fadd2_rn(C::f2(a[i]), C::f2(b[i]));  // binary32 add
-          xo[i] = C::pack(s.x, s.y);                              // RNE to 16 bits
+          const float2 sum = __fadd2_rn(C::f2(a[i]), C::f2(b[i]));  // binary32 add
+          xo[i] = C::pack(sum.x, sum.y);                            // RNE to 16 bits
         } else {
           xo[i] = a[i];
         }
@@ -432,151 +546,175 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
       const bool any_to = __any_sync(0xFFFFFFFFu, timed_out);
       if (lane == 0) {
         if (cl == 1) {
-          ss_slots[warp] = v;
-          if (any_to) *abort_any = 1;
+          ss_slots[gwarp] = v;
+          if (any_to) *abort_flag = 1;
         } else {
           for (int r = 0; r < cl; ++r) {
-            cluster.map_shared_rank(ss_slots, r)[rank * nwarps + warp] = v;
-            if (any_to) *cluster.map_shared_rank(abort_any, r) = 1;
+            cluster.map_shared_rank(ss_slots, r)[my_slot] = v;
+            if (any_to) *cluster.map_shared_rank(abort_flag, r) = 1;
           }
         }
       }
     }
-    if (cl > 1) cluster.sync(); else __syncthreads();
+    group_sync();
 
     if (MODE == LOAD_STAGED) {
-      if (*abort_any) {
+      if (*abort_flag) {
         // A copy never completed: record it, wait (bounded) for the copies this
-        // CTA still has in flight, and leave.  Every CTA of the cluster sees the
-        // flag after the same barrier, so all of them leave together.
-        if (tid == 0) {
+        // group still has in flight, and stop.  Every thread of the group (and
+        // of the cluster) sees the flag after the same barrier.
+        if (gt == 0) {
           if (atomicCAS(p.status, 0, DEV_TIMEOUT) == 0) {
             *reinterpret_cast<volatile int64_t *>(p.status + 2) = row;
           }
           if (seg_len > 0) {
             for (int s = 0; s < stages; ++s) {
               const int64_t it2 = it + s;  // the ring's outstanding iterations
-              const int64_t r2 = cluster_id + it2 * nclusters;
-              if (r2 >= p.rows) break;
+              if (group_id + it2 * ngroups >= p.rows) break;
               mbar_wait_bounded(smem_addr(&bars[it2 % stages]),
                                 static_cast<uint32_t>((it2 / stages) & 1));
             }
           }
         }
-        if (cl > 1) cluster.sync(); else __syncthreads();
-        return;
+        break;
       }
-      // every thread has read this stage: refill it with the row `stages` ahead
-      if (tid == 0 && seg_len > 0) {
-        const int64_t nrow = row + static_cast<int64_t>(stages) * nclusters;
+      // every thread of the group has read this stage: refill it
+      if (gt == 0 && seg_len > 0) {
+        const int64_t nrow = row + static_cast<int64_t>(stages) * ngroups;
         if (nrow < p.rows) issue(nrow, stage);
       }
+    }
+    // every thread read the previous row's scales before this barrier
+    if (gt == 0) {
+#pragma unroll
+      for (int o = 0; o < NOUT; ++o) sc_slot[(par2 ^ 1) * NOUT + o] = 0u;
     }
 
     double ss_row = 0.0;
     for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
     ss_row = warp_sum_d(ss_row);
-    // Rms(x) = sqrt(ss/n + eps), fp64 as in the definition
-    const double rms64 = __dsqrt_rn(
-        __dadd_rn(__ddiv_rn(ss_row, static_cast<double>(n)), static_cast<double>(p.eps)));
-    const float rinv32 = __frcp_rn(__double2float_rn(rms64));  // within 1 ulp of 1/Rms
-    const float2 rinv2 = make_float2(rinv32, rinv32);
-
-    // ---- pass 2: row max of |input_k|: binary32 scan, fp64 for the candidates
-    double cand[NOUT];
-#pragma unroll
-    for (int o = 0; o < NOUT; ++o) {
-      float m32 = 0.f;
-#pragma unroll
-      for (int k = 0; k < UPT; ++k)
-#pragma unroll
-        for (int i = 0; i < W; ++i) {
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
-          m32 = fmaxf(m32, fmaxf(fabsf(in.x), fabsf(in.y)));
-        }
-      // every element within the binary32 error bound of the thread's maximum is a
-      // candidate for the true maximum; those are re-evaluated in fp64
-      const float thr = m32 - 12.f * kUnit * (m32 + maxB[o]);
-      double c64 = 0.0;
-#pragma unroll
-      for (int k = 0; k < UPT; ++k)
-#pragma unroll
-        for (int i = 0; i < W; ++i) {
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
-          if (fabsf(in.x) >= thr && m32 > 0.f)
-            c64 = fmax(c64, fabs(input64(o, col(k, i, 0), xf[k][i].x, rms64)));
-          if (fabsf(in.y) >= thr && m32 > 0.f)
-            c64 = fmax(c64, fabs(input64(o, col(k, i, 1), xf[k][i].y, rms64)));
-        }
-      cand[o] = c64;
+    float2 rinv2;
+    {
+      const float v = __double2float_rn(__fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps)));
+      const float r = rsqrt_refined(v);
+      rinv2 = make_float2(r, r);
     }
 
-    // ---- exchange 2: row max of |input_k| (fp64)
+    // ---- pass 2: binary32 row maxima of |input_k|
+    float m32[NOUT];
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
-      const double v = warp_max_d(cand[o]);
+      float m = 0.f;
+#pragma unroll
+      for (int k = 0; k < UPT; ++k)
+#pragma unroll
+        for (int i = 0; i < W; ++i) {
+          const float4 gbv = par(o, k, i);
+          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
+                                       make_float2(gbv.z, gbv.w));
+          m = fmaxf(m, fmaxf(fabsf(in.x), fabsf(in.y)));
+        }
+      m32[o] = m;
+      const float v = warp_max_nonneg(m);
       if (lane == 0) {
         if (cl == 1) {
-          max_slots[o * nslots + warp] = v;
+          mx_slots[o * nslots + gwarp] = v;
         } else {
-          for (int r = 0; r < cl; ++r)
-            cluster.map_shared_rank(max_slots, r)[o * nslots + rank * nwarps + warp] = v;
+          for (int r = 0; r < cl; ++r) cluster.map_shared_rank(mx_slots, r)[o * nslots + my_slot] = v;
         }
       }
     }
-    if (cl > 1) cluster.sync(); else __syncthreads();
+    // ---- exchange 2: binary32 row maxima
+    group_sync();
 
-    // scale_k = fp32(row_max / Q); r = 1/scale (binary32); a zero scale gives zero
-    // codes; a scale whose reciprocal is not a normal binary32 number sends every
-    // code of the row through the fp64 path.
-    float sc[NOUT], r32[NOUT], lim[NOUT];
+    // Every element whose binary32 value is within the error bound of the row
+    // maximum is a candidate for the true maximum (usually exactly one per row).
+    // Candidates are evaluated in fp64 and each offers fp32(|input| / Q); as that
+    // rounding is monotonic, the atomic maximum of the offers (binary32 bit
+    // patterns of non-negative values order as integers) is fp32(amax / Q).
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
-      double m = 0.0;
-      for (int i = lane; i < nslots; i += 32) m = fmax(m, max_slots[o * nslots + i]);
-      m = warp_max_d(m);
-      sc[o] = __double2float_rn(__ddiv_rn(m, static_cast<double>(QI)));
-      const bool tiny = sc[o] != 0.f && sc[o] < 1.1754943508222875e-38f;
-      r32[o] = (sc[o] == 0.f || tiny) ? 0.f : __frcp_rn(sc[o]);
-      // |t - t_exact| <= 10u (|t| + |B| r) (see the file header); 12u for margin,
-      // plus the binary32 rounding of the scale itself
-      const float tau = 12.f * kUnit * (QF + maxB[o] * r32[o]) + 2.f * kUnit * QF;
-      lim[o] = tiny ? -1.f : 0.5f - tau;
-      if (tid == 0 && rank == 0) p.scale[o][row] = sc[o];
+      float g = 0.f;
+      for (int i = lane; i < nslots; i += 32) g = fmaxf(g, mx_slots[o * nslots + i]);
+      g = warp_max_nonneg(g);
+      const float thr = g - 12.f * kUnit * (g + maxBg[o]);
+      if (g > 0.f && m32[o] >= thr) {
+        const double rms = rms_exact(ss_row, n, p.eps);
+        double c64 = 0.0;
+#pragma unroll
+        for (int k = 0; k < UPT; ++k)
+#pragma unroll
+          for (int i = 0; i < W; ++i) {
+            const float4 gbv = par(o, k, i);
+            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
+                                         make_float2(gbv.z, gbv.w));
+            if (fabsf(in.x) >= thr)
+              c64 = fmax(c64, input_abs_folded(xf[k][i].x, gbv.x, gbv.z, rms));
+            if (fabsf(in.y) >= thr)
+              c64 = fmax(c64, input_abs_folded(xf[k][i].y, gbv.y, gbv.w, rms));
+          }
+        const unsigned offer =
+            __float_as_uint(__double2float_rn(__ddiv_rn(c64, static_cast<double>(QI))));
+        unsigned *slot = &sc_slot[par2 * NOUT + o];
+        if (cl == 1) {
+          atomicMax(slot, offer);
+        } else {
+          for (int r = 0; r < cl; ++r) atomicMax(cluster.map_shared_rank(slot, r), offer);
+        }
+      }
     }
+    // ---- exchange 3: the scales
+    group_sync();
 
-    // ---- pass 3: quantize (round half to even via the 1.5*2^23 trick) and store
+    // ---- pass 3: quantize (round half to even via the 1.5*2^23 trick) and store.
+    // A zero scale gives zero codes; a scale whose reciprocal is not a normal
+    // binary32 number sends every code of the row through the fp64 path.
+    double rms_cached = -1.0;
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
-      const float2 r2 = make_float2(r32[o], r32[o]);
+      const float sc = __uint_as_float(sc_slot[par2 * NOUT + o]);
+      const bool tiny = sc != 0.f && sc < 1.1754943508222875e-38f;
+      const float r32 = (sc == 0.f || tiny) ? 0.f : __frcp_rn(sc);
+      const float tau = 12.f * kUnit * (QF + maxB[o] * r32) + 2.f * kUnit * QF;
+      const float lim = tiny ? -1.f : 0.5f - tau;
+      if (gt == 0 && rank == 0) p.scale[o][row] = sc;
+      const float2 r2 = make_float2(r32, r32);
       uint8_t *y = p.y[o];
 #pragma unroll
       for (int k = 0; k < UPT; ++k) {
-        const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
+        const int u = seg_begin + gt + k * TG;
         if (u >= seg_end) continue;
         uint32_t bits[2 * W];  // low bits: the code (two's complement)
+        float dmax = 0.f;      // largest |t - RNE(t)| of the unit
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
+          const float4 gbv = par(o, k, i);
+          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
+                                       make_float2(gbv.z, gbv.w));
           const float2 t = __fmul2_rn(in, r2);
           const float2 m = __fadd2_rn(t, make_float2(kMagic, kMagic));
           const float2 rr = __fadd2_rn(m, make_float2(-kMagic, -kMagic));  // RNE(t), exact
           const float2 d = __ffma2_rn(rr, make_float2(-1.f, -1.f), t);     // t - RNE(t), exact
           bits[2 * i] = __float_as_uint(m.x);
           bits[2 * i + 1] = __float_as_uint(m.y);
-          const bool nx = fabsf(d.x) > lim[o];
-          const bool ny = fabsf(d.y) > lim[o];
-          if (nx || ny) {  // near a half-way point: decide in fp64
-            const int h0 = nx ? 0 : 1, h1 = ny ? 1 : 0;
-            for (int h = h0; h <= h1; ++h) {
-              const float xv = h ? xf[k][i].y : xf[k][i].x;
-              const double v = input64(o, col(k, i, h), xv, rms64);
-              int q = 0;
-              if (sc[o] != 0.f) {
-                q = __double2int_rn(__ddiv_rn(v, static_cast<double>(sc[o])));
-                q = min(max(q, -QI), QI);
-              }
-              bits[2 * i + h] = kMagicBits + static_cast<uint32_t>(q);
+          dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
+        }
+        if (dmax > lim) {  // some code is near a half-way point: decide those in fp64
+          if (rms_cached < 0.0) rms_cached = rms_exact(ss_row, n, p.eps);
+#pragma unroll
+          for (int i = 0; i < W; ++i) {
+            const float4 gbv = par(o, k, i);
+            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
+                                         make_float2(gbv.z, gbv.w));
+            const float2 t = __fmul2_rn(in, r2);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float th = h ? t.y : t.x;
+              const float dv = fabsf(th - rintf(th));
+              if (dv > lim)
+                bits[2 * i + h] = code_exact<T>(p.gamma, has_beta ? p.beta : nullptr,
+                                                p.smooth[o], u * U + 2 * i + h,
+                                                h ? xf[k][i].y : xf[k][i].x, rms_cached, sc, QI);
             }
           }
         }
@@ -585,8 +723,8 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
             uint32_t w = 0;
 #pragma unroll
             for (int e = 0; e < 8; ++e) w |= (bits[e] & 0xFu) << (4 * e);
-            __stcs(reinterpret_cast<unsigned int *>(y + row * (n / 2) + static_cast<int64_t>(u) * 4),
-                   w);
+            __stcs(reinterpret_cast<unsigned int *>(y + row * (n / 2) +
+                                                    static_cast<int64_t>(u) * 4), w);
           } else {     // 8 codes -> 8 bytes
             const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
                                             __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
@@ -597,7 +735,8 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT, NOUT>::value)
           }
         } else {
           if (INT4) {
-            y[row * (n / 2) + u] = static_cast<uint8_t>((bits[0] & 0xFu) | ((bits[1] & 0xFu) << 4));
+            y[row * (n / 2) + u] =
+                static_cast<uint8_t>((bits[0] & 0xFu) | ((bits[1] & 0xFu) << 4));
           } else {
             const int64_t j = row * n + 2 * static_cast<int64_t>(u);
             y[j] = static_cast<uint8_t>(bits[0] & 0xFFu);
