@@ -183,13 +183,12 @@ typedef enum arnq_kernel {
 typedef struct arnq_plan {
   int32_t kernel;        /* arnq_kernel                                        */
   int32_t cluster;       /* CTAs sharing one row: 1, 2, 4, 8 or 16             */
-  int32_t threads;       /* threads per row group (multiple of 32)             */
+  int32_t threads;       /* threads per CTA (multiple of 32)                   */
   int32_t units;         /* units per thread: 1, 2, 4 (16-byte) or 1, 4, 8 (pairs) */
-  int32_t stages;        /* staged kernel: rows in flight per row group        */
+  int32_t stages;        /* staged kernel: rows in flight per CTA (1..8)        */
   int32_t ctas_per_sm;   /* resident CTAs per SM the grid is sized for         */
   int32_t grid;          /* CTAs launched (output; multiple of cluster)        */
   int32_t vector;        /* output: 1 if 16-byte vector loads are used         */
-  int32_t groups;        /* row groups per CTA, each on its own rows (1..15)   */
 } arnq_plan;
 
 /* Fills *plan with the plan arnq_run would use for these arguments (pointers

@@ -45,7 +45,7 @@ ARNQ_KERNEL_AUTO, ARNQ_KERNEL_DIRECT, ARNQ_KERNEL_STAGED = 0, 1, 2
 class arnq_plan(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in
                 ("kernel", "cluster", "threads", "units", "stages", "ctas_per_sm", "grid",
-                 "vector", "groups")]
+                 "vector")]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -21,8 +21,6 @@ using arnq::KernelFn;
 constexpr size_t kWorkspaceBytes = 256;      // status block, padded
 constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
-constexpr int kMaxSegElems = 16384;          // elements of a row one CTA holds in registers
-constexpr int kMaxGroups = 15;               // named barriers 1..15
 
 // ---------------------------------------------------------------- kernel table
 
@@ -42,13 +40,6 @@ KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt) {
   const int s = arnq::upt_slot(mode, upt);
   if (s < 0 || nout < 1 || nout > 2) return nullptr;
   return table.fn[dt][qdt][arnq::table_index(nout, add, mode, s)];
-}
-
-// mirrors arnq::MaxThreads
-int max_threads(int mode, int upt) {
-  (void)mode;
-  (void)upt;
-  return 512;
 }
 
 // ---------------------------------------------------------------- device info
@@ -212,6 +203,25 @@ struct Launch {
   int smem, seg, units;
 };
 
+int upt_candidate(int mode, int i) {
+  static const int vec[3] = {1, 2, 4}, sca[3] = {1, 4, 8};
+  return mode == arnq::LOAD_SCALAR ? sca[i] : vec[i];
+}
+
+// Shared memory of one CTA: the exchange slots, then (staged) the input ring.
+int smem_bytes(int cl, int threads, int nout, int stages, int stage_bytes) {
+  const arnq::Layout lay = arnq::make_layout(cl * (threads / 32), nout, stages);
+  return lay.ring + stages * stage_bytes;
+}
+
+// CTAs of `fn` resident per SM (from its actual register count and the smem).
+arnq_status occupancy(KernelFn fn, int threads, int smem, int *per_sm) {
+  *per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, fn, threads, smem) != cudaSuccess)
+    return ARNQ_ERR_CUDA;
+  return ARNQ_OK;
+}
+
 arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   DeviceInfo di;
   int dev = 0;
@@ -228,13 +238,29 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   pl->vector = (mode != arnq::LOAD_SCALAR) ? 1 : 0;
   const int U = (mode == arnq::LOAD_SCALAR) ? 2 : 8;
   const int units = static_cast<int>(ceil_div(P.n, U));
-  const int max_seg = kMaxSegElems / U;
+  const int nin = P.add ? 2 : 1;
+  // the most units one CTA can hold (units per thread times the threads allowed,
+  // for the requested units per thread or the best of them)
+  int max_seg = 0;
+  for (int i = 0; i < 3; ++i) {
+    const int c = upt_candidate(mode, i);
+    if (pl->units != 0 && c != pl->units) continue;
+    const int m = c * arnq::max_threads_for(mode, c, nout);
+    if (m > max_seg) max_seg = m;
+  }
+  if (max_seg == 0) return ARNQ_ERR_PLAN;
 
-  // cluster: enough CTAs per row that one CTA's slice fits in registers, then
-  // more CTAs per row while the rows are too few to fill the SMs
+  // cluster: enough CTAs per row that one CTA's slice fits in registers (and,
+  // staged, two stages of it in shared memory), then more CTAs per row while
+  // the rows are too few to fill the SMs
   if (pl->cluster == 0) {
     int cl = 1;
-    while (cl < kMaxCluster && ceil_div(units, cl) > max_seg) cl *= 2;
+    auto too_big = [&](int c) {
+      const int64_t seg = ceil_div(units, c);
+      if (seg > max_seg) return true;
+      return mode == arnq::LOAD_STAGED && 2 * nin * seg * 16 + 8192 > di.smem_per_block_optin;
+    };
+    while (cl < kMaxCluster && too_big(cl)) cl *= 2;
     while (cl < kMaxCluster && P.rows * cl < di.sms && ceil_div(units, 2 * cl) >= 64) cl *= 2;
     pl->cluster = cl;
   }
@@ -242,59 +268,74 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   if (cl != 1 && cl != 2 && cl != 4 && cl != 8 && cl != 16) return ARNQ_ERR_PLAN;
   const int seg = static_cast<int>(ceil_div(units, cl));
   if (seg > max_seg) return ARNQ_ERR_PLAN;
+  const int stage_bytes = nin * seg * 16;
 
-  // units per thread: as many as keep at least two warps per row group
+  // units per thread: of the variants whose threads hold a slice, the one with
+  // the most resident threads per SM, then the most CTAs per SM
   if (pl->units == 0) {
-    const int cands[3] = {mode == arnq::LOAD_SCALAR ? 8 : 4, mode == arnq::LOAD_SCALAR ? 4 : 2, 1};
-    pl->units = 1;
-    for (int c : cands) {
-      const int64_t t = ceil_div(seg, c);
-      if (t >= 64 && t <= max_threads(mode, c)) { pl->units = c; break; }
+    int best = 0, best_thr = -1, best_ctas = -1;
+    for (int i = 0; i < 3; ++i) {
+      const int c = upt_candidate(mode, i);
+      const int t = round_up(static_cast<int>(ceil_div(seg, c)), 32);
+      if (t > arnq::max_threads_for(mode, c, nout)) continue;
+      if (ceil_div(seg, c) < 32 && best != 0) continue;  // no more than a warp's worth idle
+      KernelFn f = lookup(P.dt, P.qdt, nout, P.add, mode, c);
+      if (!f) continue;
+      const int sm = smem_bytes(cl, t, nout, mode == arnq::LOAD_STAGED ? 2 : 0, stage_bytes);
+      if (sm > di.smem_per_block_optin) continue;
+      st = prepare_kernel(f, dev, sm);
+      if (st != ARNQ_OK) return st;
+      int per_sm = 0;
+      st = occupancy(f, t, sm, &per_sm);
+      if (st != ARNQ_OK) return st;
+      if (per_sm < 1) continue;
+      const int thr = per_sm * t;
+      if (thr > best_thr || (thr == best_thr && per_sm > best_ctas)) {
+        best = c;
+        best_thr = thr;
+        best_ctas = per_sm;
+      }
     }
-    if (ceil_div(seg, pl->units) > max_threads(mode, pl->units))
-      pl->units = mode == arnq::LOAD_SCALAR ? 8 : 4;
+    if (best == 0) return ARNQ_ERR_PLAN;
+    pl->units = best;
   }
   if (arnq::upt_slot(mode, pl->units) < 0) return ARNQ_ERR_PLAN;
+  const int tmax = arnq::max_threads_for(mode, pl->units, nout);
   if (pl->threads == 0) {
     pl->threads = round_up(static_cast<int>(ceil_div(seg, pl->units)), 32);
     if (pl->threads < 32) pl->threads = 32;
   }
-  const int tmax = max_threads(mode, pl->units);
   if (pl->threads % 32 != 0 || pl->threads > tmax ||
       static_cast<int64_t>(pl->threads) * pl->units < seg)
     return ARNQ_ERR_PLAN;
-  // row groups per CTA: fill the CTA's thread budget, one group per cluster CTA
-  if (pl->groups == 0) {
-    int g = cl > 1 ? 1 : tmax / pl->threads;
-    if (g > kMaxGroups) g = kMaxGroups;
-    const int64_t per_sm_rows = ceil_div(P.rows, di.sms);
-    if (g > per_sm_rows) g = static_cast<int>(per_sm_rows);
-    pl->groups = g < 1 ? 1 : g;
-  }
-  if (pl->groups < 1 || pl->groups > kMaxGroups || (cl > 1 && pl->groups != 1) ||
-      pl->groups * pl->threads > tmax)
-    return ARNQ_ERR_PLAN;
-  const int cta_threads = pl->groups * pl->threads;
-  const int pairs = pl->units * (mode == arnq::LOAD_SCALAR ? 1 : 4);
 
   KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units);
   if (!fn) return ARNQ_ERR_PLAN;
-  const int stage_bytes = (P.add ? 2 : 1) * seg * 16;
-  int smem = arnq::layout_bytes(
-      arnq::make_layout(pl->groups, pl->threads, pairs, nout, cl, 0, 0), pl->groups);
+  int smem = smem_bytes(cl, pl->threads, nout, 0, 0);
   if (mode == arnq::LOAD_STAGED) {
-    if (pl->stages == 0) {  // as deep a ring as the shared memory of one CTA per SM allows
-      int s = kMaxStages;
-      while (s > 1 && arnq::layout_bytes(arnq::make_layout(pl->groups, pl->threads, pairs, nout,
-                                                           cl, s, stage_bytes),
-                                         pl->groups) > di.smem_per_block_optin)
+    if (pl->stages == 0) {
+      // a ring of up to 4 rows, as deep as keeps the CTAs per SM the registers
+      // allow (and at least 2 stages)
+      int per_sm_regs = 0;
+      st = prepare_kernel(fn, dev, smem_bytes(cl, pl->threads, nout, 1, stage_bytes));
+      if (st != ARNQ_OK) return st;
+      st = occupancy(fn, pl->threads, smem_bytes(cl, pl->threads, nout, 1, stage_bytes),
+                     &per_sm_regs);
+      if (st != ARNQ_OK) return st;
+      int s = 4;
+      while (s > 2) {
+        const int sm = smem_bytes(cl, pl->threads, nout, s, stage_bytes);
+        if (sm <= di.smem_per_block_optin &&
+            static_cast<int64_t>(per_sm_regs) * (sm + 1024) <= di.smem_per_sm)
+          break;
+        --s;
+      }
+      while (s > 1 && smem_bytes(cl, pl->threads, nout, s, stage_bytes) > di.smem_per_block_optin)
         --s;
       pl->stages = s;
     }
     if (pl->stages < 1 || pl->stages > kMaxStages) return ARNQ_ERR_PLAN;
-    smem = arnq::layout_bytes(
-        arnq::make_layout(pl->groups, pl->threads, pairs, nout, cl, pl->stages, stage_bytes),
-        pl->groups);
+    smem = smem_bytes(cl, pl->threads, nout, pl->stages, stage_bytes);
   } else {
     pl->stages = 0;
   }
@@ -306,9 +347,8 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   int64_t clusters_fit = 0;
   if (cl == 1) {
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, cta_threads, smem) !=
-        cudaSuccess)
-      return ARNQ_ERR_CUDA;
+    st = occupancy(fn, pl->threads, smem, &per_sm);
+    if (st != ARNQ_OK) return st;
     if (per_sm < 1) return ARNQ_ERR_PLAN;
     if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
     pl->ctas_per_sm = per_sm;
@@ -321,7 +361,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3(cl * 1024, 1, 1);
-    cfg.blockDim = dim3(cta_threads, 1, 1);
+    cfg.blockDim = dim3(pl->threads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
@@ -333,8 +373,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
     clusters_fit = want < nc ? want : nc;
     pl->ctas_per_sm = static_cast<int32_t>(ceil_div(clusters_fit * cl, di.sms));
   }
-  const int64_t clusters_needed = ceil_div(P.rows, pl->groups);
-  const int64_t nclusters = clusters_needed < clusters_fit ? clusters_needed : clusters_fit;
+  const int64_t nclusters = P.rows < clusters_fit ? P.rows : clusters_fit;
   pl->grid = static_cast<int32_t>(nclusters * cl);
   L->fn = fn;
   L->smem = smem;
@@ -375,14 +414,13 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   k.seg_units = L.seg;
   k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0);
   k.stages = plan.stages;
-  k.groups = plan.groups;
   k.eps = P.eps;
   k.inv_n = 1.0 / static_cast<double>(P.n);
 
   cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
   cfg.gridDim = dim3(plan.grid, 1, 1);
-  cfg.blockDim = dim3(plan.threads * plan.groups, 1, 1);
+  cfg.blockDim = dim3(plan.threads, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
   if (plan.cluster > 1) {

@@ -10,33 +10,31 @@
 //                memory with cp.async.bulk (1-D bulk copies completing on an
 //                mbarrier); a ring of `stages` rows keeps HBM reads in flight
 //                while the threads work on the current row.
-// A row is split over a thread-block cluster of `cl` CTAs when it is long or
-// when there are too few rows to fill the SMs; partial sums and maxima are then
-// exchanged through distributed shared memory.  Persistent grid: cluster c
-// handles rows c, c + nclusters, ...
-//
-// A CTA is split into row groups that each work on their own rows and meet
-// only at their own named barrier; the folded parameters live once per CTA in
-// shared memory, so a thread's registers hold just its elements of x.
+// A CTA (or a thread-block cluster of `cl` CTAs, for long rows or too few rows
+// to fill the SMs) takes one row at a time; a thread keeps its elements of x
+// and its folded parameters in registers.  Persistent grid: cluster c handles
+// rows c, c + nclusters, ...  Two barriers per row: after the sum of squares,
+// and after the row maximum.
 //
 // Arithmetic.  The bulk of the work is binary32, two lanes at a time with the
 // sm_100 packed instructions (add/mul/fma.rn.f32x2):
 //   x = RNE16(x1 + x2)                    -> xOut, kept as fp32 in registers
 //   ss = sum x^2                          fp64 (x^2 is exact; the sum agrees with
 //                                         an fp64 evaluation of the definition)
-//   rinv = 1/sqrt(ss/n + eps)             binary32, within 3 ulp
+//   Rms = sqrt(ss/n + eps)                fp64, once per warp; 1/Rms also binary32
 //   input_k = x*rinv*G_k + B_k            G_k = gamma*smooth_k, B_k = beta*smooth_k,
 //                                         exact products of two 16-bit values
-//   amax_k = max |input_k|                binary32 scan; the elements within the
-//                                         error bound of the row maximum are
-//                                         re-evaluated in fp64, so
+//   amax_k = max |input_k|                binary32 scan; each warp re-evaluates in
+//                                         fp64 the elements within the error bound
+//                                         of its own maximum (the row's true
+//                                         maximum is among them), so
 //   scale_k = fp32(amax_k / Q)            equals the fp64 evaluation's scale
 //   t = input_k * (1/scale_k)             rounded half-to-even by adding 1.5*2^23
-// |t - t_exact| <= 7u|t| + 4u|B_k|/scale_k (u = 2^-24).  A code whose binary32
-// quotient lies within that bound of a half-way point is recomputed in fp64 in
-// the definition's order, (x / Rms * gamma + beta) * smooth / scale, so every
-// rounding decision is the one an fp64 evaluation of the definition makes.
-// Nothing here is a contraction: no tensor cores.
+// |t - t_exact| <= 7u|t| + 6u|B_k|/scale_k (u = 2^-24).  A code whose binary32
+// quotient lies within that bound of a half-way point is recomputed in fp64,
+// ((x / Rms) * G_k + B_k) / scale_k, so every rounding decision is the one an
+// fp64 evaluation of the definition makes.  Nothing here is a contraction: no
+// tensor cores.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -61,42 +59,25 @@ enum : int { DEV_TIMEOUT = 11 };
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // Shared-memory layout, sized by the launch (the host computes the same):
-//   params   [NOUT][UPT][W][TG] float4 {G.x, G.y, B.x, B.y}: the folded
-//            parameters of the CTA's columns, one copy shared by all groups
-//   maxb     [NOUT][cl * warps per CTA] floats: set-up reduction of |B|
-//   per row group g (stride `group`):
-//     ss     [cl * warps per group] doubles: partial sums of squares
-//     mx     [NOUT][cl * warps per group] floats: partial binary32 maxima
-//     sc     [2][NOUT] binary32 bit patterns: the scales of the last two rows
-//     abort  int; bars [stages] mbarriers; ring [stages] rows of staged input
+//   ss    [cl * nwarps] doubles: per-warp partial sums of squares of a row
+//   cand  [NOUT][cl * nwarps] doubles: per-warp fp64 row maxima of |input_k|
+//   maxb  [NOUT][cl * nwarps] floats: set-up reduction of the bound on |B_k|
+//   abort int; bars [stages] mbarriers; ring [stages] rows of staged input
 constexpr int kMaxStagesDev = 8;
 struct Layout {
-  int params, maxb, group0, group;       // offsets and the per-group stride
-  int ss, mx, sc, abort, bars, ring;     // offsets within a group
+  int ss, cand, maxb, abort, bars, ring;
 };
-__host__ __device__ inline Layout make_layout(int groups, int tg, int pairs_per_thread, int nout,
-                                              int cl, int stages, int stage_bytes) {
+__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) {
   Layout L;
-  const int nwarps_cta = groups * tg / 32;
-  const int nslots = cl * (tg / 32);
   int off = 0;
-  L.params = off; off += nout * pairs_per_thread * tg * 16;
-  L.maxb = off;   off += nout * cl * nwarps_cta * 4;
-  L.group0 = (off + 127) & ~127;
-  int g = 0;
-  L.ss = g;    g += nslots * 8;
-  L.mx = g;    g += nout * nslots * 4;
-  L.sc = g;    g += 2 * nout * 4;
-  g = (g + 7) & ~7;
-  L.abort = g; g += 8;
-  L.bars = g;  g += stages * 8;
-  L.ring = (g + 127) & ~127;
-  g = L.ring + stages * stage_bytes;
-  L.group = (g + 127) & ~127;
+  L.ss = off;    off += nslots * 8;
+  L.cand = off;  off += nout * nslots * 8;
+  L.maxb = off;  off += nout * nslots * 4;
+  off = (off + 7) & ~7;
+  L.abort = off; off += 8;
+  L.bars = off;  off += stages * 8;
+  L.ring = (off + 127) & ~127;
   return L;
-}
-__host__ __device__ inline int layout_bytes(const Layout &L, int groups) {
-  return L.group0 + groups * L.group;
 }
 
 struct KParams {
@@ -111,8 +92,7 @@ struct KParams {
   int32_t units;              // units per row: ceil(n / U)
   int32_t seg_units;          // units per CTA of a cluster
   int32_t flags;
-  int32_t stages;             // staged kernel: ring depth per row group
-  int32_t groups;             // row groups per CTA (1 when cl > 1)
+  int32_t stages;             // staged kernel: ring depth
   float eps;
   double inv_n;               // 1 / n
 };
@@ -234,43 +214,47 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
-// Threads per CTA: 512, so a thread may use 128 registers -- x for up to 32
-// elements plus the fp64 paths, without spilling.
-template <int MODE, int UPT>
-struct MaxThreads {
-  static constexpr int value = 512;
-};
+// Threads per CTA the register budget allows.  A thread keeps, per element, x
+// and per output G and B: (1 + 2*NOUT) floats.  Up to 48 of them fit the 64
+// registers of a 1024-thread CTA, up to 112 the 128 of 512 threads; more get 255.
+__host__ __device__ constexpr int max_threads_for(int mode, int upt, int nout) {
+  return (upt * (mode == LOAD_SCALAR ? 2 : 8) * (1 + 2 * nout) <= 48)    ? 1024
+         : (upt * (mode == LOAD_SCALAR ? 2 : 8) * (1 + 2 * nout) <= 112) ? 512
+                                                                         : 256;
+}
 
 constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: v + kMagic = RNE(v) + kMagic
 constexpr uint32_t kMagicBits = 0x4B400000u;  // its bit pattern; low bits then hold RNE(v)
 constexpr float kUnit = 5.9604644775390625e-08f;  // 2^-24, binary32 unit roundoff
 
 // Rms(x) = sqrt(ss/n + eps) in fp64, IEEE-rounded operations in the
-// definition's order.
-static __device__ __forceinline__ double rms_exact(double ss, int n, float eps) {
+// definition's order.  Out of line, like the two helpers below: they run for a
+// few elements per row, and inlined copies would crowd the instruction cache.
+static __device__ __noinline__ double rms_exact(double ss, int n, float eps) {
   return __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(n)), static_cast<double>(eps)));
 }
 
 // |input| of one element in fp64 from the folded parameters, which are exact
 // products (G = gamma*smooth, B = beta*smooth fit in binary32): |x/Rms*G + B|.
-static __device__ __forceinline__ double input_abs_folded(float x, float g, float b, double rms) {
+static __device__ __noinline__ double input_abs_exact(float x, float g, float b, double rms) {
   return fabs(__fma_rn(__ddiv_rn(static_cast<double>(x), rms), static_cast<double>(g),
                        static_cast<double>(b)));
 }
 
-// The code of one element decided in fp64 exactly as the definition orders it:
+// The code of column c decided in fp64 in the definition's order:
 // round_half_even((x / Rms * gamma + beta) * smooth / scale), clamped to
-// [-Q, Q]; returned as kMagicBits + code so its low bits pack like the fast path.
+// [-qmax, qmax]; returned as kMagicBits + code so its low bits pack like the
+// binary32 path.  Runs only for codes within the error bound of a half-way point.
 template <class T>
-__device__ __forceinline__ uint32_t code_exact(const uint16_t *gamma, const uint16_t *beta,
-                                            const uint16_t *smooth, int c, float x, double rms,
-                                            float scale, int qmax) {
+static __device__ __noinline__ uint32_t code_exact(const uint16_t *gamma, const uint16_t *beta,
+                                                   const uint16_t *smooth, int c, float x,
+                                                   double rms, float scale, int qmax) {
   int q = 0;
   if (scale != 0.f) {
     double y = __dmul_rn(__ddiv_rn(static_cast<double>(x), rms),
-                         static_cast<double>(Cvt<T>::f1(gamma[c])));
-    if (beta) y = __dadd_rn(y, static_cast<double>(Cvt<T>::f1(beta[c])));
-    if (smooth) y = __dmul_rn(y, static_cast<double>(Cvt<T>::f1(smooth[c])));
+                         static_cast<double>(Cvt<T>::f1(__ldg(gamma + c))));
+    if (beta) y = __dadd_rn(y, static_cast<double>(Cvt<T>::f1(__ldg(beta + c))));
+    if (smooth) y = __dmul_rn(y, static_cast<double>(Cvt<T>::f1(__ldg(smooth + c))));
     q = __double2int_rn(__ddiv_rn(y, static_cast<double>(scale)));
     q = min(max(q, -qmax), qmax);
   }
@@ -289,16 +273,17 @@ __device__ __forceinline__ float rsqrt_refined(float v) {
 __device__ __forceinline__ float warp_max_nonneg(float v) {
   return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(v)));
 }
+__device__ __forceinline__ double warp_max_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
 
 // ---------------------------------------------------------------- row kernel
 
-// A CTA holds `groups` row groups of TG = blockDim / groups threads.  Each group
-// works on its own rows (group id g of cluster c takes rows c*groups + g,
-// + nclusters*groups, ...) and synchronizes only its own threads, with the
-// named barrier 1 + g; a cluster (cl > 1) has one group per CTA and uses the
-// cluster barrier.
 template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD>
-__global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(const KParams p) {
+__global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
+    rows_kernel(const KParams p) {
   using C = Cvt<T>;
   constexpr int U = (MODE == LOAD_SCALAR) ? 2 : 8;  // elements per unit
   constexpr int W = U / 2;                          // element pairs per unit
@@ -306,23 +291,17 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
   constexpr float QF = static_cast<float>(QI);
   constexpr int NIN = ADD ? 2 : 1;                  // staged inputs per row
 
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int nwarps = blockDim.x >> 5;
   cg::cluster_group cluster = cg::this_cluster();
   const int cl = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int64_t cluster_id = blockIdx.x / cl;
   const int64_t nclusters = gridDim.x / cl;
-  const int groups = p.groups;
-  const int TG = static_cast<int>(blockDim.x) / groups;
-  const int tid = threadIdx.x;
-  const int gid = tid / TG;           // row group
-  const int gt = tid - gid * TG;      // thread within the group
-  const int lane = tid & 31;
-  const int gwarp = gt >> 5;
-  const int nwg = TG >> 5;            // warps per group
-  const int nslots = cl * nwg;
-  const int my_slot = rank * nwg + gwarp;
-  const int64_t group_id = cluster_id * groups + gid;
-  const int64_t ngroups = nclusters * groups;
+  const int nslots = cl * nwarps;
+  const int my_slot = rank * nwarps + warp;
   const int n = p.n;
   const bool has_beta = (p.flags & F_BETA) != 0;
   const int ring_depth = (MODE == LOAD_STAGED) ? p.stages : 0;  // stages in the layout
@@ -335,37 +314,34 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
   const uint32_t stage_bytes = NIN * static_cast<uint32_t>(p.seg_units) * 16u;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const Layout lay = make_layout(groups, TG, UPT * W, NOUT, cl, ring_depth, stage_bytes);
-  float4 *params = reinterpret_cast<float4 *>(smem + lay.params);
-  float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);
-  unsigned char *gb = smem + lay.group0 + gid * lay.group;
-  double *ss_slots = reinterpret_cast<double *>(gb + lay.ss);   // [nslots]
-  float *mx_slots = reinterpret_cast<float *>(gb + lay.mx);     // [NOUT][nslots]
-  unsigned *sc_slot = reinterpret_cast<unsigned *>(gb + lay.sc);  // [2][NOUT]
-  int *abort_flag = reinterpret_cast<int *>(gb + lay.abort);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(gb + lay.bars);
-  unsigned char *ring = gb + lay.ring;
+  const Layout lay = make_layout(nslots, NOUT, ring_depth);
+  double *ss_slots = reinterpret_cast<double *>(smem + lay.ss);      // [nslots]
+  double *cand_slots = reinterpret_cast<double *>(smem + lay.cand);  // [NOUT][nslots]
+  float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
+  int *abort_flag = reinterpret_cast<int *>(smem + lay.abort);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
+  unsigned char *ring = smem + lay.ring;
 
-  auto group_sync = [&]() {
-    if (cl > 1) {
-      cluster.sync();
+  auto cta_sync = [&]() {
+    if (cl > 1) cluster.sync(); else __syncthreads();
+  };
+  // lane 0 of each warp writes one value into slot `idx` of every CTA of the cluster
+  auto publish_d = [&](double *slots, int idx, double v) {
+    if (cl == 1) {
+      slots[idx] = v;
     } else {
-      asm volatile("bar.sync %0, %1;" ::"r"(1 + gid), "r"(TG) : "memory");
+      for (int r = 0; r < cl; ++r) cluster.map_shared_rank(slots, r)[idx] = v;
     }
   };
-  // the folded parameters of pair i of this thread's k-th unit, output o
-  auto par = [&](int o, int k, int i) -> float4 {
-    return params[((o * UPT + k) * W + i) * TG + gt];
-  };
 
-  // ---- set-up: fold gamma, beta, smooth into G, B (group 0 writes the shared
-  // copy); every thread keeps the bound on |B| over its own elements
+  // ---- folded parameters for this thread's units: input_k = x*rinv*G_k + B_k
+  float2 G[NOUT][UPT][W], B[NOUT][UPT][W];
   float maxB[NOUT];
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) maxB[o] = 0.f;
 #pragma unroll
   for (int k = 0; k < UPT; ++k) {
-    const int u = seg_begin + gt + k * TG;
+    const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
     const bool ok = u < seg_end;
     uint32_t gw[W], bw[W], sw[NOUT][W];
 #pragma unroll
@@ -411,40 +387,39 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
 #pragma unroll
       for (int o = 0; o < NOUT; ++o) {
         const float2 s2 = p.smooth[o] ? C::f2(sw[o][i]) : make_float2(1.f, 1.f);
-        const float2 G = __fmul2_rn(g2, s2);  // exact: two 8- (or 11-) bit significands
-        const float2 B = __fmul2_rn(b2, s2);
-        maxB[o] = fmaxf(maxB[o], fmaxf(fabsf(B.x), fabsf(B.y)));
-        if (gid == 0) params[((o * UPT + k) * W + i) * TG + gt] = make_float4(G.x, G.y, B.x, B.y);
+        G[o][k][i] = __fmul2_rn(g2, s2);  // exact: two 8- (or 11-) bit significands
+        B[o][k][i] = __fmul2_rn(b2, s2);
+        maxB[o] = fmaxf(maxB[o], fmaxf(fabsf(B[o][k][i].x), fabsf(B[o][k][i].y)));
       }
     }
   }
-  const int nwarps_cta = static_cast<int>(blockDim.x) >> 5;
+
+  // ---- set-up exchange: the row-wide bound on |B_k|; staged ring
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     const float v = warp_max_nonneg(maxB[o]);
     if (lane == 0) {
-      const int slot = o * cl * nwarps_cta + rank * nwarps_cta + (tid >> 5);
       if (cl == 1) {
-        maxb_slots[slot] = v;
+        maxb_slots[o * nslots + warp] = v;
       } else {
-        for (int r = 0; r < cl; ++r) cluster.map_shared_rank(maxb_slots, r)[slot] = v;
+        for (int r = 0; r < cl; ++r)
+          cluster.map_shared_rank(maxb_slots, r)[o * nslots + my_slot] = v;
       }
     }
   }
-  if (gt == 0) {
+  if (tid == 0) {
     *abort_flag = 0;
-    for (int q = 0; q < 2 * NOUT; ++q) sc_slot[q] = 0u;
     if (MODE == LOAD_STAGED) {
       for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
   }
-  if (cl > 1) cluster.sync(); else __syncthreads();
-  float maxBg[NOUT];  // bound on |B| over the whole row
+  cta_sync();
+  float maxBg[NOUT];  // bound on |B_k| over the whole row
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     float m = 0.f;
-    for (int i = lane; i < cl * nwarps_cta; i += 32) m = fmaxf(m, maxb_slots[o * cl * nwarps_cta + i]);
+    for (int i = lane; i < nslots; i += 32) m = fmaxf(m, maxb_slots[o * nslots + i]);
     maxBg[o] = warp_max_nonneg(m);
   }
 
@@ -458,18 +433,17 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
     bulk_g2s(dst, p.x1 + off, seg_bytes, bar, policy);
     if (ADD) bulk_g2s(dst + seg_bytes, p.x2 + off, seg_bytes, bar, policy);
   };
-  if (MODE == LOAD_STAGED && gt == 0 && seg_len > 0) {
+  if (MODE == LOAD_STAGED && tid == 0 && seg_len > 0) {
     policy = policy_evict_first();
     for (int s = 0; s < stages; ++s) {
-      const int64_t row = group_id + s * ngroups;
+      const int64_t row = cluster_id + s * nclusters;
       if (row < p.rows) issue(row, s);
     }
   }
 
   int64_t it = 0;
-  for (int64_t row = group_id; row < p.rows; row += ngroups, ++it) {
+  for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
     const int stage = (MODE == LOAD_STAGED) ? static_cast<int>(it % stages) : 0;
-    const int par2 = static_cast<int>(it & 1);
     bool timed_out = false;
     if (MODE == LOAD_STAGED && seg_len > 0) {
       const uint32_t parity = static_cast<uint32_t>((it / stages) & 1);
@@ -481,7 +455,7 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
     double ss = 0.0;
 #pragma unroll
     for (int k = 0; k < UPT; ++k) {
-      const int u = seg_begin + gt + k * TG;
+      const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
       const bool ok = u < seg_end;
       uint32_t a[W], b[W];
 #pragma unroll
@@ -545,32 +519,31 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
       const double v = warp_sum_d(ss);
       const bool any_to = __any_sync(0xFFFFFFFFu, timed_out);
       if (lane == 0) {
-        if (cl == 1) {
-          ss_slots[gwarp] = v;
-          if (any_to) *abort_flag = 1;
-        } else {
-          for (int r = 0; r < cl; ++r) {
-            cluster.map_shared_rank(ss_slots, r)[my_slot] = v;
-            if (any_to) *cluster.map_shared_rank(abort_flag, r) = 1;
+        publish_d(ss_slots, my_slot, v);
+        if (any_to) {
+          if (cl == 1) {
+            *abort_flag = 1;
+          } else {
+            for (int r = 0; r < cl; ++r) *cluster.map_shared_rank(abort_flag, r) = 1;
           }
         }
       }
     }
-    group_sync();
+    cta_sync();
 
     if (MODE == LOAD_STAGED) {
       if (*abort_flag) {
         // A copy never completed: record it, wait (bounded) for the copies this
-        // group still has in flight, and stop.  Every thread of the group (and
-        // of the cluster) sees the flag after the same barrier.
-        if (gt == 0) {
+        // CTA still has in flight, and stop.  Every CTA of the cluster sees the
+        // flag after the same barrier.
+        if (tid == 0) {
           if (atomicCAS(p.status, 0, DEV_TIMEOUT) == 0) {
             *reinterpret_cast<volatile int64_t *>(p.status + 2) = row;
           }
           if (seg_len > 0) {
             for (int s = 0; s < stages; ++s) {
               const int64_t it2 = it + s;  // the ring's outstanding iterations
-              if (group_id + it2 * ngroups >= p.rows) break;
+              if (cluster_id + it2 * nclusters >= p.rows) break;
               mbar_wait_bounded(smem_addr(&bars[it2 % stages]),
                                 static_cast<uint32_t>((it2 / stages) & 1));
             }
@@ -578,21 +551,19 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
         }
         break;
       }
-      // every thread of the group has read this stage: refill it
-      if (gt == 0 && seg_len > 0) {
-        const int64_t nrow = row + static_cast<int64_t>(stages) * ngroups;
+      // every thread has read this stage: refill it
+      if (tid == 0 && seg_len > 0) {
+        const int64_t nrow = row + static_cast<int64_t>(stages) * nclusters;
         if (nrow < p.rows) issue(nrow, stage);
       }
-    }
-    // every thread read the previous row's scales before this barrier
-    if (gt == 0) {
-#pragma unroll
-      for (int o = 0; o < NOUT; ++o) sc_slot[(par2 ^ 1) * NOUT + o] = 0u;
     }
 
     double ss_row = 0.0;
     for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
     ss_row = warp_sum_d(ss_row);
+    // Rms in fp64 as the definition has it, computed by a lane when it first
+    // needs it; 1/Rms in binary32 for the bulk
+    double rms = -1.0;
     float2 rinv2;
     {
       const float v = __double2float_rn(__fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps)));
@@ -600,8 +571,10 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
       rinv2 = make_float2(r, r);
     }
 
-    // ---- pass 2: binary32 row maxima of |input_k|
-    float m32[NOUT];
+    // ---- pass 2: row maxima of |input_k|.  A binary32 scan; then every element
+    // within the error bound of its warp's maximum is re-evaluated in fp64 (the
+    // row's true maximum is among those of its warp) and the warp's fp64 maximum
+    // is published.
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
       float m = 0.f;
@@ -609,88 +582,57 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
       for (int k = 0; k < UPT; ++k)
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-          const float4 gbv = par(o, k, i);
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
-                                       make_float2(gbv.z, gbv.w));
+          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
           m = fmaxf(m, fmaxf(fabsf(in.x), fabsf(in.y)));
         }
-      m32[o] = m;
-      const float v = warp_max_nonneg(m);
-      if (lane == 0) {
-        if (cl == 1) {
-          mx_slots[o * nslots + gwarp] = v;
-        } else {
-          for (int r = 0; r < cl; ++r) cluster.map_shared_rank(mx_slots, r)[o * nslots + my_slot] = v;
-        }
-      }
-    }
-    // ---- exchange 2: binary32 row maxima
-    group_sync();
-
-    // Every element whose binary32 value is within the error bound of the row
-    // maximum is a candidate for the true maximum (usually exactly one per row).
-    // Candidates are evaluated in fp64 and each offers fp32(|input| / Q); as that
-    // rounding is monotonic, the atomic maximum of the offers (binary32 bit
-    // patterns of non-negative values order as integers) is fp32(amax / Q).
-#pragma unroll
-    for (int o = 0; o < NOUT; ++o) {
-      float g = 0.f;
-      for (int i = lane; i < nslots; i += 32) g = fmaxf(g, mx_slots[o * nslots + i]);
-      g = warp_max_nonneg(g);
-      const float thr = g - 12.f * kUnit * (g + maxBg[o]);
-      if (g > 0.f && m32[o] >= thr) {
-        const double rms = rms_exact(ss_row, n, p.eps);
-        double c64 = 0.0;
+      const float wm = warp_max_nonneg(m);
+      const float thr = wm - 12.f * kUnit * (wm + maxBg[o]);
+      double c64 = 0.0;
+      if (wm > 0.f && m >= thr) {
+        if (rms < 0.0) rms = rms_exact(ss_row, n, p.eps);
 #pragma unroll
         for (int k = 0; k < UPT; ++k)
 #pragma unroll
           for (int i = 0; i < W; ++i) {
-            const float4 gbv = par(o, k, i);
-            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
-                                         make_float2(gbv.z, gbv.w));
+            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
             if (fabsf(in.x) >= thr)
-              c64 = fmax(c64, input_abs_folded(xf[k][i].x, gbv.x, gbv.z, rms));
+              c64 = fmax(c64, input_abs_exact(xf[k][i].x, G[o][k][i].x, B[o][k][i].x, rms));
             if (fabsf(in.y) >= thr)
-              c64 = fmax(c64, input_abs_folded(xf[k][i].y, gbv.y, gbv.w, rms));
+              c64 = fmax(c64, input_abs_exact(xf[k][i].y, G[o][k][i].y, B[o][k][i].y, rms));
           }
-        const unsigned offer =
-            __float_as_uint(__double2float_rn(__ddiv_rn(c64, static_cast<double>(QI))));
-        unsigned *slot = &sc_slot[par2 * NOUT + o];
-        if (cl == 1) {
-          atomicMax(slot, offer);
-        } else {
-          for (int r = 0; r < cl; ++r) atomicMax(cluster.map_shared_rank(slot, r), offer);
-        }
       }
+      c64 = warp_max_d(c64);
+      if (lane == 0) publish_d(cand_slots, o * nslots + my_slot, c64);
     }
-    // ---- exchange 3: the scales
-    group_sync();
+    // ---- exchange 2: fp64 row maxima
+    cta_sync();
 
     // ---- pass 3: quantize (round half to even via the 1.5*2^23 trick) and store.
     // A zero scale gives zero codes; a scale whose reciprocal is not a normal
     // binary32 number sends every code of the row through the fp64 path.
-    double rms_cached = -1.0;
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
-      const float sc = __uint_as_float(sc_slot[par2 * NOUT + o]);
+      double am = 0.0;
+      for (int i = lane; i < nslots; i += 32) am = fmax(am, cand_slots[o * nslots + i]);
+      am = warp_max_d(am);
+      const float sc = __double2float_rn(__ddiv_rn(am, static_cast<double>(QI)));
       const bool tiny = sc != 0.f && sc < 1.1754943508222875e-38f;
       const float r32 = (sc == 0.f || tiny) ? 0.f : __frcp_rn(sc);
+      // |t - t_exact| <= tau for the codes of this thread
       const float tau = 12.f * kUnit * (QF + maxB[o] * r32) + 2.f * kUnit * QF;
       const float lim = tiny ? -1.f : 0.5f - tau;
-      if (gt == 0 && rank == 0) p.scale[o][row] = sc;
+      if (tid == 0 && rank == 0) p.scale[o][row] = sc;
       const float2 r2 = make_float2(r32, r32);
       uint8_t *y = p.y[o];
 #pragma unroll
       for (int k = 0; k < UPT; ++k) {
-        const int u = seg_begin + gt + k * TG;
+        const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
         if (u >= seg_end) continue;
         uint32_t bits[2 * W];  // low bits: the code (two's complement)
         float dmax = 0.f;      // largest |t - RNE(t)| of the unit
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-          const float4 gbv = par(o, k, i);
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
-                                       make_float2(gbv.z, gbv.w));
+          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
           const float2 t = __fmul2_rn(in, r2);
           const float2 m = __fadd2_rn(t, make_float2(kMagic, kMagic));
           const float2 rr = __fadd2_rn(m, make_float2(-kMagic, -kMagic));  // RNE(t), exact
@@ -699,23 +641,19 @@ __global__ void __launch_bounds__(MaxThreads<MODE, UPT>::value) rows_kernel(cons
           bits[2 * i + 1] = __float_as_uint(m.y);
           dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
         }
-        if (dmax > lim) {  // some code is near a half-way point: decide those in fp64
-          if (rms_cached < 0.0) rms_cached = rms_exact(ss_row, n, p.eps);
+        if (dmax > lim) {  // some code of the unit is near a half-way point (rare)
+          if (rms < 0.0) rms = rms_exact(ss_row, n, p.eps);
+          const uint16_t *beta = has_beta ? p.beta : nullptr;
 #pragma unroll
           for (int i = 0; i < W; ++i) {
-            const float4 gbv = par(o, k, i);
-            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), make_float2(gbv.x, gbv.y),
-                                         make_float2(gbv.z, gbv.w));
+            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
             const float2 t = __fmul2_rn(in, r2);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float th = h ? t.y : t.x;
-              const float dv = fabsf(th - rintf(th));
-              if (dv > lim)
-                bits[2 * i + h] = code_exact<T>(p.gamma, has_beta ? p.beta : nullptr,
-                                                p.smooth[o], u * U + 2 * i + h,
-                                                h ? xf[k][i].y : xf[k][i].x, rms_cached, sc, QI);
-            }
+            const int c = U * u + 2 * i;  // column of the pair's first element
+            if (fabsf(t.x - rintf(t.x)) > lim)
+              bits[2 * i] = code_exact<T>(p.gamma, beta, p.smooth[o], c, xf[k][i].x, rms, sc, QI);
+            if (fabsf(t.y - rintf(t.y)) > lim && c + 1 < n)
+              bits[2 * i + 1] =
+                  code_exact<T>(p.gamma, beta, p.smooth[o], c + 1, xf[k][i].y, rms, sc, QI);
           }
         }
         if (MODE != LOAD_SCALAR) {

@@ -1,6 +1,6 @@
 // arnq_table.h -- the table of row-kernel instantiations the host dispatches
-// into, indexed by output count, add / no-add, load mode, units per thread and
-// rows per iteration.  Each (dtype, code type) quarter of the table is
+// into, indexed by output count, add / no-add, load mode and units per
+// thread.  Each (dtype, code type) quarter of the table is
 // instantiated in its own translation unit so they compile in parallel.
 #pragma once
 

@@ -154,5 +154,5 @@ def test_v1_and_no_add_entry_points_validate():
 
 
 def test_plan_struct_layout():
-    assert ctypes.sizeof(A.arnq_plan) == 36
+    assert ctypes.sizeof(A.arnq_plan) == 32
     assert ctypes.sizeof(A.arnq_workspace_status) == 16

@@ -195,15 +195,17 @@ def plan(**kw):
 PLAN_CASES = [
     dict(kernel=A.ARNQ_KERNEL_DIRECT),
     dict(kernel=A.ARNQ_KERNEL_DIRECT, units=2),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, units=1),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, units=4),
     dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=2),
     dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=16),
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=1),
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=2, units=2),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=3, cluster=4),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=2, cluster=8, units=2),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=4, cluster=16),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=5, ctas_per_sm=1),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4, ctas_per_sm=1, units=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=4, units=4),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, units=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, stages=1, cluster=4),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=8, units=2),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=16),
 ]
 
 
@@ -220,7 +222,7 @@ def test_plans(pk, shape):
     compare(g, o, qdt, str(pk))
 
 
-@pytest.mark.parametrize("units,cluster", [(1, 2), (1, 4), (4, 1), (4, 4), (8, 1), (8, 2)])
+@pytest.mark.parametrize("units,cluster", [(1, 4), (1, 8), (4, 1), (4, 4), (8, 1), (8, 2)])
 def test_scalar_plans(units, cluster):
     # n not a multiple of 8 forces 2-element units (1501 pairs per row)
     w = wl.random_case(53, 3002, seed=units * 10 + cluster, beta=True, smooth1=True)
