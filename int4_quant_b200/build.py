@@ -16,9 +16,9 @@ import sys
 PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 SRC_DIR = os.path.join(PKG, "csrc")
-SOURCES = [os.path.join(SRC_DIR, f) for f in (
-    "arnq_api.cu", "arnq_k_bf16_int8.cu", "arnq_k_bf16_int4.cu", "arnq_k_fp16_int8.cu",
-    "arnq_k_fp16_int4.cu")]
+SOURCES = [os.path.join(SRC_DIR, f) for f in ["arnq_api.cu"] + [
+    f"arnq_k_{dt}_{q}{cl}.cu" for dt in ("bf16", "fp16") for q in ("int8", "int4")
+    for cl in ("", "_cl")]]
 DEPS = SOURCES + [os.path.join(SRC_DIR, "arnq_kernels.cuh"), os.path.join(SRC_DIR, "arnq_table.h"),
                   os.path.join(ROOT, "include", "arnq.h")]
 LIB = os.path.join(PKG, "libarnq.so")

@@ -32,14 +32,18 @@ struct KernelTable {
     arnq::fill_table_bf16_int4(fn[0][1]);
     arnq::fill_table_fp16_int8(fn[1][0]);
     arnq::fill_table_fp16_int4(fn[1][1]);
+    arnq::fill_table_bf16_int8_cl(fn[0][0]);
+    arnq::fill_table_bf16_int4_cl(fn[0][1]);
+    arnq::fill_table_fp16_int8_cl(fn[1][0]);
+    arnq::fill_table_fp16_int4_cl(fn[1][1]);
   }
 };
 
-KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt) {
+KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt, int cluster) {
   static const KernelTable table;
   const int s = arnq::upt_slot(mode, upt);
   if (s < 0 || nout < 1 || nout > 2) return nullptr;
-  return table.fn[dt][qdt][arnq::table_index(nout, add, mode, s)];
+  return table.fn[dt][qdt][arnq::table_index(nout, add, mode, s, cluster > 1)];
 }
 
 // ---------------------------------------------------------------- device info
@@ -279,7 +283,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       const int t = round_up(static_cast<int>(ceil_div(seg, c)), 32);
       if (t > arnq::max_threads_for(mode, c, nout)) continue;
       if (ceil_div(seg, c) < 32 && best != 0) continue;  // no more than a warp's worth idle
-      KernelFn f = lookup(P.dt, P.qdt, nout, P.add, mode, c);
+      KernelFn f = lookup(P.dt, P.qdt, nout, P.add, mode, c, cl);
       if (!f) continue;
       const int sm = smem_bytes(cl, t, nout, mode == arnq::LOAD_STAGED ? 2 : 0, stage_bytes);
       if (sm > di.smem_per_block_optin) continue;
@@ -309,7 +313,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       static_cast<int64_t>(pl->threads) * pl->units < seg)
     return ARNQ_ERR_PLAN;
 
-  KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units);
+  KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units, cl);
   if (!fn) return ARNQ_ERR_PLAN;
   int smem = smem_bytes(cl, pl->threads, nout, 0, 0);
   if (mode == arnq::LOAD_STAGED) {

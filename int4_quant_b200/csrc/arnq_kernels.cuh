@@ -10,31 +10,44 @@
 //                memory with cp.async.bulk (1-D bulk copies completing on an
 //                mbarrier); a ring of `stages` rows keeps HBM reads in flight
 //                while the threads work on the current row.
-// A CTA (or a thread-block cluster of `cl` CTAs, for long rows or too few rows
-// to fill the SMs) takes one row at a time; a thread keeps its elements of x
-// and its folded parameters in registers.  Persistent grid: cluster c handles
-// rows c, c + nclusters, ...  Two barriers per row: after the sum of squares,
-// and after the row maximum.
+// A CTA (or, for rows too long for one CTA or too few rows to fill the SMs, a
+// thread-block cluster of CTAs sharing a row through distributed shared memory)
+// takes one row at a time; each thread keeps its elements of x and its folded
+// parameters in registers.  Persistent grid: cluster c handles rows c,
+// c + nclusters, ...  Two barriers per row: after the sum of squares and after
+// the row maximum.
 //
-// Arithmetic.  The bulk of the work is binary32, two lanes at a time with the
-// sm_100 packed instructions (add/mul/fma.rn.f32x2):
-//   x = RNE16(x1 + x2)                    -> xOut, kept as fp32 in registers
-//   ss = sum x^2                          fp64 (x^2 is exact; the sum agrees with
-//                                         an fp64 evaluation of the definition)
-//   Rms = sqrt(ss/n + eps)                fp64, once per warp; 1/Rms also binary32
-//   input_k = x*rinv*G_k + B_k            G_k = gamma*smooth_k, B_k = beta*smooth_k,
-//                                         exact products of two 16-bit values
-//   amax_k = max |input_k|                binary32 scan; each warp re-evaluates in
-//                                         fp64 the elements within the error bound
-//                                         of its own maximum (the row's true
-//                                         maximum is among them), so
-//   scale_k = fp32(amax_k / Q)            equals the fp64 evaluation's scale
-//   t = input_k * (1/scale_k)             rounded half-to-even by adding 1.5*2^23
-// |t - t_exact| <= 7u|t| + 6u|B_k|/scale_k (u = 2^-24).  A code whose binary32
-// quotient lies within that bound of a half-way point is recomputed in fp64,
-// ((x / Rms) * G_k + B_k) / scale_k, so every rounding decision is the one an
-// fp64 evaluation of the definition makes.  Nothing here is a contraction: no
-// tensor cores.
+// Arithmetic of the fast path, binary32 two lanes at a time with the sm_100
+// packed instructions (add/mul/fma.rn.f32x2):
+//   x = RN16(x1 + x2)            add.rn.{bf16,f16}x2 -- the correctly rounded
+//                                sum, which equals rounding the binary32 sum
+//   ss = sum x^2                 fp64 (each x^2 is exact)
+//   1/Rms                        binary32 from ss (within a few ulp)
+//   input_k = x*rinv*G_k + B_k   G_k = gamma*smooth_k, B_k = beta*smooth_k, exact
+//                                products of two 16-bit values
+//   s~_k = max|input_k| / Q      approximate scale
+//   code = RNE(input_k / s~_k)   rounded half-to-even by adding 1.5*2^23
+// The result must be what an fp64 evaluation of the definition gives, with the
+// scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
+// code = RNE(input_k / scale_k).  Two pieces of exact work settle that, both
+// off the fast path and finished one row late, after the next barrier:
+//  * the exact scale: the few elements within the binary32 error bound of the
+//    row maximum (the true maximum is among them) are evaluated in fp64 by the
+//    threads that hold them, and their maximum lands in shared memory;
+//  * the exact codes: |t - t_exact| <= tau for the binary32 quotient t (tau
+//    covers the binary32 error and the distance between s~ and the exact
+//    scale), so a code can differ from the fp64 one only if t lies within tau
+//    of a half-way point.  Such elements (a few per row) have their input
+//    evaluated in fp64 into a two-entry queue per thread; the code is decided
+//    once the exact scale is known.
+// These fp64 evaluations use 1/Rms and 1/scale from Newton steps (a few fp64
+// ulp) instead of divisions: the decisions they settle sit at distances of
+// about the binary32 rounding of the scale (~1e-7 relative) from a half-way
+// point, many orders above fp64 rounding.  A row the queue cannot hold (many
+// exact ties in one thread) or whose sum of squares or scale leaves the normal
+// binary32 range is put on a list and recomputed whole, in fp64 with IEEE
+// divisions in the definition's order, after the CTA's last row.
+// Nothing here is a contraction: no tensor cores.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -58,23 +71,34 @@ enum : int { DEV_TIMEOUT = 11 };
 // A bounded wait gives up after this long (nanoseconds of %globaltimer).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
+// row flags exchanged at the first barrier of the next row
+enum : int { RF_REDO = 1, RF_ABORT = 2 };
+
 // Shared-memory layout, sized by the launch (the host computes the same):
-//   ss    [cl * nwarps] doubles: per-warp partial sums of squares of a row
-//   cand  [NOUT][cl * nwarps] doubles: per-warp fp64 row maxima of |input_k|
-//   maxb  [NOUT][cl * nwarps] floats: set-up reduction of the bound on |B_k|
-//   abort int; bars [stages] mbarriers; ring [stages] rows of staged input
+//   ss    [nslots] doubles: per-warp partial sums (also the exact path's reductions)
+//   wmax  [NOUT][nslots] floats: per-warp binary32 row maxima of |input_k|
+//   maxb  [NOUT][nslots] floats: set-up reduction of the bound on |B_k|
+//   amax  [2][2] u64: fp64 row maxima of |input_k| (double bits), by row parity
+//   flags [2] ints: RF_* of a row, by row parity
+//   redo  count (int64) + kRedoCap row indices (int64): rows to recompute in fp64
+//   bars  [stages] mbarriers; ring [stages] rows of staged input
+// nslots = warps per CTA times CTAs per cluster.
 constexpr int kMaxStagesDev = 8;
+constexpr int kRedoCap = 32;
 struct Layout {
-  int ss, cand, maxb, abort, bars, ring;
+  int ss, wmax, maxb, amax, flags, redo, bars, ring;
 };
 __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) {
   Layout L;
   int off = 0;
   L.ss = off;    off += nslots * 8;
-  L.cand = off;  off += nout * nslots * 8;
+  L.wmax = off;  off += nout * nslots * 4;
   L.maxb = off;  off += nout * nslots * 4;
   off = (off + 7) & ~7;
-  L.abort = off; off += 8;
+  L.amax = off;  off += 4 * 8;
+  L.flags = off; off += 2 * 4;
+  off = (off + 7) & ~7;
+  L.redo = off;  off += (1 + kRedoCap) * 8;
   L.bars = off;  off += stages * 8;
   L.ring = (off + 127) & ~127;
   return L;
@@ -86,7 +110,7 @@ struct KParams {
   uint8_t *y[2];              // per output slot
   float *scale[2];            // per output slot
   uint16_t *x_out;
-  int32_t *status;            // workspace status block (staged kernel only)
+  int32_t *status;            // workspace status block
   int64_t rows;
   int32_t n;                  // row length in elements
   int32_t units;              // units per row: ceil(n / U)
@@ -116,6 +140,15 @@ template <> struct Cvt<Bf16> {
     memcpy(&w, &h, 4);
     return w;
   }
+  // correctly rounded sum of two packed pairs.  The binary32 sum of two bf16
+  // values is exact unless their exponents differ by more than 16, and then the
+  // smaller one is below half an ulp of the result and cannot move a rounding
+  // decision: RN16(a + b) == RN16(RN32(a + b)).
+  static __device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+  }
 };
 template <> struct Cvt<Fp16> {
   static __device__ __forceinline__ float2 f2(uint32_t w) {
@@ -133,6 +166,13 @@ template <> struct Cvt<Fp16> {
     uint32_t w;
     memcpy(&w, &h, 4);
     return w;
+  }
+  // as for bf16: the binary32 sum of two fp16 values is exact unless the
+  // exponents differ by more than 13, when the smaller is below half an ulp.
+  static __device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
   }
 };
 
@@ -214,51 +254,14 @@ __device__ __forceinline__ double warp_sum_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
-// Threads per CTA the register budget allows.  A thread keeps, per element, x
-// and per output G and B: (1 + 2*NOUT) floats.  Up to 48 of them fit the 64
-// registers of a 1024-thread CTA, up to 112 the 128 of 512 threads; more get 255.
-__host__ __device__ constexpr int max_threads_for(int mode, int upt, int nout) {
-  return (upt * (mode == LOAD_SCALAR ? 2 : 8) * (1 + 2 * nout) <= 48)    ? 1024
-         : (upt * (mode == LOAD_SCALAR ? 2 : 8) * (1 + 2 * nout) <= 112) ? 512
-                                                                         : 256;
+__device__ __forceinline__ double warp_max_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
 }
-
-constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: v + kMagic = RNE(v) + kMagic
-constexpr uint32_t kMagicBits = 0x4B400000u;  // its bit pattern; low bits then hold RNE(v)
-constexpr float kUnit = 5.9604644775390625e-08f;  // 2^-24, binary32 unit roundoff
-
-// Rms(x) = sqrt(ss/n + eps) in fp64, IEEE-rounded operations in the
-// definition's order.  Out of line, like the two helpers below: they run for a
-// few elements per row, and inlined copies would crowd the instruction cache.
-static __device__ __noinline__ double rms_exact(double ss, int n, float eps) {
-  return __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(n)), static_cast<double>(eps)));
-}
-
-// |input| of one element in fp64 from the folded parameters, which are exact
-// products (G = gamma*smooth, B = beta*smooth fit in binary32): |x/Rms*G + B|.
-static __device__ __noinline__ double input_abs_exact(float x, float g, float b, double rms) {
-  return fabs(__fma_rn(__ddiv_rn(static_cast<double>(x), rms), static_cast<double>(g),
-                       static_cast<double>(b)));
-}
-
-// The code of column c decided in fp64 in the definition's order:
-// round_half_even((x / Rms * gamma + beta) * smooth / scale), clamped to
-// [-qmax, qmax]; returned as kMagicBits + code so its low bits pack like the
-// binary32 path.  Runs only for codes within the error bound of a half-way point.
-template <class T>
-static __device__ __noinline__ uint32_t code_exact(const uint16_t *gamma, const uint16_t *beta,
-                                                   const uint16_t *smooth, int c, float x,
-                                                   double rms, float scale, int qmax) {
-  int q = 0;
-  if (scale != 0.f) {
-    double y = __dmul_rn(__ddiv_rn(static_cast<double>(x), rms),
-                         static_cast<double>(Cvt<T>::f1(__ldg(gamma + c))));
-    if (beta) y = __dadd_rn(y, static_cast<double>(Cvt<T>::f1(__ldg(beta + c))));
-    if (smooth) y = __dmul_rn(y, static_cast<double>(Cvt<T>::f1(__ldg(smooth + c))));
-    q = __double2int_rn(__ddiv_rn(y, static_cast<double>(scale)));
-    q = min(max(q, -qmax), qmax);
-  }
-  return kMagicBits + static_cast<uint32_t>(q);
+// max over lanes of non-negative floats (their bit patterns order as integers)
+__device__ __forceinline__ float warp_max_nonneg(float v) {
+  return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(v)));
 }
 
 // 1/sqrt(v) in binary32: the hardware estimate refined by one Newton-Raphson
@@ -269,21 +272,178 @@ __device__ __forceinline__ float rsqrt_refined(float v) {
   return r * __fmaf_rn(-h * r, r, 1.5f);
 }
 
-// max over lanes of non-negative floats (their bit patterns order as integers)
-__device__ __forceinline__ float warp_max_nonneg(float v) {
-  return __uint_as_float(__reduce_max_sync(0xFFFFFFFFu, __float_as_uint(v)));
+// Threads per CTA the register budget allows.  A thread keeps, per element, x
+// and per output G and B: (1 + 2*NOUT) floats.  Up to 48 of them fit the 64
+// registers of a 1024-thread CTA, up to 112 the 128 of 512 threads; more get 255.
+__host__ __device__ constexpr int max_threads_for(int mode, int upt, int nout) {
+  return (upt * (mode == LOAD_SCALAR ? 2 : 8) * (1 + 2 * nout) <= 48)    ? 1024
+         : (upt * (mode == LOAD_SCALAR ? 2 : 8) * (1 + 2 * nout) <= 112) ? 512
+                                                                         : 256;
 }
-__device__ __forceinline__ double warp_max_d(double v) {
+
+constexpr float kMagic = 12582912.0f;        // 1.5 * 2^23: v + kMagic = RNE(v) + kMagic
+constexpr float kUnit = 5.9604644775390625e-08f;  // 2^-24, binary32 unit roundoff
+
+// ------------------------------------------------------- exact (fp64) pieces
+
+// 1/sqrt(v) in fp64 to a few ulp, for v in the normal binary32 range: the
+// binary32 estimate refined by two Newton steps r' = r + r(1 - v r^2)/2.
+__device__ __forceinline__ double rsqrt64(double v) {
+  double r = static_cast<double>(rsqrtf(__double2float_rn(v)));
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
+  for (int i = 0; i < 2; ++i) {
+    const double e = __fma_rn(-__dmul_rn(v, r), r, 1.0);
+    r = __fma_rn(__dmul_rn(0.5, r), e, r);
+  }
+  return r;
+}
+// 1/s in fp64 to a few ulp, for a normal binary32 s: r' = r + r(1 - s r).
+__device__ __forceinline__ double rcp64(float s) {
+  const double d = static_cast<double>(s);
+  double r = static_cast<double>(__frcp_rn(s));
+#pragma unroll
+  for (int i = 0; i < 2; ++i) r = __fma_rn(r, __fma_rn(-d, r, 1.0), r);
+  return r;
+}
+// round half to even, clamped to [-qmax, qmax]
+__device__ __forceinline__ int code_of_t(double t, int qmax) {
+  return min(max(__double2int_rn(t), -qmax), qmax);
+}
+
+// In the definition's order with IEEE-rounded fp64 operations (the slow path):
+//   Rms = sqrt(ss / n + eps);  y = x / Rms * gamma (+ beta);  input = y (* smooth)
+__device__ __forceinline__ double rms_of(double ss, int n, float eps) {
+  return __dsqrt_rn(__dadd_rn(__ddiv_rn(ss, static_cast<double>(n)), static_cast<double>(eps)));
+}
+
+template <class T>
+__device__ __forceinline__ double input_of(const KParams &p, int o, int c, float x, double rms) {
+  double y = __dmul_rn(__ddiv_rn(static_cast<double>(x), rms),
+                       static_cast<double>(Cvt<T>::f1(__ldg(p.gamma + c))));
+  if (p.flags & F_BETA) y = __dadd_rn(y, static_cast<double>(Cvt<T>::f1(__ldg(p.beta + c))));
+  if (p.smooth[o]) y = __dmul_rn(y, static_cast<double>(Cvt<T>::f1(__ldg(p.smooth[o] + c))));
+  return y;
+}
+
+// round_half_even(input / scale) clamped to [-qmax, qmax]; 0 for a zero scale
+__device__ __forceinline__ int code_of(double in, float scale, int qmax) {
+  if (scale == 0.f) return 0;
+  return code_of_t(__ddiv_rn(in, static_cast<double>(scale)), qmax);
+}
+
+// ---------------------------------------------------------------- exchange
+
+// How the threads sharing a row meet: one CTA, or a cluster through
+// distributed shared memory.
+template <bool CL>
+struct Exchange {
+  cg::cluster_group cluster;
+  int cl, rank;
+  __device__ __forceinline__ Exchange() : cluster(cg::this_cluster()) {
+    if (CL) {
+      cl = static_cast<int>(cluster.num_blocks());
+      rank = static_cast<int>(cluster.block_rank());
+    } else {
+      cl = 1;
+      rank = 0;
+    }
+  }
+  __device__ __forceinline__ void sync() {
+    if (CL) cluster.sync(); else __syncthreads();
+  }
+  template <class V>
+  __device__ __forceinline__ void publish(V *slots, int idx, V v) {  // to every CTA's copy
+    if (CL) {
+      for (int r = 0; r < cl; ++r) cluster.map_shared_rank(slots, r)[idx] = v;
+    } else {
+      slots[idx] = v;
+    }
+  }
+  __device__ __forceinline__ void flag(int *flags, int par, int bits) {
+    if (CL) {
+      for (int r = 0; r < cl; ++r) atomicOr(cluster.map_shared_rank(flags, r) + par, bits);
+    } else {
+      atomicOr(flags + par, bits);
+    }
+  }
+  // the row-maximum slots live in the first CTA of the cluster
+  __device__ __forceinline__ unsigned long long *amax_slot(unsigned long long *amax, int i) {
+    return CL ? cluster.map_shared_rank(amax, 0) + i : amax + i;
+  }
+};
+
+// Whole row in fp64, in the definition's order, by all threads of the CTA (or
+// cluster), reading x back from xOut (or from the inputs when xOut is not
+// written: then x1 and x2 are unchanged).  The slow path for rows the fast
+// path cannot settle; it runs after the CTA's last row, so it takes no
+// registers from the fast path.  Columns [c_begin, c_end) are this CTA's.
+template <class T, bool INT4, int NOUT, bool ADD, bool CL>
+__device__ __forceinline__ void exact_row(const KParams &p, int64_t row, int c_begin, int c_end,
+                                          double *slots, int nslots, int my_slot) {
+  using C = Cvt<T>;
+  constexpr int QI = INT4 ? 7 : 127;
+  Exchange<CL> ex;
+  const int lane = threadIdx.x & 31;
+  const int64_t base = row * p.n;
+  auto x_at = [&](int c) -> float {
+    if (ADD && (p.flags & F_XOUT)) return C::f1(p.x_out[base + c]);
+    if (!ADD) return C::f1(p.x1[base + c]);
+    const float s = C::f1(p.x1[base + c]) + C::f1(p.x2[base + c]);
+    return C::f2(C::pack(s, 0.f)).x;
+  };
+  // every thread gets the sum (or maximum) of v over the row
+  auto reduce = [&](double v, bool is_max) -> double {
+    v = is_max ? warp_max_d(v) : warp_sum_d(v);
+    ex.sync();  // every thread is done with the slots' previous contents
+    if (lane == 0) ex.publish(slots, my_slot, v);
+    ex.sync();
+    double t = 0.0;
+    for (int i = lane; i < nslots; i += 32) t = is_max ? fmax(t, slots[i]) : __dadd_rn(t, slots[i]);
+    return is_max ? warp_max_d(t) : warp_sum_d(t);
+  };
+  const int step = 2 * static_cast<int>(blockDim.x);
+  const int c0 = c_begin + 2 * static_cast<int>(threadIdx.x);  // element pairs (c, c+1)
+  double ss = 0.0;
+  for (int c = c0; c < c_end; c += step) {
+    const double a = x_at(c);
+    ss = __fma_rn(a, a, ss);
+    if (c + 1 < c_end) {
+      const double b = x_at(c + 1);
+      ss = __fma_rn(b, b, ss);
+    }
+  }
+  ss = reduce(ss, false);
+  const double rms = rms_of(ss, p.n, p.eps);
+#pragma unroll
+  for (int o = 0; o < NOUT; ++o) {
+    double m = 0.0;
+    for (int c = c0; c < c_end; c += step) {
+      m = fmax(m, fabs(input_of<T>(p, o, c, x_at(c), rms)));
+      if (c + 1 < c_end) m = fmax(m, fabs(input_of<T>(p, o, c + 1, x_at(c + 1), rms)));
+    }
+    m = reduce(m, true);
+    const float sc = __double2float_rn(__ddiv_rn(m, static_cast<double>(QI)));
+    if (threadIdx.x == 0 && ex.rank == 0) p.scale[o][row] = sc;
+    for (int c = c0; c < c_end; c += step) {
+      const int q0 = code_of(input_of<T>(p, o, c, x_at(c), rms), sc, QI);
+      const int q1 =
+          c + 1 < c_end ? code_of(input_of<T>(p, o, c + 1, x_at(c + 1), rms), sc, QI) : 0;
+      if (INT4) {
+        p.y[o][row * (p.n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+      } else {
+        p.y[o][base + c] = static_cast<uint8_t>(q0);
+        if (c + 1 < c_end) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
+      }
+    }
+  }
+  ex.sync();  // the slots are free again
 }
 
 // ---------------------------------------------------------------- row kernel
 
-template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD>
+template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD, bool CL>
 __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
-    rows_kernel(const KParams p) {
+    rows_kernel(const __grid_constant__ KParams p) {
   using C = Cvt<T>;
   constexpr int U = (MODE == LOAD_SCALAR) ? 2 : 8;  // elements per unit
   constexpr int W = U / 2;                          // element pairs per unit
@@ -291,19 +451,18 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   constexpr float QF = static_cast<float>(QI);
   constexpr int NIN = ADD ? 2 : 1;                  // staged inputs per row
 
+  Exchange<CL> ex;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
   const int warp = tid >> 5;
   const int nwarps = blockDim.x >> 5;
-  cg::cluster_group cluster = cg::this_cluster();
-  const int cl = static_cast<int>(cluster.num_blocks());
-  const int rank = static_cast<int>(cluster.block_rank());
+  const int cl = ex.cl;
+  const int rank = ex.rank;
   const int64_t cluster_id = blockIdx.x / cl;
   const int64_t nclusters = gridDim.x / cl;
   const int nslots = cl * nwarps;
   const int my_slot = rank * nwarps + warp;
   const int n = p.n;
-  const bool has_beta = (p.flags & F_BETA) != 0;
   const int ring_depth = (MODE == LOAD_STAGED) ? p.stages : 0;  // stages in the layout
   const int stages = (MODE == LOAD_STAGED) ? p.stages : 1;      // ring arithmetic
 
@@ -316,23 +475,13 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   extern __shared__ __align__(128) unsigned char smem[];
   const Layout lay = make_layout(nslots, NOUT, ring_depth);
   double *ss_slots = reinterpret_cast<double *>(smem + lay.ss);      // [nslots]
-  double *cand_slots = reinterpret_cast<double *>(smem + lay.cand);  // [NOUT][nslots]
+  float *wmax_slots = reinterpret_cast<float *>(smem + lay.wmax);    // [NOUT][nslots]
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
-  int *abort_flag = reinterpret_cast<int *>(smem + lay.abort);
+  unsigned long long *amax = reinterpret_cast<unsigned long long *>(smem + lay.amax);  // [2][2]
+  int *rflags = reinterpret_cast<int *>(smem + lay.flags);           // [2]
+  int64_t *redo_list = reinterpret_cast<int64_t *>(smem + lay.redo);  // [0] count, then rows
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
   unsigned char *ring = smem + lay.ring;
-
-  auto cta_sync = [&]() {
-    if (cl > 1) cluster.sync(); else __syncthreads();
-  };
-  // lane 0 of each warp writes one value into slot `idx` of every CTA of the cluster
-  auto publish_d = [&](double *slots, int idx, double v) {
-    if (cl == 1) {
-      slots[idx] = v;
-    } else {
-      for (int r = 0; r < cl; ++r) cluster.map_shared_rank(slots, r)[idx] = v;
-    }
-  };
 
   // ---- folded parameters for this thread's units: input_k = x*rinv*G_k + B_k
   float2 G[NOUT][UPT][W], B[NOUT][UPT][W];
@@ -354,7 +503,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       if (MODE != LOAD_SCALAR) {
         const uint4 g = ld_param16(p.gamma + static_cast<int64_t>(u) * 8);
         gw[0] = g.x; gw[1] = g.y; gw[2] = g.z; gw[3] = g.w;
-        if (has_beta) {
+        if (p.flags & F_BETA) {
           const uint4 b = ld_param16(p.beta + static_cast<int64_t>(u) * 8);
           bw[0] = b.x; bw[1] = b.y; bw[2] = b.z; bw[3] = b.w;
         }
@@ -370,7 +519,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
         const bool two = j + 1 < n;
         gw[0] = static_cast<uint32_t>(__ldg(p.gamma + j)) |
                 (two ? static_cast<uint32_t>(__ldg(p.gamma + j + 1)) << 16 : 0u);
-        if (has_beta)
+        if (p.flags & F_BETA)
           bw[0] = static_cast<uint32_t>(__ldg(p.beta + j)) |
                   (two ? static_cast<uint32_t>(__ldg(p.beta + j + 1)) << 16 : 0u);
 #pragma unroll
@@ -394,27 +543,20 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     }
   }
 
-  // ---- set-up exchange: the row-wide bound on |B_k|; staged ring
+  // ---- set-up exchange: the row-wide bound on |B_k|; shared state; staged ring
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     const float v = warp_max_nonneg(maxB[o]);
-    if (lane == 0) {
-      if (cl == 1) {
-        maxb_slots[o * nslots + warp] = v;
-      } else {
-        for (int r = 0; r < cl; ++r)
-          cluster.map_shared_rank(maxb_slots, r)[o * nslots + my_slot] = v;
-      }
-    }
+    if (lane == 0) ex.publish(maxb_slots, o * nslots + my_slot, v);
   }
-  if (tid == 0) {
-    *abort_flag = 0;
-    if (MODE == LOAD_STAGED) {
-      for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
-      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
+  if (tid < 4) amax[tid] = 0ull;
+  if (tid < 2) rflags[tid] = 0;
+  if (tid == 0) redo_list[0] = 0;
+  if (MODE == LOAD_STAGED && tid == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  cta_sync();
+  ex.sync();
   float maxBg[NOUT];  // bound on |B_k| over the whole row
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
@@ -441,8 +583,54 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     }
   }
 
+  // ---- the previous row's unfinished business, settled after the next barrier
+  int64_t prev_row = -1;
+  bool redo = false;        // this thread cannot settle the current row
+  int qn = 0;               // near-tie queue of the current row: fp64 input, column
+  double qi0 = 0.0, qi1 = 0.0;
+  uint32_t qe0 = 0, qe1 = 0;  // column | output << 31
+  const double inv_q = 1.0 / static_cast<double>(QI);
+  // Run by every thread right after a first barrier; fl = the flags of the
+  // previous row, pp = its parity.
+  auto settle_prev = [&](int fl, int pp) {
+    if (fl & RF_REDO) {
+      if (tid == 0) {
+        const int64_t k = redo_list[0]++;
+        if (k < kRedoCap) redo_list[1 + k] = prev_row;
+      }
+    } else {
+      float sc[2] = {0.f, 0.f};
+#pragma unroll
+      for (int o = 0; o < NOUT; ++o) {
+        const double m =
+            __longlong_as_double(static_cast<long long>(*ex.amax_slot(amax, pp * 2 + o)));
+        sc[o] = __double2float_rn(__dmul_rn(m, inv_q));
+        if (tid == 0 && rank == 0) p.scale[o][prev_row] = sc[o];
+      }
+      if (qn > 0) {  // rare: decide the queued codes with the exact scale
+        for (int e = 0; e < 2; ++e) {
+          if (e >= qn) break;
+          const uint32_t ent = e == 0 ? qe0 : qe1;
+          const int o = static_cast<int>(ent >> 31);
+          const int c = static_cast<int>(ent & 0x7FFFFFFFu);
+          const float so = o == 0 ? sc[0] : sc[1];
+          const int q = so == 0.f ? 0 : code_of_t(__dmul_rn(e == 0 ? qi0 : qi1, rcp64(so)), QI);
+          if (INT4) {
+            uint8_t *bp = p.y[o] + prev_row * (n / 2) + c / 2;
+            const int sh = (c & 1) * 4;
+            *bp = static_cast<uint8_t>((*bp & ~(0xF << sh)) | ((q & 0xF) << sh));
+          } else {
+            p.y[o][prev_row * n + c] = static_cast<uint8_t>(q);
+          }
+        }
+      }
+    }
+    qn = 0;
+  };
+
   int64_t it = 0;
   for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
+    const int par = static_cast<int>(it & 1);
     const int stage = (MODE == LOAD_STAGED) ? static_cast<int>(it % stages) : 0;
     bool timed_out = false;
     if (MODE == LOAD_STAGED && seg_len > 0) {
@@ -450,7 +638,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), parity);
     }
 
-    // ---- pass 1: x = RNE16(x1 + x2) (or x1), xOut, sum of squares (fp64)
+    // ---- pass 1: x = RN16(x1 + x2) (or x1), xOut, sum of squares (fp64)
     float2 xf[UPT][W];
     double ss = 0.0;
 #pragma unroll
@@ -491,12 +679,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       uint32_t xo[W];
 #pragma unroll
       for (int i = 0; i < W; ++i) {
-        if (ADD) {
-          const float2 sum = __fadd2_rn(C::f2(a[i]), C::f2(b[i]));  // binary32 add
-          xo[i] = C::pack(sum.x, sum.y);                            // RNE to 16 bits
-        } else {
-          xo[i] = a[i];
-        }
+        xo[i] = ADD ? C::add2(a[i], b[i]) : a[i];
         const float2 xv = C::f2(xo[i]);  // the x that is normalised
         xf[k][i] = xv;
         ss = __fma_rn(static_cast<double>(xv.x), static_cast<double>(xv.x), ss);
@@ -514,25 +697,22 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       }
     }
 
-    // ---- exchange 1: sum of squares over the row (and the abort flag)
+    // ---- exchange 1: sum of squares; the previous row's flags
     {
       const double v = warp_sum_d(ss);
       const bool any_to = __any_sync(0xFFFFFFFFu, timed_out);
+      const bool any_redo = __any_sync(0xFFFFFFFFu, redo);
       if (lane == 0) {
-        publish_d(ss_slots, my_slot, v);
-        if (any_to) {
-          if (cl == 1) {
-            *abort_flag = 1;
-          } else {
-            for (int r = 0; r < cl; ++r) *cluster.map_shared_rank(abort_flag, r) = 1;
-          }
-        }
+        ex.publish(ss_slots, my_slot, v);
+        if (any_to || any_redo)
+          ex.flag(rflags, par ^ 1, (any_to ? RF_ABORT : 0) | (any_redo ? RF_REDO : 0));
       }
     }
-    cta_sync();
+    ex.sync();
+    const int fl = rflags[par ^ 1];
 
     if (MODE == LOAD_STAGED) {
-      if (*abort_flag) {
+      if (fl & RF_ABORT) {
         // A copy never completed: record it, wait (bounded) for the copies this
         // CTA still has in flight, and stop.  Every CTA of the cluster sees the
         // flag after the same barrier.
@@ -549,6 +729,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
             }
           }
         }
+        prev_row = -1;
         break;
       }
       // every thread has read this stage: refill it
@@ -561,20 +742,20 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     double ss_row = 0.0;
     for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
     ss_row = warp_sum_d(ss_row);
-    // Rms in fp64 as the definition has it, computed by a lane when it first
-    // needs it; 1/Rms in binary32 for the bulk
-    double rms = -1.0;
+    // v = ss/n + eps; 1/sqrt(v) in binary32 for the bulk, in fp64 when needed
+    const double v64 = __fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps));
+    const float v32 = __double2float_rn(v64);
     float2 rinv2;
     {
-      const float v = __double2float_rn(__fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps)));
-      const float r = rsqrt_refined(v);
+      const float r = rsqrt_refined(v32);
       rinv2 = make_float2(r, r);
     }
+    if (prev_row >= 0) settle_prev(fl, par ^ 1);
+    // outside the normal binary32 range the bulk arithmetic is not trusted
+    redo = !(v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f);
 
-    // ---- pass 2: row maxima of |input_k|.  A binary32 scan; then every element
-    // within the error bound of its warp's maximum is re-evaluated in fp64 (the
-    // row's true maximum is among those of its warp) and the warp's fp64 maximum
-    // is published.
+    // ---- pass 2: binary32 row maxima of |input_k|
+    float m32[NOUT];
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
       float m = 0.f;
@@ -585,43 +766,52 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
           const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
           m = fmaxf(m, fmaxf(fabsf(in.x), fabsf(in.y)));
         }
+      m32[o] = m;
       const float wm = warp_max_nonneg(m);
-      const float thr = wm - 12.f * kUnit * (wm + maxBg[o]);
-      double c64 = 0.0;
-      if (wm > 0.f && m >= thr) {
-        if (rms < 0.0) rms = rms_exact(ss_row, n, p.eps);
+      if (lane == 0) ex.publish(wmax_slots, o * nslots + my_slot, wm);
+    }
+    // ---- exchange 2: row maxima.  The previous row's slots are free now.
+    ex.sync();
+    if (tid < NOUT && rank == 0) amax[(par ^ 1) * 2 + tid] = 0ull;
+    if (tid == 0) rflags[par ^ 1] = 0;
+
+    // ---- pass 3: quantize with the approximate scale s~ = max / Q (rounded half
+    // to even via the 1.5*2^23 trick); queue the codes near a half-way point
+#pragma unroll
+    for (int o = 0; o < NOUT; ++o) {
+      float gm = 0.f;
+      for (int i = lane; i < nslots; i += 32) gm = fmaxf(gm, wmax_slots[o * nslots + i]);
+      gm = warp_max_nonneg(gm);
+      const float sa = __fdiv_rn(gm, QF);
+      const bool normal = sa >= 1.1754943508222875e-38f;
+      if (sa != 0.f && !normal) redo = true;  // 1/s~ would overflow: exact path
+      const float r32 = normal ? __frcp_rn(sa) : 0.f;
+      // candidates for the row maximum: within the binary32 error of it
+      const float thr = gm - 12.f * kUnit * (gm + maxBg[o]);
+      if (gm > 0.f && m32[o] >= thr && !redo) {  // about one thread per row
+        const double ri = rsqrt64(v64);
+        double c64 = 0.0;
 #pragma unroll
         for (int k = 0; k < UPT; ++k)
 #pragma unroll
           for (int i = 0; i < W; ++i) {
             const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
-            if (fabsf(in.x) >= thr)
-              c64 = fmax(c64, input_abs_exact(xf[k][i].x, G[o][k][i].x, B[o][k][i].x, rms));
-            if (fabsf(in.y) >= thr)
-              c64 = fmax(c64, input_abs_exact(xf[k][i].y, G[o][k][i].y, B[o][k][i].y, rms));
-          }
-      }
-      c64 = warp_max_d(c64);
-      if (lane == 0) publish_d(cand_slots, o * nslots + my_slot, c64);
-    }
-    // ---- exchange 2: fp64 row maxima
-    cta_sync();
-
-    // ---- pass 3: quantize (round half to even via the 1.5*2^23 trick) and store.
-    // A zero scale gives zero codes; a scale whose reciprocal is not a normal
-    // binary32 number sends every code of the row through the fp64 path.
 #pragma unroll
-    for (int o = 0; o < NOUT; ++o) {
-      double am = 0.0;
-      for (int i = lane; i < nslots; i += 32) am = fmax(am, cand_slots[o * nslots + i]);
-      am = warp_max_d(am);
-      const float sc = __double2float_rn(__ddiv_rn(am, static_cast<double>(QI)));
-      const bool tiny = sc != 0.f && sc < 1.1754943508222875e-38f;
-      const float r32 = (sc == 0.f || tiny) ? 0.f : __frcp_rn(sc);
-      // |t - t_exact| <= tau for the codes of this thread
-      const float tau = 12.f * kUnit * (QF + maxB[o] * r32) + 2.f * kUnit * QF;
-      const float lim = tiny ? -1.f : 0.5f - tau;
-      if (tid == 0 && rank == 0) p.scale[o][row] = sc;
+            for (int h = 0; h < 2; ++h) {
+              if (fabsf(h ? in.y : in.x) >= thr) {
+                const double xr = __dmul_rn(static_cast<double>(h ? xf[k][i].y : xf[k][i].x), ri);
+                c64 = fmax(c64, fabs(__fma_rn(xr, static_cast<double>(h ? G[o][k][i].y : G[o][k][i].x),
+                                              static_cast<double>(h ? B[o][k][i].y : B[o][k][i].x))));
+              }
+            }
+          }
+        atomicMax(ex.amax_slot(amax, par * 2 + o),
+                  static_cast<unsigned long long>(__double_as_longlong(c64)));
+      }
+      // |t - t_exact| <= tau: the binary32 error of t (12u(Q + |B| r) + 2uQ) plus
+      // the distance between s~ and the exact scale (10uQ + 6u maxB r)
+      const float tau = 24.f * kUnit * QF + 18.f * kUnit * maxBg[o] * r32;
+      const float lim = 0.5f - tau;
       const float2 r2 = make_float2(r32, r32);
       uint8_t *y = p.y[o];
 #pragma unroll
@@ -641,19 +831,33 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
           bits[2 * i + 1] = __float_as_uint(m.y);
           dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
         }
-        if (dmax > lim) {  // some code of the unit is near a half-way point (rare)
-          if (rms < 0.0) rms = rms_exact(ss_row, n, p.eps);
-          const uint16_t *beta = has_beta ? p.beta : nullptr;
+        if (dmax > lim && !redo) {  // some code of the unit is near a half-way point (rare)
+          const double ri = rsqrt64(v64);
 #pragma unroll
           for (int i = 0; i < W; ++i) {
             const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
             const float2 t = __fmul2_rn(in, r2);
-            const int c = U * u + 2 * i;  // column of the pair's first element
-            if (fabsf(t.x - rintf(t.x)) > lim)
-              bits[2 * i] = code_exact<T>(p.gamma, beta, p.smooth[o], c, xf[k][i].x, rms, sc, QI);
-            if (fabsf(t.y - rintf(t.y)) > lim && c + 1 < n)
-              bits[2 * i + 1] =
-                  code_exact<T>(p.gamma, beta, p.smooth[o], c + 1, xf[k][i].y, rms, sc, QI);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const float th = h ? t.y : t.x;
+              const int c = U * u + 2 * i + h;
+              if (fabsf(th - rintf(th)) > lim && c < n) {
+                const uint32_t e = static_cast<uint32_t>(c) | (static_cast<uint32_t>(o) << 31);
+                const double xr = __dmul_rn(static_cast<double>(h ? xf[k][i].y : xf[k][i].x), ri);
+                const double in64 = __fma_rn(xr, static_cast<double>(h ? G[o][k][i].y : G[o][k][i].x),
+                                             static_cast<double>(h ? B[o][k][i].y : B[o][k][i].x));
+                if (qn == 0) {
+                  qe0 = e;
+                  qi0 = in64;
+                } else if (qn == 1) {
+                  qe1 = e;
+                  qi1 = in64;
+                } else {
+                  redo = true;
+                }
+                ++qn;
+              }
+            }
           }
         }
         if (MODE != LOAD_SCALAR) {
@@ -683,9 +887,33 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
         }
       }
     }
+    prev_row = row;
+  }
+
+  // ---- settle the last row
+  if (prev_row >= 0) {
+    const int par = static_cast<int>(it & 1);
+    const bool any_redo = __any_sync(0xFFFFFFFFu, redo);
+    if (lane == 0 && any_redo) ex.flag(rflags, par ^ 1, RF_REDO);
+    ex.sync();
+    settle_prev(rflags[par ^ 1], par ^ 1);
+    // ---- rows for the slow path: the listed ones, or (list overflowed) all
+    ex.sync();
+    const int64_t nredo = redo_list[0];
+    if (nredo > 0) {
+      const int c_begin = seg_begin * U, c_end = min(seg_end * U, n);
+      if (nredo <= kRedoCap) {
+        for (int64_t i = 0; i < nredo; ++i)
+          exact_row<T, INT4, NOUT, ADD, CL>(p, redo_list[1 + i], c_begin, c_end, ss_slots, nslots,
+                                            my_slot);
+      } else {
+        for (int64_t r = cluster_id; r < p.rows; r += nclusters)
+          exact_row<T, INT4, NOUT, ADD, CL>(p, r, c_begin, c_end, ss_slots, nslots, my_slot);
+      }
+    }
   }
   // no CTA leaves while a peer may still touch its shared memory
-  if (cl > 1) cluster.sync();
+  if (CL) ex.sync();
 }
 
 }  // namespace arnq
