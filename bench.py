@@ -262,6 +262,21 @@ def run_reference(args, w, on1, on2):
 
 # ---------------------------------------------------------------- our arm
 
+def max_over_ranks(value_ms, dist, device):
+    """The slowest rank's time: every rank passes its own and gets the max."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value_ms)
+    import torch
+    t = torch.tensor([float(value_ms)], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_step, steps, world, total_ms):
+    """Whole-job throughput: every rank moves bytes_per_step per step (replicas)."""
+    return bytes_per_step * steps * world / (total_ms / 1e3) / 1e9
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -370,13 +385,10 @@ def main():
     wsh = ws[:16].cpu().numpy().view(np.int32)
     if wsh[0] != 0:
         raise RuntimeError(f"kernel reported device status {wsh[0]}")
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     nbytes = workload_bytes(w, on1, on2)
-    value = nbytes * K * world / (total_ms / 1e3) / 1e9
+    value = job_gbs(nbytes, K, world, total_ms)
     rows_per_s = w.rows * K * world / (total_ms / 1e3)
     mean_launch_ms = statistics.fmean(launch_ms)
     achieved = nbytes / (mean_launch_ms / 1e3) / 1e9
@@ -418,11 +430,8 @@ def main():
     e_end.record(stream)
     barrier()
     e2e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e_value = nbytes * e2e_steps * world / (e2e_ms / 1e3) / 1e9
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    e2e_value = job_gbs(nbytes, e2e_steps, world, e2e_ms)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -318,22 +318,9 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   int smem = smem_bytes(cl, pl->threads, nout, 0, 0);
   if (mode == arnq::LOAD_STAGED) {
     if (pl->stages == 0) {
-      // a ring of up to 4 rows, as deep as keeps the CTAs per SM the registers
-      // allow (and at least 2 stages)
-      int per_sm_regs = 0;
-      st = prepare_kernel(fn, dev, smem_bytes(cl, pl->threads, nout, 1, stage_bytes));
-      if (st != ARNQ_OK) return st;
-      st = occupancy(fn, pl->threads, smem_bytes(cl, pl->threads, nout, 1, stage_bytes),
-                     &per_sm_regs);
-      if (st != ARNQ_OK) return st;
-      int s = 4;
-      while (s > 2) {
-        const int sm = smem_bytes(cl, pl->threads, nout, s, stage_bytes);
-        if (sm <= di.smem_per_block_optin &&
-            static_cast<int64_t>(per_sm_regs) * (sm + 1024) <= di.smem_per_sm)
-          break;
-        --s;
-      }
+      // two rows in flight per CTA (measured best on 4096..16384-element rows;
+      // deeper rings cost CTAs per SM), one if two do not fit
+      int s = 2;
       while (s > 1 && smem_bytes(cl, pl->threads, nout, s, stage_bytes) > di.smem_per_block_optin)
         --s;
       pl->stages = s;
