@@ -84,16 +84,17 @@ def measured_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the device code (the kernel template and its instantiation table)."""
     h = hashlib.sha256()
-    for f in ("int4_quant_b200/csrc/arnq_kernels.cuh", "int4_quant_b200/csrc/arnq_api.cu"):
+    for f in ("int4_quant_b200/csrc/arnq_kernels.cuh", "int4_quant_b200/csrc/arnq_table.h"):
         with open(os.path.join(ROOT, f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload_name):
+def recorded_traffic(workload_name, plan=None):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
-    the current kernel source; else None."""
+    the current kernel source with the same launch plan; else None."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
@@ -102,6 +103,8 @@ def recorded_traffic(workload_name):
         return None
     e = d.get(workload_name)
     if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    if plan is not None and e.get("plan") is not None and e["plan"] != plan:
         return None
     return e.get("dram_bytes_per_launch")
 
@@ -476,7 +479,7 @@ def main():
             "peak": peak,
             "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": recorded_traffic(w.name),
+            "traffic": recorded_traffic(w.name, plan.as_dict()),
             "peak_kind": peak_kind,
             "kernel": "arnq::rows_kernel",
             "mean_launch_us": mean_launch_ms * 1e3,

@@ -208,6 +208,34 @@ ARNQ_API arnq_status arnq_run_planned(const void *x1, const void *x2, const void
                              void *x_out, void *workspace, size_t workspace_bytes, void *stream,
                              const arnq_plan *plan);
 
+/* ---- no-allocation variant ----------------------------------------------
+ *
+ * The paper has no counterpart: the pages' two-phase call always takes a
+ * caller-allocated workspace.  This entry point is arnq_run with the workspace
+ * replaced by a file-scope device array inside the library
+ * (ARNQ_STATIC_SCRATCH_BYTES per device), so a caller that cannot allocate
+ * (no allocator at hand, a fixed memory budget) still gets the operator.
+ * It allocates nothing: no cudaMalloc / cudaFree and no allocating library
+ * routine.  Arguments and results are those of arnq_run; in addition
+ *   - ARNQ_ERR_WORKSPACE if the problem needs more scratch than
+ *     ARNQ_STATIC_SCRATCH_BYTES (arnq_workspace_size larger than the array);
+ *   - ARNQ_ERR_CUDA if the array's device address cannot be obtained
+ *     (cudaGetSymbolAddress fails) or its set-up fails.
+ * The status block at the start of the array must be zero when a kernel
+ * starts: every call clears it first (an async memset on `stream`).  The first
+ * call on each device does set-up (looks up the array's address and zeroes
+ * it, synchronously): make it before any stream capture.  The array is shared
+ * by every call on a device: calls that overlap (other streams, other host
+ * threads) race on it; serialise them.  A device-side timeout status lands in
+ * the array and is not readable from the host: use arnq_run with a workspace
+ * where that status matters. */
+#define ARNQ_STATIC_SCRATCH_BYTES 4096
+ARNQ_API arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *gamma,
+                                    const void *beta, const void *smooth1, const void *smooth2,
+                                    int64_t rows, int64_t n, arnq_dtype dt, float eps,
+                                    int out_mask, arnq_qdtype qdt, void *y1, float *scale1,
+                                    void *y2, float *scale2, void *x_out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

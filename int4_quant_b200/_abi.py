@@ -40,6 +40,7 @@ ARNQ_MASK_Y1, ARNQ_MASK_Y2 = 1, 2
 ARNQ_MAX_N = 131072
 
 ARNQ_KERNEL_AUTO, ARNQ_KERNEL_DIRECT, ARNQ_KERNEL_STAGED = 0, 1, 2
+ARNQ_STATIC_SCRATCH_BYTES = 4096
 
 
 class arnq_plan(ctypes.Structure):
@@ -80,6 +81,8 @@ _SIGS = {
                        _i32),
     "arnq_run_planned": ([_p, _p, _p, _p, _p, _p, _i64, _i64, _i32, _f32, _i32, _i32, _p, _p, _p,
                           _p, _p, _p, _sz, _p, _p], _i32),
+    "arnq_run_static_scratch": ([_p, _p, _p, _p, _p, _p, _i64, _i64, _i32, _f32, _i32, _i32, _p, _p,
+                                 _p, _p, _p, _p], _i32),
 }
 
 
@@ -197,3 +200,12 @@ def arnq_run_planned(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, eps, ou
                                   _ptr(scale2), _ptr(x_out), _ptr(workspace),
                                   int(workspace_bytes), _stream(stream),
                                   ctypes.addressof(plan))
+
+
+def arnq_run_static_scratch(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, eps, out_mask, qdt,
+                            y1, scale1, y2, scale2, x_out, stream) -> int:
+    return lib().arnq_run_static_scratch(_ptr(x1), _ptr(x2), _ptr(gamma), _ptr(beta),
+                                         _ptr(smooth1), _ptr(smooth2), int(rows), int(n), int(dt),
+                                         float(eps), int(out_mask), int(qdt), _ptr(y1),
+                                         _ptr(scale1), _ptr(y2), _ptr(scale2), _ptr(x_out),
+                                         _stream(stream))

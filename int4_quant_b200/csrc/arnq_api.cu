@@ -438,6 +438,27 @@ Problem problem(const void *x1, const void *x2, const void *gamma, const void *b
   return P;
 }
 
+// ---------------------------------------------------------------- static scratch
+
+// The no-allocation entry point's scratch: one array per device, in the
+// library's own device memory.  Its address is looked up once per device.
+static __device__ __align__(256) unsigned char g_static_scratch[ARNQ_STATIC_SCRATCH_BYTES];
+void *g_scratch_addr[kMaxDevices];
+
+arnq_status static_scratch(void **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ARNQ_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mu);
+  if (!g_scratch_addr[dev]) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return ARNQ_ERR_CUDA;
+    if (cudaMemset(p, 0, ARNQ_STATIC_SCRATCH_BYTES) != cudaSuccess) return ARNQ_ERR_CUDA;
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return ARNQ_OK;
+}
+
 arnq_status run_common(Problem P, int out_mask, void *workspace, size_t workspace_bytes,
                        void *stream, const arnq_plan *plan) {
   arnq_status st = validate(P, out_mask, workspace, workspace_bytes);
@@ -543,6 +564,39 @@ arnq_status arnq_make_plan(const void *x1, const void *x2, const void *gamma, co
   if (st != ARNQ_OK) return st;
   Launch L;
   return make_plan(P, plan, &L);
+}
+
+arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *gamma,
+                                    const void *beta, const void *smooth1, const void *smooth2,
+                                    int64_t rows, int64_t n, arnq_dtype dt, float eps,
+                                    int out_mask, arnq_qdtype qdt, void *y1, float *scale1,
+                                    void *y2, float *scale2, void *x_out, void *stream) {
+  Problem P = problem(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, eps, qdt, y1, scale1, y2,
+                      scale2, x_out, true);
+  // the host-side checks first: a rejected call touches no device
+  static_assert(kWorkspaceBytes <= ARNQ_STATIC_SCRATCH_BYTES, "scratch too small");
+  arnq_status st = check_shape(P.rows, P.n, P.dt, P.qdt, P.eps);
+  if (st != ARNQ_OK) return st;
+  size_t need = 0;
+  st = arnq_workspace_size(rows, n, dt, qdt, out_mask, smooth1 != nullptr, smooth2 != nullptr,
+                           &need);
+  if (st != ARNQ_OK) return st;
+  if (need > ARNQ_STATIC_SCRATCH_BYTES) return ARNQ_ERR_WORKSPACE;
+  {
+    // every other argument check, with an aligned stand-in for the scratch
+    // address (validate only inspects the pointer's value)
+    Problem Q = P;
+    st = validate(Q, out_mask, reinterpret_cast<void *>(static_cast<uintptr_t>(256)),
+                  ARNQ_STATIC_SCRATCH_BYTES);
+    if (st != ARNQ_OK) return st;
+  }
+  void *scratch = nullptr;
+  st = static_scratch(&scratch);
+  if (st != ARNQ_OK) return st;
+  // the status block must start at zero
+  if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return ARNQ_ERR_CUDA;
+  return run_common(P, out_mask, scratch, ARNQ_STATIC_SCRATCH_BYTES, stream, nullptr);
 }
 
 }  // extern "C"

@@ -156,3 +156,16 @@ def test_v1_and_no_add_entry_points_validate():
 def test_plan_struct_layout():
     assert ctypes.sizeof(A.arnq_plan) == 32
     assert ctypes.sizeof(A.arnq_workspace_status) == 16
+
+
+def test_static_scratch_entry_validates_on_the_host():
+    # rejected before the library touches a device (no set-up, no copy)
+    assert A.arnq_run_static_scratch(None, None, None, None, None, None, 8, 64, 0, 1e-6, -1, 0,
+                                     None, None, None, None, None, None) == A.ARNQ_ERR_NULL_PTR
+    assert A.arnq_run_static_scratch(P["x1"], P["x2"], P["g"], None, None, None, 0, 64, 0, 1e-6,
+                                     -1, 0, P["y1"], P["sc1"], None, None, None,
+                                     None) == A.ARNQ_ERR_EMPTY
+    assert A.arnq_run_static_scratch(P["x1"], P["x2"], P["g"], None, None, P["s2"], 8, 64, 0, 1e-6,
+                                     -1, 0, P["y1"], P["sc1"], None, None, None,
+                                     None) == A.ARNQ_ERR_MASK
+    assert A.ARNQ_STATIC_SCRATCH_BYTES >= A.arnq_workspace_size(8, 64, 0, 0, -1, 0, 0)[1]
