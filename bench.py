@@ -343,14 +343,16 @@ def main():
             y2=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if on2 else None,
             s2=torch.empty((w.rows,), dtype=torch.float32, device=dev) if on2 else None,
             xo=torch.empty((w.rows, w.n), dtype=TDT, device=dev)))
-    ws = torch.zeros(256, dtype=torch.uint8, device=dev)
+    ws_bytes = A.arnq_workspace_size(w.rows, w.n, dt_code, q_code, mc, w.smooth1 is not None,
+                                     w.smooth2 is not None)[1]
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     sptr = stream.cuda_stream
 
     def launch(s):
         st = A.arnq_run(s["x1"], s["x2"], params[0], params[1], params[2], params[3], w.rows, w.n,
                         dt_code, w.eps, mc, q_code, s["y1"], s["s1"], s["y2"], s["s2"], s["xo"], ws,
-                        256, sptr)
+                        ws_bytes, sptr)
         if st != A.ARNQ_OK:
             raise A.ArnqError(st, "arnq_run")
 

@@ -112,11 +112,14 @@ ARNQ_API arnq_status arnq_selected_outputs(int out_mask, int has_smooth1, int ha
                                   int *y2_on);
 
 /* Workspace bytes arnq_run needs for this problem (first phase of the pages'
- * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize").  The
- * workspace holds a status block the kernels write only on error; the caller
- * allocates it on the device, zero-fills it once, and may reuse it for any
- * number of calls on one stream.  Validates the same arguments as arnq_run
- * (except pointers).  Host only. */
+ * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize"):
+ * 256 + rows * 1856.  The workspace holds a 16-byte status block, which the
+ * kernels write only on error, and one record per row that the kernel writes
+ * and reads back within the call (the row's sum of squares and the few units
+ * the binary32 arithmetic cannot settle).  The caller allocates it on the
+ * device and zero-fills the status block once; it may be reused for any
+ * number of calls on one stream (not by calls that overlap).  Validates the
+ * same arguments as arnq_run (except pointers).  Host only. */
 ARNQ_API arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdtype qdt,
                                 int out_mask, int has_smooth1, int has_smooth2, size_t *bytes);
 
@@ -213,7 +216,8 @@ ARNQ_API arnq_status arnq_run_planned(const void *x1, const void *x2, const void
  * The paper has no counterpart: the pages' two-phase call always takes a
  * caller-allocated workspace.  This entry point is arnq_run with the workspace
  * replaced by a file-scope device array inside the library
- * (ARNQ_STATIC_SCRATCH_BYTES per device), so a caller that cannot allocate
+ * (ARNQ_STATIC_SCRATCH_BYTES = 4 MiB per device: problems of up to 2259 rows),
+ * so a caller that cannot allocate
  * (no allocator at hand, a fixed memory budget) still gets the operator.
  * It allocates nothing: no cudaMalloc / cudaFree and no allocating library
  * routine.  Arguments and results are those of arnq_run; in addition
@@ -229,7 +233,7 @@ ARNQ_API arnq_status arnq_run_planned(const void *x1, const void *x2, const void
  * threads) race on it; serialise them.  A device-side timeout status lands in
  * the array and is not readable from the host: use arnq_run with a workspace
  * where that status matters. */
-#define ARNQ_STATIC_SCRATCH_BYTES 4096
+#define ARNQ_STATIC_SCRATCH_BYTES (4 << 20)
 ARNQ_API arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *gamma,
                                     const void *beta, const void *smooth1, const void *smooth2,
                                     int64_t rows, int64_t n, arnq_dtype dt, float eps,

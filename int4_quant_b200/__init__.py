@@ -29,12 +29,14 @@ def mask_code(output_mask) -> int:
     return (_abi.ARNQ_MASK_Y1 if m0 else 0) | (_abi.ARNQ_MASK_Y2 if m1 else 0)
 
 
-def workspace(device, nbytes: int = 256):
-    """A zero-filled device workspace, cached per device (one per process)."""
+def workspace(device, nbytes: int, stream=None):
+    """A device workspace of at least nbytes with a zeroed status block, cached
+    per (device, stream) and grown on demand: calls on one stream may share it,
+    calls that overlap on other streams get their own."""
     import torch
-    key = (str(device), nbytes)
+    key = (str(device), _abi._stream(stream) or 0)
     ws = _workspaces.get(key)
-    if ws is None:
+    if ws is None or ws.numel() < nbytes:
         ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         _workspaces[key] = ws
     return ws
@@ -105,9 +107,9 @@ def add_rms_norm_dynamic_quant(x1, x2, gamma, beta=None, smooth1=None, smooth2=N
                                           smooth1 is not None, smooth2 is not None)
     if st != _abi.ARNQ_OK:
         raise ArnqError(st, "arnq_workspace_size")
-    ws = workspace(x1.device, nbytes)
     if stream is None:
         stream = torch.cuda.current_stream(x1.device)
+    ws = workspace(x1.device, nbytes, stream)
     st = _abi.arnq_run(x1, x2, gamma, beta, smooth1, smooth2, rows, n, _DT[str(dt)], eps, mc,
                        _QDT[qdtype], y1, s1, y2, s2, xo, ws, ws.numel(), stream)
     if st != _abi.ARNQ_OK:
@@ -132,9 +134,13 @@ def rms_norm_dynamic_quant(x, gamma, beta=None, smooth=None, *, eps: float = 1e-
     y = torch.empty(cshape, dtype=torch.int8 if qdtype == "int8" else torch.uint8,
                     device=x.device)
     scale = torch.empty(lead, dtype=torch.float32, device=x.device)
-    ws = workspace(x.device)
+    st, nbytes = _abi.arnq_workspace_size(rows, n, _DT[str(dt)], _QDT[qdtype],
+                                          _abi.ARNQ_MASK_ABSENT, smooth is not None, False)
+    if st != _abi.ARNQ_OK:
+        raise ArnqError(st, "arnq_workspace_size")
     if stream is None:
         stream = torch.cuda.current_stream(x.device)
+    ws = workspace(x.device, nbytes, stream)
     st = _abi.arnq_rms_norm_dynamic_quant(x, gamma, beta, smooth, rows, n, _DT[str(dt)], eps,
                                           _QDT[qdtype], y, scale, ws, ws.numel(), stream)
     if st != _abi.ARNQ_OK:

@@ -40,7 +40,7 @@ ARNQ_MASK_Y1, ARNQ_MASK_Y2 = 1, 2
 ARNQ_MAX_N = 131072
 
 ARNQ_KERNEL_AUTO, ARNQ_KERNEL_DIRECT, ARNQ_KERNEL_STAGED = 0, 1, 2
-ARNQ_STATIC_SCRATCH_BYTES = 4096
+ARNQ_STATIC_SCRATCH_BYTES = 4 << 20
 
 
 class arnq_plan(ctypes.Structure):

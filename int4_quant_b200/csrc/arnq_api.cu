@@ -18,7 +18,11 @@ namespace {
 using arnq::KParams;
 using arnq::KernelFn;
 
-constexpr size_t kWorkspaceBytes = 256;      // status block, padded
+// workspace: the status block (padded to kRecordBase), then one record per row
+size_t workspace_bytes_for(int64_t rows) {
+  return static_cast<size_t>(arnq::kRecordBase) +
+         static_cast<size_t>(rows) * static_cast<size_t>(arnq::kRecordBytes);
+}
 constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
 
@@ -178,7 +182,7 @@ arnq_status validate(Problem &P, int out_mask, const void *workspace, size_t wor
   for (const void *q : h16)
     if (q && !aligned(q, 2)) return ARNQ_ERR_ALIGN;
   if ((P.on1 && !aligned(P.scale1, 4)) || (P.on2 && !aligned(P.scale2, 4))) return ARNQ_ERR_ALIGN;
-  if (!workspace || workspace_bytes < kWorkspaceBytes) return ARNQ_ERR_WORKSPACE;
+  if (!workspace || workspace_bytes < workspace_bytes_for(P.rows)) return ARNQ_ERR_WORKSPACE;
   if (!aligned(workspace, 8)) return ARNQ_ERR_ALIGN;
   return ARNQ_OK;
 }
@@ -399,6 +403,7 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   }
   k.x_out = static_cast<uint16_t *>(P.x_out);
   k.status = static_cast<int32_t *>(workspace);
+  k.records = static_cast<unsigned char *>(workspace) + arnq::kRecordBase;
   k.rows = P.rows;
   k.n = static_cast<int32_t>(P.n);
   k.units = L.units;
@@ -505,7 +510,7 @@ arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdt
   if (st != ARNQ_OK) return st;
   st = selected(out_mask, has_smooth1 != 0, has_smooth2 != 0, nullptr, nullptr);
   if (st != ARNQ_OK) return st;
-  *bytes = kWorkspaceBytes;
+  *bytes = workspace_bytes_for(rows);
   return ARNQ_OK;
 }
 
@@ -574,7 +579,6 @@ arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *
   Problem P = problem(x1, x2, gamma, beta, smooth1, smooth2, rows, n, dt, eps, qdt, y1, scale1, y2,
                       scale2, x_out, true);
   // the host-side checks first: a rejected call touches no device
-  static_assert(kWorkspaceBytes <= ARNQ_STATIC_SCRATCH_BYTES, "scratch too small");
   arnq_status st = check_shape(P.rows, P.n, P.dt, P.qdt, P.eps);
   if (st != ARNQ_OK) return st;
   size_t need = 0;
@@ -593,8 +597,10 @@ arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *
   void *scratch = nullptr;
   st = static_scratch(&scratch);
   if (st != ARNQ_OK) return st;
-  // the status block must start at zero
-  if (cudaMemsetAsync(scratch, 0, need, static_cast<cudaStream_t>(stream)) != cudaSuccess)
+  // the status block must start at zero (the row records need no clearing:
+  // each is written before it is read)
+  if (cudaMemsetAsync(scratch, 0, arnq::kRecordBase, static_cast<cudaStream_t>(stream)) !=
+      cudaSuccess)
     return ARNQ_ERR_CUDA;
   return run_common(P, out_mask, scratch, ARNQ_STATIC_SCRATCH_BYTES, stream, nullptr);
 }

@@ -29,24 +29,26 @@
 //   code = RNE(input_k / s~_k)   rounded half-to-even by adding 1.5*2^23
 // The result must be what an fp64 evaluation of the definition gives, with the
 // scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
-// code = RNE(input_k / scale_k).  Two pieces of exact work settle that, both
-// off the fast path and finished one row late, after the next barrier:
-//  * the exact scale: the few elements within the binary32 error bound of the
-//    row maximum (the true maximum is among them) are evaluated in fp64 by the
-//    threads that hold them, and their maximum lands in shared memory;
-//  * the exact codes: |t - t_exact| <= tau for the binary32 quotient t (tau
-//    covers the binary32 error and the distance between s~ and the exact
-//    scale), so a code can differ from the fp64 one only if t lies within tau
-//    of a half-way point.  Such elements (a few per row) have their input
-//    evaluated in fp64 into a two-entry queue per thread; the code is decided
-//    once the exact scale is known.
-// These fp64 evaluations use 1/Rms and 1/scale from Newton steps (a few fp64
-// ulp) instead of divisions: the decisions they settle sit at distances of
-// about the binary32 rounding of the scale (~1e-7 relative) from a half-way
-// point, many orders above fp64 rounding.  A row the queue cannot hold (many
-// exact ties in one thread) or whose sum of squares or scale leaves the normal
-// binary32 range is put on a list and recomputed whole, in fp64 with IEEE
-// divisions in the definition's order, after the CTA's last row.
+// code = RNE(input_k / scale_k).  The fast path writes its codes and, for
+// each row, a record in the workspace: the row's fp64 sum of squares and the
+// few units (8 or 2 elements) that the binary32 arithmetic cannot settle:
+//  * candidate units: holding an element within the binary32 error bound of
+//    the row maximum (the true maximum is among them);
+//  * near-tie units: holding a code whose binary32 quotient t lies within tau
+//    of a half-way point, where |t - t_exact| <= tau covers the binary32
+//    error and the distance between s~ and the exact scale.
+// After its last row each CTA settles its rows' records, when no row state
+// is left in registers (x read back from xOut or the inputs, the parameters
+// from memory): the exact scale RN32(max fp64 |input| over the candidates /
+// Q), then the near-tie units' codes recomputed in fp64.  A record holds only
+// unit indices: storing more from the fast path costs it register spills.  These
+// fp64 evaluations use 1/Rms and 1/scale from Newton steps (a few fp64 ulp)
+// instead of divisions: the decisions they settle sit at distances of about
+// the binary32 rounding of the scale (~1e-7 relative) from a half-way point,
+// many orders above fp64 rounding.  A row whose record overflows (many equal
+// maxima, many exact ties) or whose sum of squares or scale leaves the normal
+// binary32 range is recomputed whole, in fp64 with IEEE divisions in the
+// definition's order.
 // Nothing here is a contraction: no tensor cores.
 #pragma once
 
@@ -74,13 +76,24 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 // row flags exchanged at the first barrier of the next row
 enum : int { RF_REDO = 1, RF_ABORT = 2 };
 
+// Row records, in the workspace after the status block (kRecordBase bytes):
+// one per row, kRecordBytes each:
+//   header (64 B): double ss; int ncand, ntie, flags (RF_REDO); pad
+//   units [kCandCap + kTieCap] ints: unit | output << 31; candidates first,
+//     then near ties.
+constexpr int kRecordBase = 256;
+constexpr int kCandCap = 4;     // candidate units per row
+constexpr int kTieCap = 12;     // near-tie units per row
+constexpr int kRecordBytes = 64 + (kCandCap + kTieCap) * 4;
+
 // Shared-memory layout, sized by the launch (the host computes the same):
 //   ss    [nslots] doubles: per-warp partial sums (also the exact path's reductions)
 //   wmax  [NOUT][nslots] floats: per-warp binary32 row maxima of |input_k|
 //   maxb  [NOUT][nslots] floats: set-up reduction of the bound on |B_k|
-//   amax  [2][2] u64: fp64 row maxima of |input_k| (double bits), by row parity
+//   lcnt  [2][2] ints: candidate and near-tie units recorded, by row parity
+//         (in the first CTA of a cluster)
 //   flags [2] ints: RF_* of a row, by row parity
-//   redo  count (int64) + kRedoCap row indices (int64): rows to recompute in fp64
+//   redo  count (int64) + kRedoCap row indices (int64): rows for the slow path
 //   bars  [stages] mbarriers; ring [stages] rows of staged input
 // nslots = warps per CTA times CTAs per cluster.
 constexpr int kMaxStagesDev = 8;
@@ -95,7 +108,7 @@ __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) 
   L.wmax = off;  off += nout * nslots * 4;
   L.maxb = off;  off += nout * nslots * 4;
   off = (off + 7) & ~7;
-  L.amax = off;  off += 4 * 8;
+  L.amax = off;  off += 4 * 4;
   L.flags = off; off += 2 * 4;
   off = (off + 7) & ~7;
   L.redo = off;  off += (1 + kRedoCap) * 8;
@@ -111,6 +124,7 @@ struct KParams {
   float *scale[2];            // per output slot
   uint16_t *x_out;
   int32_t *status;            // workspace status block
+  unsigned char *records;     // workspace row records (kRecordBytes per row)
   int64_t rows;
   int32_t n;                  // row length in elements
   int32_t units;              // units per row: ceil(n / U)
@@ -366,11 +380,22 @@ struct Exchange {
       atomicOr(flags + par, bits);
     }
   }
-  // the row-maximum slots live in the first CTA of the cluster
-  __device__ __forceinline__ unsigned long long *amax_slot(unsigned long long *amax, int i) {
-    return CL ? cluster.map_shared_rank(amax, 0) + i : amax + i;
+  // the row's record counters live in the first CTA of the cluster
+  __device__ __forceinline__ int *lcnt_slot(int *lcnt, int i) {
+    return CL ? cluster.map_shared_rank(lcnt, 0) + i : lcnt + i;
   }
 };
+
+// x of column c of a row, read back from memory: xOut when written, else the
+// inputs (then unchanged: an in-place update always writes xOut).
+template <class T, bool ADD>
+__device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) {
+  using C = Cvt<T>;
+  const int64_t j = row * p.n + c;
+  if (!ADD) return C::f1(p.x1[j]);
+  if (p.flags & F_XOUT) return C::f1(p.x_out[j]);
+  return C::f2(C::add2(p.x1[j], p.x2[j])).x;
+}
 
 // Whole row in fp64, in the definition's order, by all threads of the CTA (or
 // cluster), reading x back from xOut (or from the inputs when xOut is not
@@ -477,7 +502,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   double *ss_slots = reinterpret_cast<double *>(smem + lay.ss);      // [nslots]
   float *wmax_slots = reinterpret_cast<float *>(smem + lay.wmax);    // [NOUT][nslots]
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
-  unsigned long long *amax = reinterpret_cast<unsigned long long *>(smem + lay.amax);  // [2][2]
+  int *lcnt = reinterpret_cast<int *>(smem + lay.amax);                // [2 parity][2 lists]
   int *rflags = reinterpret_cast<int *>(smem + lay.flags);           // [2]
   int64_t *redo_list = reinterpret_cast<int64_t *>(smem + lay.redo);  // [0] count, then rows
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
@@ -549,7 +574,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     const float v = warp_max_nonneg(maxB[o]);
     if (lane == 0) ex.publish(maxb_slots, o * nslots + my_slot, v);
   }
-  if (tid < 4) amax[tid] = 0ull;
+  if (tid < 4) lcnt[tid] = 0;
   if (tid < 2) rflags[tid] = 0;
   if (tid == 0) redo_list[0] = 0;
   if (MODE == LOAD_STAGED && tid == 0) {
@@ -583,49 +608,18 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     }
   }
 
-  // ---- the previous row's unfinished business, settled after the next barrier
+  // ---- row records
   int64_t prev_row = -1;
-  bool redo = false;        // this thread cannot settle the current row
-  int qn = 0;               // near-tie queue of the current row: fp64 input, column
-  double qi0 = 0.0, qi1 = 0.0;
-  uint32_t qe0 = 0, qe1 = 0;  // column | output << 31
-  const double inv_q = 1.0 / static_cast<double>(QI);
-  // Run by every thread right after a first barrier; fl = the flags of the
-  // previous row, pp = its parity.
-  auto settle_prev = [&](int fl, int pp) {
-    if (fl & RF_REDO) {
-      if (tid == 0) {
-        const int64_t k = redo_list[0]++;
-        if (k < kRedoCap) redo_list[1 + k] = prev_row;
-      }
-    } else {
-      float sc[2] = {0.f, 0.f};
-#pragma unroll
-      for (int o = 0; o < NOUT; ++o) {
-        const double m =
-            __longlong_as_double(static_cast<long long>(*ex.amax_slot(amax, pp * 2 + o)));
-        sc[o] = __double2float_rn(__dmul_rn(m, inv_q));
-        if (tid == 0 && rank == 0) p.scale[o][prev_row] = sc[o];
-      }
-      if (qn > 0) {  // rare: decide the queued codes with the exact scale
-        for (int e = 0; e < 2; ++e) {
-          if (e >= qn) break;
-          const uint32_t ent = e == 0 ? qe0 : qe1;
-          const int o = static_cast<int>(ent >> 31);
-          const int c = static_cast<int>(ent & 0x7FFFFFFFu);
-          const float so = o == 0 ? sc[0] : sc[1];
-          const int q = so == 0.f ? 0 : code_of_t(__dmul_rn(e == 0 ? qi0 : qi1, rcp64(so)), QI);
-          if (INT4) {
-            uint8_t *bp = p.y[o] + prev_row * (n / 2) + c / 2;
-            const int sh = (c & 1) * 4;
-            *bp = static_cast<uint8_t>((*bp & ~(0xF << sh)) | ((q & 0xF) << sh));
-          } else {
-            p.y[o][prev_row * n + c] = static_cast<uint8_t>(q);
-          }
-        }
-      }
-    }
-    qn = 0;
+  auto header = [&](int64_t r) -> int * {
+    return reinterpret_cast<int *>(p.records + r * kRecordBytes);
+  };
+  // record unit u of output o on list l (0 candidate, 1 near tie) of row r;
+  // an overflowing list only counts, and the row goes to the slow path
+  auto record = [&](int l, int pp, int64_t r, int u, int o) {
+    const int k = atomicAdd(ex.lcnt_slot(lcnt, pp * 2 + l), 1);
+    if (k >= (l == 0 ? kCandCap : kTieCap)) return;
+    header(r)[16 + (l == 0 ? k : kCandCap + k)] =
+        static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
   };
 
   int64_t it = 0;
@@ -701,11 +695,9 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     {
       const double v = warp_sum_d(ss);
       const bool any_to = __any_sync(0xFFFFFFFFu, timed_out);
-      const bool any_redo = __any_sync(0xFFFFFFFFu, redo);
       if (lane == 0) {
         ex.publish(ss_slots, my_slot, v);
-        if (any_to || any_redo)
-          ex.flag(rflags, par ^ 1, (any_to ? RF_ABORT : 0) | (any_redo ? RF_REDO : 0));
+        if (any_to) ex.flag(rflags, par ^ 1, RF_ABORT);
       }
     }
     ex.sync();
@@ -750,29 +742,43 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       const float r = rsqrt_refined(v32);
       rinv2 = make_float2(r, r);
     }
-    if (prev_row >= 0) settle_prev(fl, par ^ 1);
-    // outside the normal binary32 range the bulk arithmetic is not trusted
-    redo = !(v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f);
+    // the record: this row's sum of squares and flags (outside the normal
+    // binary32 range the bulk arithmetic is not trusted), the previous row's
+    // unit counts; this row's counters start at zero
+    if (tid == 0 && rank == 0) {
+      int *h = header(row);
+      *reinterpret_cast<double *>(h) = ss_row;
+      h[4] = (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
+      if (prev_row >= 0) {
+        int *hp = header(prev_row);
+        hp[2] = lcnt[(par ^ 1) * 2 + 0];
+        hp[3] = lcnt[(par ^ 1) * 2 + 1];
+      }
+      lcnt[par * 2 + 0] = 0;
+      lcnt[par * 2 + 1] = 0;
+    }
 
-    // ---- pass 2: binary32 row maxima of |input_k|
-    float m32[NOUT];
+    // ---- pass 2: binary32 maxima of |input_k|, per unit and over the row
+    float mu[NOUT][UPT];
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
       float m = 0.f;
 #pragma unroll
-      for (int k = 0; k < UPT; ++k)
+      for (int k = 0; k < UPT; ++k) {
+        float mk = 0.f;
 #pragma unroll
         for (int i = 0; i < W; ++i) {
           const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
-          m = fmaxf(m, fmaxf(fabsf(in.x), fabsf(in.y)));
+          mk = fmaxf(mk, fmaxf(fabsf(in.x), fabsf(in.y)));
         }
-      m32[o] = m;
+        mu[o][k] = mk;
+        m = fmaxf(m, mk);
+      }
       const float wm = warp_max_nonneg(m);
       if (lane == 0) ex.publish(wmax_slots, o * nslots + my_slot, wm);
     }
-    // ---- exchange 2: row maxima.  The previous row's slots are free now.
+    // ---- exchange 2: row maxima
     ex.sync();
-    if (tid < NOUT && rank == 0) amax[(par ^ 1) * 2 + tid] = 0ull;
     if (tid == 0) rflags[par ^ 1] = 0;
 
     // ---- pass 3: quantize with the approximate scale s~ = max / Q (rounded half
@@ -784,29 +790,17 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       gm = warp_max_nonneg(gm);
       const float sa = __fdiv_rn(gm, QF);
       const bool normal = sa >= 1.1754943508222875e-38f;
-      if (sa != 0.f && !normal) redo = true;  // 1/s~ would overflow: exact path
+      // 1/s~ would overflow: the slow path
+      if (sa != 0.f && !normal && tid == 0 && rank == 0) header(row)[4] = RF_REDO;
       const float r32 = normal ? __frcp_rn(sa) : 0.f;
       // candidates for the row maximum: within the binary32 error of it
       const float thr = gm - 12.f * kUnit * (gm + maxBg[o]);
-      if (gm > 0.f && m32[o] >= thr && !redo) {  // about one thread per row
-        const double ri = rsqrt64(v64);
-        double c64 = 0.0;
+      if (gm > 0.f) {  // about one unit per row
 #pragma unroll
-        for (int k = 0; k < UPT; ++k)
-#pragma unroll
-          for (int i = 0; i < W; ++i) {
-            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              if (fabsf(h ? in.y : in.x) >= thr) {
-                const double xr = __dmul_rn(static_cast<double>(h ? xf[k][i].y : xf[k][i].x), ri);
-                c64 = fmax(c64, fabs(__fma_rn(xr, static_cast<double>(h ? G[o][k][i].y : G[o][k][i].x),
-                                              static_cast<double>(h ? B[o][k][i].y : B[o][k][i].x))));
-              }
-            }
-          }
-        atomicMax(ex.amax_slot(amax, par * 2 + o),
-                  static_cast<unsigned long long>(__double_as_longlong(c64)));
+        for (int k = 0; k < UPT; ++k) {
+          const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
+          if (mu[o][k] >= thr && u < seg_end) record(0, par, row, u, o);
+        }
       }
       // |t - t_exact| <= tau: the binary32 error of t (12u(Q + |B| r) + 2uQ) plus
       // the distance between s~ and the exact scale (10uQ + 6u maxB r)
@@ -830,35 +824,6 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
           bits[2 * i] = __float_as_uint(m.x);
           bits[2 * i + 1] = __float_as_uint(m.y);
           dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-        }
-        if (dmax > lim && !redo) {  // some code of the unit is near a half-way point (rare)
-          const double ri = rsqrt64(v64);
-#pragma unroll
-          for (int i = 0; i < W; ++i) {
-            const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
-            const float2 t = __fmul2_rn(in, r2);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const float th = h ? t.y : t.x;
-              const int c = U * u + 2 * i + h;
-              if (fabsf(th - rintf(th)) > lim && c < n) {
-                const uint32_t e = static_cast<uint32_t>(c) | (static_cast<uint32_t>(o) << 31);
-                const double xr = __dmul_rn(static_cast<double>(h ? xf[k][i].y : xf[k][i].x), ri);
-                const double in64 = __fma_rn(xr, static_cast<double>(h ? G[o][k][i].y : G[o][k][i].x),
-                                             static_cast<double>(h ? B[o][k][i].y : B[o][k][i].x));
-                if (qn == 0) {
-                  qe0 = e;
-                  qi0 = in64;
-                } else if (qn == 1) {
-                  qe1 = e;
-                  qi1 = in64;
-                } else {
-                  redo = true;
-                }
-                ++qn;
-              }
-            }
-          }
         }
         if (MODE != LOAD_SCALAR) {
           if (INT4) {  // 8 codes -> 4 bytes, even column in the low nibble
@@ -885,27 +850,98 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
             if (2 * u + 1 < n) y[j + 1] = static_cast<uint8_t>(bits[1] & 0xFFu);
           }
         }
+        // some code of the unit is near a half-way point (rare): record the unit
+        if (dmax > lim) record(1, par, row, u, o);
       }
     }
     prev_row = row;
   }
 
-  // ---- settle the last row
+  // ---- settle the records: the last row's counts, then every row of this
+  // stream in the first CTA of its cluster, one warp per row
   if (prev_row >= 0) {
-    const int par = static_cast<int>(it & 1);
-    const bool any_redo = __any_sync(0xFFFFFFFFu, redo);
-    if (lane == 0 && any_redo) ex.flag(rflags, par ^ 1, RF_REDO);
+    const int par = static_cast<int>((it + 1) & 1);  // the last row's parity
     ex.sync();
-    settle_prev(rflags[par ^ 1], par ^ 1);
+    if (tid == 0 && rank == 0) {
+      int *hp = header(prev_row);
+      hp[2] = lcnt[par * 2 + 0];
+      hp[3] = lcnt[par * 2 + 1];
+    }
+    ex.sync();  // every record complete and visible
+    if (rank == 0) {
+      const double inv_q = 1.0 / static_cast<double>(QI);
+      int64_t i = 0;
+      for (int64_t r = cluster_id; r < p.rows; r += nclusters, ++i) {
+        if (static_cast<int>(i % nwarps) != warp) continue;
+        const int *h = header(r);
+        const double ssr = *reinterpret_cast<const double *>(h);
+        const int nc = h[2], nt = h[3], fl = h[4];
+        if ((fl & RF_REDO) || nc > kCandCap || nt > kTieCap) {  // the slow path
+          if (lane == 0) {
+            const int64_t k = atomicAdd(reinterpret_cast<unsigned long long *>(redo_list), 1ull);
+            if (k < kRedoCap) redo_list[1 + k] = r;
+          }
+          continue;
+        }
+        const double ri = rsqrt64(__fma_rn(ssr, p.inv_n, static_cast<double>(p.eps)));
+        const int *units = h + 16;
+        // fp64 input of column c of output o: x * rinv * G + B, with x read back
+        // and G = gamma * smooth, B = beta * smooth exact in fp64
+        auto input64 = [&](int o, int c) -> double {
+          const double x = static_cast<double>(x_reload<T, ADD>(p, r, c));
+          double g = static_cast<double>(C::f1(__ldg(p.gamma + c)));
+          double b = (p.flags & F_BETA) ? static_cast<double>(C::f1(__ldg(p.beta + c))) : 0.0;
+          if (p.smooth[o]) {
+            const double sm = static_cast<double>(C::f1(__ldg(p.smooth[o] + c)));
+            g = __dmul_rn(g, sm);
+            b = __dmul_rn(b, sm);
+          }
+          return __fma_rn(__dmul_rn(x, ri), g, b);
+        };
+        // exact scales: fp64 maximum over the candidate elements, one per lane
+        double m[2] = {0.0, 0.0};
+        for (int e = lane; e < nc * U; e += 32) {
+          const uint32_t hd = static_cast<uint32_t>(units[e / U]);
+          const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
+          const int c = U * u + e % U;
+          if (c >= n) continue;
+          const double v = fabs(input64(o, c));
+          if (o == 0) m[0] = fmax(m[0], v); else m[1] = fmax(m[1], v);
+        }
+        float sc[2];
+#pragma unroll
+        for (int o = 0; o < NOUT; ++o) {
+          sc[o] = __double2float_rn(__dmul_rn(warp_max_d(m[o]), inv_q));
+          if (lane == 0) p.scale[o][r] = sc[o];
+        }
+        // near-tie units: codes in fp64, one element pair (one INT4 byte) per lane
+        for (int e = lane; e < nt * (U / 2); e += 32) {
+          const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / (U / 2)]);
+          const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
+          const int c = U * u + 2 * (e % (U / 2));
+          const float so = o == 0 ? sc[0] : sc[1];
+          const double rs = so == 0.f ? 0.0 : rcp64(so);
+          const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(o, c), rs), QI);
+          const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(o, c + 1), rs), QI);
+          if (INT4) {
+            p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+          } else {
+            p.y[o][r * n + c] = static_cast<uint8_t>(q0);
+            if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
+          }
+        }
+      }
+    }
     // ---- rows for the slow path: the listed ones, or (list overflowed) all
     ex.sync();
-    const int64_t nredo = redo_list[0];
+    const int64_t nredo = CL ? *ex.cluster.map_shared_rank(redo_list, 0) : redo_list[0];
     if (nredo > 0) {
       const int c_begin = seg_begin * U, c_end = min(seg_end * U, n);
       if (nredo <= kRedoCap) {
-        for (int64_t i = 0; i < nredo; ++i)
-          exact_row<T, INT4, NOUT, ADD, CL>(p, redo_list[1 + i], c_begin, c_end, ss_slots, nslots,
-                                            my_slot);
+        for (int64_t i = 0; i < nredo; ++i) {
+          const int64_t r = CL ? ex.cluster.map_shared_rank(redo_list, 0)[1 + i] : redo_list[1 + i];
+          exact_row<T, INT4, NOUT, ADD, CL>(p, r, c_begin, c_end, ss_slots, nslots, my_slot);
+        }
       } else {
         for (int64_t r = cluster_id; r < p.rows; r += nclusters)
           exact_row<T, INT4, NOUT, ADD, CL>(p, r, c_begin, c_end, ss_slots, nslots, my_slot);

@@ -69,6 +69,10 @@ def test_selected_outputs_rejects_unknown_mask_bits():
 def test_workspace_size():
     st, nb = A.arnq_workspace_size(8192, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
     assert st == A.ARNQ_OK and nb >= 16
+    # a status block plus one fixed-size record per row
+    st1, nb1 = A.arnq_workspace_size(1, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
+    st2, nb2 = A.arnq_workspace_size(2, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
+    assert st1 == st2 == A.ARNQ_OK and nb - nb1 == 8191 * (nb2 - nb1)
     assert A.arnq_workspace_size(0, 4096, 0, 0, -1, 0, 0)[0] == A.ARNQ_ERR_EMPTY
     assert A.arnq_workspace_size(8, 0, 0, 0, -1, 0, 0)[0] == A.ARNQ_ERR_EMPTY
     assert A.arnq_workspace_size(8, 7, 0, A.ARNQ_INT4, -1, 0, 0)[0] == A.ARNQ_ERR_SHAPE
@@ -90,7 +94,7 @@ def run(**kw):
     a = dict(x1=P["x1"], x2=P["x2"], gamma=P["g"], beta=None, smooth1=None, smooth2=None,
              rows=16, n=64, dt=A.ARNQ_BF16, eps=1e-6, out_mask=A.ARNQ_MASK_ABSENT,
              qdt=A.ARNQ_INT8, y1=P["y1"], scale1=P["sc1"], y2=None, scale2=None, x_out=P["xo"],
-             workspace=P["ws"], workspace_bytes=256, stream=None)
+             workspace=P["ws"], workspace_bytes=1 << 20, stream=None)
     a.update(kw)
     return A.arnq_run(**a)
 
@@ -169,3 +173,10 @@ def test_static_scratch_entry_validates_on_the_host():
                                      -1, 0, P["y1"], P["sc1"], None, None, None,
                                      None) == A.ARNQ_ERR_MASK
     assert A.ARNQ_STATIC_SCRATCH_BYTES >= A.arnq_workspace_size(8, 64, 0, 0, -1, 0, 0)[1]
+    # a problem needing more than the static array is refused before any device work
+    big = 1
+    while A.arnq_workspace_size(big, 64, 0, 0, -1, 0, 0)[1] <= A.ARNQ_STATIC_SCRATCH_BYTES:
+        big *= 2
+    assert A.arnq_run_static_scratch(P["x1"], P["x2"], P["g"], None, None, None, big, 64, 0, 1e-6,
+                                     -1, 0, P["y1"], P["sc1"], None, None, None,
+                                     None) == A.ARNQ_ERR_WORKSPACE

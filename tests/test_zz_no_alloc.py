@@ -37,8 +37,10 @@ def _call(entry, w, ins, out, mask):
     args = [ins["x1"], ins["x2"], ins["g"], ins["b"], ins["s1"], ins["s2"], w.rows, w.n, dt, w.eps,
             mask, qd, out["y1"], out["s1"], out["y2"], out["s2"], out["xo"]]
     if entry == "ws":
-        ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
-        st = A.arnq_run(*args, ws, 256, torch.cuda.current_stream())
+        nb = A.arnq_workspace_size(w.rows, w.n, dt, qd, mask, ins["s1"] is not None,
+                                   ins["s2"] is not None)[1]
+        ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+        st = A.arnq_run(*args, ws, nb, torch.cuda.current_stream())
     else:
         st = A.arnq_run_static_scratch(*args, torch.cuda.current_stream())
     assert st == A.ARNQ_OK, A.arnq_status_string(st)
