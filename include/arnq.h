@@ -113,13 +113,14 @@ ARNQ_API arnq_status arnq_selected_outputs(int out_mask, int has_smooth1, int ha
 
 /* Workspace bytes arnq_run needs for this problem (first phase of the pages'
  * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize"):
- * 256 + rows * 1856.  The workspace holds a 16-byte status block, which the
- * kernels write only on error, and one record per row that the kernel writes
- * and reads back within the call (the row's sum of squares and the few units
- * the binary32 arithmetic cannot settle).  The caller allocates it on the
- * device and zero-fills the status block once; it may be reused for any
- * number of calls on one stream (not by calls that overlap).  Validates the
- * same arguments as arnq_run (except pointers).  Host only. */
+ * 256 + rows * R, R = 80 + 4 * (12 + ceil(n * nout / 256)) rounded up to a
+ * multiple of 16, nout = outputs produced.  The workspace holds a 16-byte status block, which the kernels
+ * write only on error, and one record per row that the call writes and reads
+ * back (the row's fp64 sum of squares and the few units the binary32
+ * arithmetic cannot settle).  The caller allocates it on the device and
+ * zero-fills the status block once; it may be reused for any number of calls
+ * on one stream (not by calls that overlap).  Validates the same arguments as
+ * arnq_run (except pointers).  Host only. */
 ARNQ_API arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdtype qdt,
                                 int out_mask, int has_smooth1, int has_smooth2, size_t *bytes);
 
@@ -216,7 +217,8 @@ ARNQ_API arnq_status arnq_run_planned(const void *x1, const void *x2, const void
  * The paper has no counterpart: the pages' two-phase call always takes a
  * caller-allocated workspace.  This entry point is arnq_run with the workspace
  * replaced by a file-scope device array inside the library
- * (ARNQ_STATIC_SCRATCH_BYTES = 4 MiB per device: problems of up to 2259 rows),
+ * (ARNQ_STATIC_SCRATCH_BYTES = 4 MiB per device; arnq_workspace_size tells
+ * whether a problem fits: about 21000 rows of 4096 columns, one output),
  * so a caller that cannot allocate
  * (no allocator at hand, a fixed memory budget) still gets the operator.
  * It allocates nothing: no cudaMalloc / cudaFree and no allocating library

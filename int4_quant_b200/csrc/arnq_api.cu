@@ -19,19 +19,27 @@ using arnq::KParams;
 using arnq::KernelFn;
 
 // workspace: the status block (padded to kRecordBase), then one record per row
-size_t workspace_bytes_for(int64_t rows) {
+size_t workspace_bytes_for(int64_t rows, int64_t n, int nout) {
+  const int rec = arnq::record_bytes(arnq::tie_cap(static_cast<int>(n), nout));
   return static_cast<size_t>(arnq::kRecordBase) +
-         static_cast<size_t>(rows) * static_cast<size_t>(arnq::kRecordBytes);
+         static_cast<size_t>(rows) * static_cast<size_t>(rec);
 }
 constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
+constexpr int kSettleRowsPerBlock = 8;  // settle kernel: one warp per row
 
 // ---------------------------------------------------------------- kernel table
 
 struct KernelTable {
   KernelFn fn[2][2][arnq::kTableSize];  // [dtype][qdtype][...]
+  arnq::SettleFn settle[2][2][arnq::kSettleSize];
   KernelTable() {
     std::memset(fn, 0, sizeof fn);
+    std::memset(settle, 0, sizeof settle);
+    arnq::fill_settle_bf16_int8(settle[0][0]);
+    arnq::fill_settle_bf16_int4(settle[0][1]);
+    arnq::fill_settle_fp16_int8(settle[1][0]);
+    arnq::fill_settle_fp16_int4(settle[1][1]);
     arnq::fill_table_bf16_int8(fn[0][0]);
     arnq::fill_table_bf16_int4(fn[0][1]);
     arnq::fill_table_fp16_int8(fn[1][0]);
@@ -43,8 +51,18 @@ struct KernelTable {
   }
 };
 
-KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt, int cluster) {
+const KernelTable &kernel_table() {
   static const KernelTable table;
+  return table;
+}
+
+arnq::SettleFn lookup_settle(int dt, int qdt, int nout, bool add, bool vec) {
+  if (nout < 1 || nout > 2) return nullptr;
+  return kernel_table().settle[dt][qdt][arnq::settle_index(nout, add, vec)];
+}
+
+KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt, int cluster) {
+  const KernelTable &table = kernel_table();
   const int s = arnq::upt_slot(mode, upt);
   if (s < 0 || nout < 1 || nout > 2) return nullptr;
   return table.fn[dt][qdt][arnq::table_index(nout, add, mode, s, cluster > 1)];
@@ -150,6 +168,7 @@ arnq_status check_shape(int64_t rows, int64_t n, int dt, int qdt, float eps) {
   if (dt != ARNQ_BF16 && dt != ARNQ_FP16) return ARNQ_ERR_DTYPE;
   if (qdt != ARNQ_INT8 && qdt != ARNQ_INT4) return ARNQ_ERR_DTYPE;
   if (rows < 0 || n < 0) return ARNQ_ERR_SHAPE;
+  if (rows > INT32_MAX) return ARNQ_ERR_SHAPE;  // row indices are 32-bit in the kernels' lists
   if (rows == 0 || n == 0) return ARNQ_ERR_EMPTY;
   if (n > ARNQ_MAX_N) return ARNQ_ERR_SHAPE;
   if (qdt == ARNQ_INT4 && (n % 2) != 0) return ARNQ_ERR_SHAPE;
@@ -182,7 +201,9 @@ arnq_status validate(Problem &P, int out_mask, const void *workspace, size_t wor
   for (const void *q : h16)
     if (q && !aligned(q, 2)) return ARNQ_ERR_ALIGN;
   if ((P.on1 && !aligned(P.scale1, 4)) || (P.on2 && !aligned(P.scale2, 4))) return ARNQ_ERR_ALIGN;
-  if (!workspace || workspace_bytes < workspace_bytes_for(P.rows)) return ARNQ_ERR_WORKSPACE;
+  if (!workspace ||
+      workspace_bytes < workspace_bytes_for(P.rows, P.n, (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0)))
+    return ARNQ_ERR_WORKSPACE;
   if (!aligned(workspace, 8)) return ARNQ_ERR_ALIGN;
   return ARNQ_OK;
 }
@@ -279,9 +300,11 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   const int stage_bytes = nin * seg * 16;
 
   // units per thread: of the variants whose threads hold a slice, the one with
-  // the most resident threads per SM, then the most CTAs per SM
+  // the most CTAs (rows in flight) per SM, then the most units per thread
+  // (fewer threads share a row: cheaper reductions); measured best on
+  // 4096..16384-column rows
   if (pl->units == 0) {
-    int best = 0, best_thr = -1, best_ctas = -1;
+    int best = 0, best_ctas = -1;
     for (int i = 0; i < 3; ++i) {
       const int c = upt_candidate(mode, i);
       const int t = round_up(static_cast<int>(ceil_div(seg, c)), 32);
@@ -297,10 +320,8 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       st = occupancy(f, t, sm, &per_sm);
       if (st != ARNQ_OK) return st;
       if (per_sm < 1) continue;
-      const int thr = per_sm * t;
-      if (thr > best_thr || (thr == best_thr && per_sm > best_ctas)) {
+      if (per_sm > best_ctas || (per_sm == best_ctas && c > best)) {
         best = c;
-        best_thr = thr;
         best_ctas = per_sm;
       }
     }
@@ -404,6 +425,8 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   k.x_out = static_cast<uint16_t *>(P.x_out);
   k.status = static_cast<int32_t *>(workspace);
   k.records = static_cast<unsigned char *>(workspace) + arnq::kRecordBase;
+  k.tie_cap = arnq::tie_cap(static_cast<int>(P.n), (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0));
+  k.rec_bytes = arnq::record_bytes(k.tie_cap);
   k.rows = P.rows;
   k.n = static_cast<int32_t>(P.n);
   k.units = L.units;
@@ -428,6 +451,21 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
     cfg.numAttrs = 1;
   }
   if (cudaLaunchKernelEx(&cfg, L.fn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
+
+  // the settle kernel: one warp per row, a programmatic dependent of the row
+  // kernel (it may start early and waits for the row kernel's results)
+  arnq::SettleFn sfn = lookup_settle(P.dt, P.qdt, slot, P.add, plan.vector != 0);
+  if (!sfn) return ARNQ_ERR_PLAN;
+  cudaLaunchConfig_t sc = {};
+  cudaLaunchAttribute sattr[1];
+  sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  sattr[0].val.programmaticStreamSerializationAllowed = 1;
+  sc.gridDim = dim3(static_cast<unsigned>(ceil_div(P.rows, kSettleRowsPerBlock)), 1, 1);
+  sc.blockDim = dim3(32 * kSettleRowsPerBlock, 1, 1);
+  sc.stream = stream;
+  sc.attrs = sattr;
+  sc.numAttrs = 1;
+  if (cudaLaunchKernelEx(&sc, sfn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
   return ARNQ_OK;
 }
 
@@ -508,9 +546,10 @@ arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdt
   if (!bytes) return ARNQ_ERR_NULL_PTR;
   arnq_status st = check_shape(rows, n, dt, qdt, 0.0f);
   if (st != ARNQ_OK) return st;
-  st = selected(out_mask, has_smooth1 != 0, has_smooth2 != 0, nullptr, nullptr);
+  int on1 = 0, on2 = 0;
+  st = selected(out_mask, has_smooth1 != 0, has_smooth2 != 0, &on1, &on2);
   if (st != ARNQ_OK) return st;
-  *bytes = workspace_bytes_for(rows);
+  *bytes = workspace_bytes_for(rows, n, on1 + on2);
   return ARNQ_OK;
 }
 

@@ -37,18 +37,19 @@
 //  * near-tie units: holding a code whose binary32 quotient t lies within tau
 //    of a half-way point, where |t - t_exact| <= tau covers the binary32
 //    error and the distance between s~ and the exact scale.
-// After its last row each CTA settles its rows' records, when no row state
-// is left in registers (x read back from xOut or the inputs, the parameters
-// from memory): the exact scale RN32(max fp64 |input| over the candidates /
-// Q), then the near-tie units' codes recomputed in fp64.  A record holds only
-// unit indices: storing more from the fast path costs it register spills.  These
+// A second, small kernel (settle_kernel, one warp per row, launched as a
+// programmatic dependent of the first) settles the records: x read back from
+// xOut or the inputs, the parameters from memory, the exact scale RN32(max
+// fp64 |input| over the candidates / Q), then the near-tie units' codes
+// recomputed in fp64.  A record holds only unit indices: storing more from
+// the fast path costs it register spills.  These
 // fp64 evaluations use 1/Rms and 1/scale from Newton steps (a few fp64 ulp)
 // instead of divisions: the decisions they settle sit at distances of about
 // the binary32 rounding of the scale (~1e-7 relative) from a half-way point,
 // many orders above fp64 rounding.  A row whose record overflows (many equal
 // maxima, many exact ties) or whose sum of squares or scale leaves the normal
-// binary32 range is recomputed whole, in fp64 with IEEE divisions in the
-// definition's order.
+// binary32 range is recomputed whole by its warp of settle_kernel, in fp64
+// with IEEE divisions in the definition's order.
 // Nothing here is a contraction: no tensor cores.
 #pragma once
 
@@ -77,14 +78,21 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 enum : int { RF_REDO = 1, RF_ABORT = 2 };
 
 // Row records, in the workspace after the status block (kRecordBase bytes):
-// one per row, kRecordBytes each:
+// one per row, record_bytes(tie_cap) each:
 //   header (64 B): double ss; int ncand, ntie, flags (RF_REDO); pad
-//   units [kCandCap + kTieCap] ints: unit | output << 31; candidates first,
+//   units [kCandCap + tie_cap] ints: unit | output << 31; candidates first,
 //     then near ties.
+// A near tie needs |t - RNE(t)| > 0.5 - tau, about 2 tau ~ 1e-3 of the codes
+// or fewer; tie_cap leaves several times that for a row of n columns and
+// nout outputs, so rows overflow (and go to the slow path) only by design:
+// many exact ties.
 constexpr int kRecordBase = 256;
 constexpr int kCandCap = 4;     // candidate units per row
-constexpr int kTieCap = 12;     // near-tie units per row
-constexpr int kRecordBytes = 64 + (kCandCap + kTieCap) * 4;
+__host__ __device__ inline int tie_cap(int n, int nout) { return 12 + (n * nout + 255) / 256; }
+// (a multiple of 16 bytes: the header's double must stay 8-byte aligned)
+__host__ __device__ inline int record_bytes(int tcap) {
+  return (64 + (kCandCap + tcap) * 4 + 15) & ~15;
+}
 
 // Shared-memory layout, sized by the launch (the host computes the same):
 //   ss    [nslots] doubles: per-warp partial sums (also the exact path's reductions)
@@ -93,13 +101,11 @@ constexpr int kRecordBytes = 64 + (kCandCap + kTieCap) * 4;
 //   lcnt  [2][2] ints: candidate and near-tie units recorded, by row parity
 //         (in the first CTA of a cluster)
 //   flags [2] ints: RF_* of a row, by row parity
-//   redo  count (int64) + kRedoCap row indices (int64): rows for the slow path
 //   bars  [stages] mbarriers; ring [stages] rows of staged input
 // nslots = warps per CTA times CTAs per cluster.
 constexpr int kMaxStagesDev = 8;
-constexpr int kRedoCap = 32;
 struct Layout {
-  int ss, wmax, maxb, amax, flags, redo, bars, ring;
+  int ss, wmax, maxb, amax, flags, bars, ring;
 };
 __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) {
   Layout L;
@@ -111,7 +117,6 @@ __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) 
   L.amax = off;  off += 4 * 4;
   L.flags = off; off += 2 * 4;
   off = (off + 7) & ~7;
-  L.redo = off;  off += (1 + kRedoCap) * 8;
   L.bars = off;  off += stages * 8;
   L.ring = (off + 127) & ~127;
   return L;
@@ -124,7 +129,9 @@ struct KParams {
   float *scale[2];            // per output slot
   uint16_t *x_out;
   int32_t *status;            // workspace status block
-  unsigned char *records;     // workspace row records (kRecordBytes per row)
+  unsigned char *records;     // workspace row records (rec_bytes per row)
+  int32_t tie_cap;            // near-tie units a record holds
+  int32_t rec_bytes;          // bytes per record
   int64_t rows;
   int32_t n;                  // row length in elements
   int32_t units;              // units per row: ceil(n / U)
@@ -397,71 +404,112 @@ __device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) 
   return C::f2(C::add2(p.x1[j], p.x2[j])).x;
 }
 
-// Whole row in fp64, in the definition's order, by all threads of the CTA (or
-// cluster), reading x back from xOut (or from the inputs when xOut is not
-// written: then x1 and x2 are unchanged).  The slow path for rows the fast
-// path cannot settle; it runs after the CTA's last row, so it takes no
-// registers from the fast path.  Columns [c_begin, c_end) are this CTA's.
-template <class T, bool INT4, int NOUT, bool ADD, bool CL>
-__device__ __forceinline__ void exact_row(const KParams &p, int64_t row, int c_begin, int c_end,
-                                          double *slots, int nslots, int my_slot) {
-  using C = Cvt<T>;
+// Whole row in fp64, in the definition's order, by one warp, x read back from
+// memory: the slow path for rows the fast path cannot settle.
+template <class T, bool INT4, int NOUT, bool ADD>
+__device__ __forceinline__ void exact_row_warp(const KParams &p, int64_t row) {
   constexpr int QI = INT4 ? 7 : 127;
-  Exchange<CL> ex;
   const int lane = threadIdx.x & 31;
-  const int64_t base = row * p.n;
-  auto x_at = [&](int c) -> float {
-    if (ADD && (p.flags & F_XOUT)) return C::f1(p.x_out[base + c]);
-    if (!ADD) return C::f1(p.x1[base + c]);
-    const float s = C::f1(p.x1[base + c]) + C::f1(p.x2[base + c]);
-    return C::f2(C::pack(s, 0.f)).x;
-  };
-  // every thread gets the sum (or maximum) of v over the row
-  auto reduce = [&](double v, bool is_max) -> double {
-    v = is_max ? warp_max_d(v) : warp_sum_d(v);
-    ex.sync();  // every thread is done with the slots' previous contents
-    if (lane == 0) ex.publish(slots, my_slot, v);
-    ex.sync();
-    double t = 0.0;
-    for (int i = lane; i < nslots; i += 32) t = is_max ? fmax(t, slots[i]) : __dadd_rn(t, slots[i]);
-    return is_max ? warp_max_d(t) : warp_sum_d(t);
-  };
-  const int step = 2 * static_cast<int>(blockDim.x);
-  const int c0 = c_begin + 2 * static_cast<int>(threadIdx.x);  // element pairs (c, c+1)
+  const int n = p.n;
+  const int64_t base = row * n;
   double ss = 0.0;
-  for (int c = c0; c < c_end; c += step) {
-    const double a = x_at(c);
+  for (int c = lane; c < n; c += 32) {
+    const double a = x_reload<T, ADD>(p, row, c);
     ss = __fma_rn(a, a, ss);
-    if (c + 1 < c_end) {
-      const double b = x_at(c + 1);
-      ss = __fma_rn(b, b, ss);
-    }
   }
-  ss = reduce(ss, false);
-  const double rms = rms_of(ss, p.n, p.eps);
+  const double rms = rms_of(warp_sum_d(ss), n, p.eps);
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     double m = 0.0;
-    for (int c = c0; c < c_end; c += step) {
-      m = fmax(m, fabs(input_of<T>(p, o, c, x_at(c), rms)));
-      if (c + 1 < c_end) m = fmax(m, fabs(input_of<T>(p, o, c + 1, x_at(c + 1), rms)));
-    }
-    m = reduce(m, true);
-    const float sc = __double2float_rn(__ddiv_rn(m, static_cast<double>(QI)));
-    if (threadIdx.x == 0 && ex.rank == 0) p.scale[o][row] = sc;
-    for (int c = c0; c < c_end; c += step) {
-      const int q0 = code_of(input_of<T>(p, o, c, x_at(c), rms), sc, QI);
+    for (int c = lane; c < n; c += 32)
+      m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
+    const float sc = __double2float_rn(__ddiv_rn(warp_max_d(m), static_cast<double>(QI)));
+    if (lane == 0) p.scale[o][row] = sc;
+    for (int c = 2 * lane; c < n; c += 64) {  // element pairs: an INT4 byte has one writer
+      const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
       const int q1 =
-          c + 1 < c_end ? code_of(input_of<T>(p, o, c + 1, x_at(c + 1), rms), sc, QI) : 0;
+          c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
+                    : 0;
       if (INT4) {
-        p.y[o][row * (p.n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+        p.y[o][row * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
       } else {
         p.y[o][base + c] = static_cast<uint8_t>(q0);
-        if (c + 1 < c_end) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
+        if (c + 1 < n) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
       }
     }
   }
-  ex.sync();  // the slots are free again
+}
+
+// ---------------------------------------------------------------- settle kernel
+
+// Settles the row records the row kernel wrote: one warp per row.  Launched
+// after the row kernel on the same stream (as a programmatic dependent: it
+// waits for the row kernel's completion and memory before reading anything).
+// U = elements per unit of the row kernel that wrote the records.
+template <class T, bool INT4, int NOUT, bool ADD, int U>
+__global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KParams p) {
+  using C = Cvt<T>;
+  constexpr int QI = INT4 ? 7 : 127;
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  const int lane = threadIdx.x & 31;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (r >= p.rows) return;
+  const int n = p.n;
+  const int *h = reinterpret_cast<const int *>(p.records + r * p.rec_bytes);
+  const double ss = *reinterpret_cast<const double *>(h);
+  const int nc = h[2], nt = h[3], fl = h[4];
+  if ((fl & RF_REDO) || nc > kCandCap || nt > p.tie_cap) {
+    exact_row_warp<T, INT4, NOUT, ADD>(p, r);
+    return;
+  }
+  const int *units = h + 16;
+  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
+  const double inv_q = 1.0 / static_cast<double>(QI);
+  // fp64 input of column c of output o: x * rinv * G + B, with x read back and
+  // G = gamma * smooth, B = beta * smooth exact in fp64
+  auto input64 = [&](int o, int c) -> double {
+    const double x = static_cast<double>(x_reload<T, ADD>(p, r, c));
+    double g = static_cast<double>(C::f1(__ldg(p.gamma + c)));
+    double b = (p.flags & F_BETA) ? static_cast<double>(C::f1(__ldg(p.beta + c))) : 0.0;
+    if (p.smooth[o]) {
+      const double sm = static_cast<double>(C::f1(__ldg(p.smooth[o] + c)));
+      g = __dmul_rn(g, sm);
+      b = __dmul_rn(b, sm);
+    }
+    return __fma_rn(__dmul_rn(x, ri), g, b);
+  };
+  // exact scales: fp64 maximum over the candidate elements, one per lane
+  double m[2] = {0.0, 0.0};
+  for (int e = lane; e < nc * U; e += 32) {
+    const uint32_t hd = static_cast<uint32_t>(units[e / U]);
+    const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
+    const int c = U * u + e % U;
+    if (c >= n) continue;
+    const double v = fabs(input64(o, c));
+    if (o == 0) m[0] = fmax(m[0], v); else m[1] = fmax(m[1], v);
+  }
+  float sc[2] = {0.f, 0.f};
+#pragma unroll
+  for (int o = 0; o < NOUT; ++o) {
+    sc[o] = __double2float_rn(__dmul_rn(warp_max_d(m[o]), inv_q));
+    if (lane == 0) p.scale[o][r] = sc[o];
+  }
+  // near-tie units: codes in fp64, one element pair (one INT4 byte) per lane
+  for (int e = lane; e < nt * (U / 2); e += 32) {
+    const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / (U / 2)]);
+    const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
+    const int c = U * u + 2 * (e % (U / 2));
+    const float so = o == 0 ? sc[0] : sc[1];
+    const double rs = so == 0.f ? 0.0 : rcp64(so);
+    const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(o, c), rs), QI);
+    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(o, c + 1), rs), QI);
+    if (INT4) {
+      p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+    } else {
+      p.y[o][r * n + c] = static_cast<uint8_t>(q0);
+      if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- row kernel
@@ -504,7 +552,6 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
   int *lcnt = reinterpret_cast<int *>(smem + lay.amax);                // [2 parity][2 lists]
   int *rflags = reinterpret_cast<int *>(smem + lay.flags);           // [2]
-  int64_t *redo_list = reinterpret_cast<int64_t *>(smem + lay.redo);  // [0] count, then rows
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
   unsigned char *ring = smem + lay.ring;
 
@@ -576,7 +623,6 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   }
   if (tid < 4) lcnt[tid] = 0;
   if (tid < 2) rflags[tid] = 0;
-  if (tid == 0) redo_list[0] = 0;
   if (MODE == LOAD_STAGED && tid == 0) {
     for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -611,13 +657,13 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   // ---- row records
   int64_t prev_row = -1;
   auto header = [&](int64_t r) -> int * {
-    return reinterpret_cast<int *>(p.records + r * kRecordBytes);
+    return reinterpret_cast<int *>(p.records + r * p.rec_bytes);
   };
   // record unit u of output o on list l (0 candidate, 1 near tie) of row r;
   // an overflowing list only counts, and the row goes to the slow path
   auto record = [&](int l, int pp, int64_t r, int u, int o) {
     const int k = atomicAdd(ex.lcnt_slot(lcnt, pp * 2 + l), 1);
-    if (k >= (l == 0 ? kCandCap : kTieCap)) return;
+    if (k >= (l == 0 ? kCandCap : p.tie_cap)) return;
     header(r)[16 + (l == 0 ? k : kCandCap + k)] =
         static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
   };
@@ -857,8 +903,7 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     prev_row = row;
   }
 
-  // ---- settle the records: the last row's counts, then every row of this
-  // stream in the first CTA of its cluster, one warp per row
+  // ---- the last row's unit counts (the settle kernel takes it from here)
   if (prev_row >= 0) {
     const int par = static_cast<int>((it + 1) & 1);  // the last row's parity
     ex.sync();
@@ -866,86 +911,6 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       int *hp = header(prev_row);
       hp[2] = lcnt[par * 2 + 0];
       hp[3] = lcnt[par * 2 + 1];
-    }
-    ex.sync();  // every record complete and visible
-    if (rank == 0) {
-      const double inv_q = 1.0 / static_cast<double>(QI);
-      int64_t i = 0;
-      for (int64_t r = cluster_id; r < p.rows; r += nclusters, ++i) {
-        if (static_cast<int>(i % nwarps) != warp) continue;
-        const int *h = header(r);
-        const double ssr = *reinterpret_cast<const double *>(h);
-        const int nc = h[2], nt = h[3], fl = h[4];
-        if ((fl & RF_REDO) || nc > kCandCap || nt > kTieCap) {  // the slow path
-          if (lane == 0) {
-            const int64_t k = atomicAdd(reinterpret_cast<unsigned long long *>(redo_list), 1ull);
-            if (k < kRedoCap) redo_list[1 + k] = r;
-          }
-          continue;
-        }
-        const double ri = rsqrt64(__fma_rn(ssr, p.inv_n, static_cast<double>(p.eps)));
-        const int *units = h + 16;
-        // fp64 input of column c of output o: x * rinv * G + B, with x read back
-        // and G = gamma * smooth, B = beta * smooth exact in fp64
-        auto input64 = [&](int o, int c) -> double {
-          const double x = static_cast<double>(x_reload<T, ADD>(p, r, c));
-          double g = static_cast<double>(C::f1(__ldg(p.gamma + c)));
-          double b = (p.flags & F_BETA) ? static_cast<double>(C::f1(__ldg(p.beta + c))) : 0.0;
-          if (p.smooth[o]) {
-            const double sm = static_cast<double>(C::f1(__ldg(p.smooth[o] + c)));
-            g = __dmul_rn(g, sm);
-            b = __dmul_rn(b, sm);
-          }
-          return __fma_rn(__dmul_rn(x, ri), g, b);
-        };
-        // exact scales: fp64 maximum over the candidate elements, one per lane
-        double m[2] = {0.0, 0.0};
-        for (int e = lane; e < nc * U; e += 32) {
-          const uint32_t hd = static_cast<uint32_t>(units[e / U]);
-          const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
-          const int c = U * u + e % U;
-          if (c >= n) continue;
-          const double v = fabs(input64(o, c));
-          if (o == 0) m[0] = fmax(m[0], v); else m[1] = fmax(m[1], v);
-        }
-        float sc[2];
-#pragma unroll
-        for (int o = 0; o < NOUT; ++o) {
-          sc[o] = __double2float_rn(__dmul_rn(warp_max_d(m[o]), inv_q));
-          if (lane == 0) p.scale[o][r] = sc[o];
-        }
-        // near-tie units: codes in fp64, one element pair (one INT4 byte) per lane
-        for (int e = lane; e < nt * (U / 2); e += 32) {
-          const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / (U / 2)]);
-          const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
-          const int c = U * u + 2 * (e % (U / 2));
-          const float so = o == 0 ? sc[0] : sc[1];
-          const double rs = so == 0.f ? 0.0 : rcp64(so);
-          const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(o, c), rs), QI);
-          const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(o, c + 1), rs), QI);
-          if (INT4) {
-            p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
-          } else {
-            p.y[o][r * n + c] = static_cast<uint8_t>(q0);
-            if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
-          }
-        }
-      }
-    }
-    // ---- rows for the slow path: the listed ones, or (list overflowed) all
-    ex.sync();
-    const int64_t nredo = CL ? *ex.cluster.map_shared_rank(redo_list, 0) : redo_list[0];
-    if (nredo > 0) {
-      const int c_begin = seg_begin * U, c_end = min(seg_end * U, n);
-      if (nredo <= kRedoCap) {
-        for (int64_t i = 0; i < nredo; ++i) {
-          const int64_t r = CL ? ex.cluster.map_shared_rank(redo_list, 0)[1 + i] : redo_list[1 + i];
-          exact_row<T, INT4, NOUT, ADD, CL>(p, r, c_begin, c_end, ss_slots, nslots, my_slot);
-        }
-      } else {
-        for (int64_t r = cluster_id; r < p.rows; r += nclusters)
-          exact_row<T, INT4, NOUT, ADD, CL>(p, r, c_begin, c_end, ss_slots, nslots, my_slot);
-      }
     }
   }
   // no CTA leaves while a peer may still touch its shared memory

@@ -66,6 +66,16 @@ def test_selected_outputs_rejects_unknown_mask_bits():
     assert A.arnq_selected_outputs(-2, 0, 0)[0] == A.ARNQ_ERR_MASK
 
 
+def test_workspace_records_stay_aligned():
+    # per-row records hold a double: their size must keep every record 8-byte
+    # (here: 16-byte) aligned for any row length and output count
+    for n in list(range(2, 600, 2)) + [4096, 4098, 7168, 16384, 131072]:
+        for mask, s1, s2 in ((-1, 0, 0), (3, 1, 1)):
+            a = A.arnq_workspace_size(1, n, A.ARNQ_BF16, A.ARNQ_INT8, mask, s1, s2)[1]
+            b = A.arnq_workspace_size(2, n, A.ARNQ_BF16, A.ARNQ_INT8, mask, s1, s2)[1]
+            assert (b - a) % 16 == 0 and a % 16 == 0, (n, mask)
+
+
 def test_workspace_size():
     st, nb = A.arnq_workspace_size(8192, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
     assert st == A.ARNQ_OK and nb >= 16

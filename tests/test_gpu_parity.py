@@ -54,9 +54,11 @@ def canary_bytes(nbytes, offset=0):
     return buf[offset:]
 
 
-def workspace_for(rows):
-    """A workspace of the size arnq_workspace_size asks for, status block zeroed."""
-    st, nb = A.arnq_workspace_size(max(rows, 1), 8, A.ARNQ_BF16, A.ARNQ_INT8, -1, 0, 0)
+def workspace_for(rows, n):
+    """A workspace of the size arnq_workspace_size asks for with two outputs
+    (enough for any call on rows x n), status block zeroed."""
+    st, nb = A.arnq_workspace_size(max(rows, 1), max(n, 2), A.ARNQ_BF16, A.ARNQ_INT8,
+                                   A.ARNQ_MASK_Y1 | A.ARNQ_MASK_Y2, 1, 1)
     assert st == A.ARNQ_OK
     return torch.zeros(nb, dtype=torch.uint8, device="cuda"), nb
 
@@ -80,7 +82,7 @@ def run_gpu(w, plan=None, offset=0, inplace=False, mask="use", smooth="use", str
     sc1 = canary_bytes(rows * 4).view(torch.float32)  # scales must be 4-byte aligned
     sc2 = canary_bytes(rows * 4).view(torch.float32)
     xo = x1 if inplace else canary_bytes(rows * n * 2, 2 * offset).view(torch.int16)
-    ws, nb = workspace_for(rows)
+    ws, nb = workspace_for(rows, n)
     args = (x1, x2, g, b, d1, d2, rows, n, DT[w.dtype], w.eps, mc, QDT[w.qdtype], y1, sc1, y2,
             sc2, xo, ws, nb, stream)
     if plan is None:
@@ -240,7 +242,7 @@ def test_scalar_plans(units, cluster):
 def test_bad_plans_are_rejected():
     w = wl.random_case(8, 1002, seed=1)
     x = dev_bits(w.x1, "bf16")
-    ws, nb = workspace_for(8)
+    ws, nb = workspace_for(8, 1002)
     y = torch.empty(8 * 1002, dtype=torch.int8, device="cuda")
     s = torch.empty(8, dtype=torch.float32, device="cuda")
     gm = dev_bits(w.gamma, "bf16")
@@ -319,7 +321,7 @@ def test_rms_norm_dynamic_quant_no_add(dt, qdt, smooth):
     cb = w.n if qdt == "int8" else w.n // 2
     y = torch.empty(w.rows * cb, dtype=torch.uint8, device="cuda")
     s = torch.empty(w.rows, dtype=torch.float32, device="cuda")
-    ws, nb = workspace_for(w.rows)
+    ws, nb = workspace_for(w.rows, w.n)
     st = A.arnq_rms_norm_dynamic_quant(x, dev_bits(w.gamma, dt), dev_bits(w.beta, dt),
                                        dev_bits(w.smooth1, dt), w.rows, w.n, DT[dt], w.eps,
                                        QDT[qdt], y, s, ws, nb, None)
@@ -343,7 +345,7 @@ def test_v1_entry_point():
     s1 = torch.empty(w.rows, dtype=torch.float32, device="cuda")
     s2 = torch.empty(w.rows, dtype=torch.float32, device="cuda")
     xo = torch.empty(w.rows * w.n, dtype=torch.int16, device="cuda")
-    ws, nb = workspace_for(w.rows)
+    ws, nb = workspace_for(w.rows, w.n)
     st = A.arnq_run_v1(x1, x2, dev_bits(w.gamma, dt), dev_bits(w.smooth1, dt),
                        dev_bits(w.smooth2, dt), w.rows, w.n, A.ARNQ_BF16, w.eps, A.ARNQ_INT8, y1,
                        s1, y2, s2, xo, ws, nb, None)
