@@ -450,65 +450,100 @@ template <class T, bool INT4, int NOUT, bool ADD, int U>
 __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KParams p) {
   using C = Cvt<T>;
   constexpr int QI = INT4 ? 7 : 127;
+  constexpr int PAIRS = U / 2;  // element pairs per unit
   asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
   if (r >= p.rows) return;
   const int n = p.n;
+  const int tcap = p.tie_cap;
   const int *h = reinterpret_cast<const int *>(p.records + r * p.rec_bytes);
+  const int *units = h + 16;
+  // first round of loads, all independent: the header, this lane's candidate
+  // entry and its first two near-tie entries (read ahead of the counts; every
+  // index stays inside the record)
   const double ss = *reinterpret_cast<const double *>(h);
   const int nc = h[2], nt = h[3], fl = h[4];
-  if ((fl & RF_REDO) || nc > kCandCap || nt > p.tie_cap) {
+  const uint32_t ce = static_cast<uint32_t>(units[min(lane / U, kCandCap - 1)]);
+  const uint32_t te0 = static_cast<uint32_t>(units[kCandCap + min(lane / PAIRS, tcap - 1)]);
+  const uint32_t te1 = static_cast<uint32_t>(units[kCandCap + min((lane + 32) / PAIRS, tcap - 1)]);
+  if ((fl & RF_REDO) || nc > kCandCap || nt > tcap) {
     exact_row_warp<T, INT4, NOUT, ADD>(p, r);
     return;
   }
-  const int *units = h + 16;
-  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
-  const double inv_q = 1.0 / static_cast<double>(QI);
-  // fp64 input of column c of output o: x * rinv * G + B, with x read back and
-  // G = gamma * smooth, B = beta * smooth exact in fp64
-  auto input64 = [&](int o, int c) -> double {
-    const double x = static_cast<double>(x_reload<T, ADD>(p, r, c));
-    double g = static_cast<double>(C::f1(__ldg(p.gamma + c)));
-    double b = (p.flags & F_BETA) ? static_cast<double>(C::f1(__ldg(p.beta + c))) : 0.0;
-    if (p.smooth[o]) {
-      const double sm = static_cast<double>(C::f1(__ldg(p.smooth[o] + c)));
-      g = __dmul_rn(g, sm);
-      b = __dmul_rn(b, sm);
-    }
-    return __fma_rn(__dmul_rn(x, ri), g, b);
+  // x, gamma, beta and the smooth scale of column c of output o
+  struct Elem { float x, g, b, s; };
+  auto load = [&](int o, int c) -> Elem {
+    Elem e;
+    e.x = x_reload<T, ADD>(p, r, c);
+    e.g = C::f1(__ldg(p.gamma + c));
+    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) : 0.f;
+    e.s = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
+    return e;
   };
-  // exact scales: fp64 maximum over the candidate elements, one per lane
-  double m[2] = {0.0, 0.0};
-  for (int e = lane; e < nc * U; e += 32) {
-    const uint32_t hd = static_cast<uint32_t>(units[e / U]);
-    const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
-    const int c = U * u + e % U;
-    if (c >= n) continue;
-    const double v = fabs(input64(o, c));
-    if (o == 0) m[0] = fmax(m[0], v); else m[1] = fmax(m[1], v);
+  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
+  // fp64 input: x * rinv * (gamma * smooth) + beta * smooth (exact products)
+  auto input64 = [&](const Elem &e) -> double {
+    const double sm = static_cast<double>(e.s);
+    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), __dmul_rn(static_cast<double>(e.g), sm),
+                    __dmul_rn(static_cast<double>(e.b), sm));
+  };
+  auto unit_of = [](uint32_t hd) { return static_cast<int>(hd & 0x7FFFFFFFu); };
+  auto out_of = [](uint32_t hd) { return static_cast<int>(hd >> 31); };
+  // second round: every element this lane needs (one candidate element, two
+  // element pairs of near-tie units), loaded before any arithmetic
+  const int cc = U * unit_of(ce) + lane % U;
+  const bool has_c = lane < nc * U && cc < n;
+  Elem ec = {0.f, 0.f, 0.f, 0.f};
+  if (has_c) ec = load(out_of(ce), cc);
+  const int ct0 = U * unit_of(te0) + 2 * (lane % PAIRS);
+  const int ct1 = U * unit_of(te1) + 2 * ((lane + 32) % PAIRS);
+  const bool has_t0 = lane < nt * PAIRS, has_t1 = lane + 32 < nt * PAIRS;
+  Elem t00 = {0.f, 0.f, 0.f, 0.f}, t01 = t00, t10 = t00, t11 = t00;
+  if (has_t0) {
+    t00 = load(out_of(te0), ct0);
+    if (ct0 + 1 < n) t01 = load(out_of(te0), ct0 + 1);
   }
+  if (has_t1) {
+    t10 = load(out_of(te1), ct1);
+    if (ct1 + 1 < n) t11 = load(out_of(te1), ct1 + 1);
+  }
+  // exact scales: fp64 maximum over the candidate elements
+  double m[2] = {0.0, 0.0};
+  if (has_c) {
+    const double v = fabs(input64(ec));
+    if (out_of(ce) == 0) m[0] = v; else m[1] = v;
+  }
+  const double inv_q = 1.0 / static_cast<double>(QI);
   float sc[2] = {0.f, 0.f};
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     sc[o] = __double2float_rn(__dmul_rn(warp_max_d(m[o]), inv_q));
     if (lane == 0) p.scale[o][r] = sc[o];
   }
-  // near-tie units: codes in fp64, one element pair (one INT4 byte) per lane
-  for (int e = lane; e < nt * (U / 2); e += 32) {
-    const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / (U / 2)]);
-    const int u = static_cast<int>(hd & 0x7FFFFFFFu), o = static_cast<int>(hd >> 31);
-    const int c = U * u + 2 * (e % (U / 2));
+  // near-tie codes in fp64, one element pair (one INT4 byte) at a time
+  auto put = [&](uint32_t hd, int c, const Elem &e0, const Elem &e1) {
+    const int o = out_of(hd);
     const float so = o == 0 ? sc[0] : sc[1];
     const double rs = so == 0.f ? 0.0 : rcp64(so);
-    const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(o, c), rs), QI);
-    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(o, c + 1), rs), QI);
+    const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(e0), rs), QI);
+    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(e1), rs), QI);
     if (INT4) {
       p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
     } else {
       p.y[o][r * n + c] = static_cast<uint8_t>(q0);
       if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
     }
+  };
+  if (has_t0) put(te0, ct0, t00, t01);
+  if (has_t1) put(te1, ct1, t10, t11);
+  // more near-tie pairs than two per lane (rare): one pair at a time
+  for (int e = lane + 64; e < nt * PAIRS; e += 32) {
+    const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / PAIRS]);
+    const int c = U * unit_of(hd) + 2 * (e % PAIRS);
+    const Elem e0 = load(out_of(hd), c);
+    const Elem e1 = c + 1 < n ? load(out_of(hd), c + 1) : Elem{0.f, 0.f, 0.f, 0.f};
+    put(hd, c, e0, e1);
   }
 }
 
@@ -727,8 +762,9 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       }
       if (ADD && ok && (p.flags & F_XOUT)) {
         if (MODE != LOAD_SCALAR) {
-          __stcs(reinterpret_cast<uint4 *>(p.x_out + row * n + static_cast<int64_t>(u) * 8),
-                 make_uint4(xo[0], xo[1], xo[2], xo[3]));
+          // a plain store: the settle kernel may read it back soon, from L2
+          *reinterpret_cast<uint4 *>(p.x_out + row * n + static_cast<int64_t>(u) * 8) =
+              make_uint4(xo[0], xo[1], xo[2], xo[3]);
         } else {
           const int64_t j = row * n + 2 * static_cast<int64_t>(u);
           p.x_out[j] = static_cast<uint16_t>(xo[0] & 0xFFFFu);
