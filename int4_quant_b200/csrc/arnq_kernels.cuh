@@ -574,8 +574,8 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   const int ring_depth = (MODE == LOAD_STAGED) ? p.stages : 0;  // stages in the layout
   const int stages = (MODE == LOAD_STAGED) ? p.stages : 1;      // ring arithmetic
 
-  const int seg_begin = rank * p.seg_units;
-  const int seg_end = min(seg_begin + p.seg_units, p.units);
+  const int seg_begin = CL ? rank * p.seg_units : 0;  // a CTA alone holds the whole row
+  const int seg_end = CL ? min(seg_begin + p.seg_units, p.units) : p.units;
   const int seg_len = max(seg_end - seg_begin, 0);
   const uint32_t seg_bytes = static_cast<uint32_t>(seg_len) * 16u;  // staged: bytes per input
   const uint32_t stage_bytes = NIN * static_cast<uint32_t>(p.seg_units) * 16u;
@@ -704,13 +704,13 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   };
 
   int64_t it = 0;
+  int stage = 0;          // staged: it % stages, kept incrementally
+  uint32_t phase = 0;     // staged: (it / stages) & 1, the mbarrier phase to wait for
   for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
     const int par = static_cast<int>(it & 1);
-    const int stage = (MODE == LOAD_STAGED) ? static_cast<int>(it % stages) : 0;
     bool timed_out = false;
     if (MODE == LOAD_STAGED && seg_len > 0) {
-      const uint32_t parity = static_cast<uint32_t>((it / stages) & 1);
-      timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), parity);
+      timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), phase);
     }
 
     // ---- pass 1: x = RN16(x1 + x2) (or x1), xOut, sum of squares (fp64)
@@ -870,7 +870,8 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       float gm = 0.f;
       for (int i = lane; i < nslots; i += 32) gm = fmaxf(gm, wmax_slots[o * nslots + i]);
       gm = warp_max_nonneg(gm);
-      const float sa = __fdiv_rn(gm, QF);
+      // s~ = gm * RN32(1/Q): within 2u of gm / Q (the error bound below allows it)
+      const float sa = gm * (1.f / QF);
       const bool normal = sa >= 1.1754943508222875e-38f;
       // 1/s~ would overflow: the slow path
       if (sa != 0.f && !normal && tid == 0 && rank == 0) header(row)[4] = RF_REDO;
@@ -935,6 +936,10 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
         // some code of the unit is near a half-way point (rare): record the unit
         if (dmax > lim) record(1, par, row, u, o);
       }
+    }
+    if (MODE == LOAD_STAGED && ++stage == stages) {
+      stage = 0;
+      phase ^= 1u;
     }
     prev_row = row;
   }
