@@ -26,7 +26,7 @@ size_t workspace_bytes_for(int64_t rows, int64_t n, int nout) {
 }
 constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
-constexpr int kSettleRowsPerBlock = 8;  // settle kernel: one warp per row
+constexpr int kSettleRowsPerBlock = 16;  // settle kernel: 16 lanes per row, 256 threads
 
 // ---------------------------------------------------------------- kernel table
 
@@ -452,7 +452,7 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   }
   if (cudaLaunchKernelEx(&cfg, L.fn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
 
-  // the settle kernel: one warp per row, a programmatic dependent of the row
+  // the settle kernel: a half warp per row, a programmatic dependent of the row
   // kernel (it may start early and waits for the row kernel's results)
   arnq::SettleFn sfn = lookup_settle(P.dt, P.qdt, slot, P.add, plan.vector != 0);
   if (!sfn) return ARNQ_ERR_PLAN;
@@ -461,7 +461,7 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   sattr[0].val.programmaticStreamSerializationAllowed = 1;
   sc.gridDim = dim3(static_cast<unsigned>(ceil_div(P.rows, kSettleRowsPerBlock)), 1, 1);
-  sc.blockDim = dim3(32 * kSettleRowsPerBlock, 1, 1);
+  sc.blockDim = dim3(16 * kSettleRowsPerBlock, 1, 1);
   sc.stream = stream;
   sc.attrs = sattr;
   sc.numAttrs = 1;

@@ -37,7 +37,7 @@
 //  * near-tie units: holding a code whose binary32 quotient t lies within tau
 //    of a half-way point, where |t - t_exact| <= tau covers the binary32
 //    error and the distance between s~ and the exact scale.
-// A second, small kernel (settle_kernel, one warp per row, launched as a
+// A second, small kernel (settle_kernel, 16 lanes per row, launched as a
 // programmatic dependent of the first) settles the records: x read back from
 // xOut or the inputs, the parameters from memory, the exact scale RN32(max
 // fp64 |input| over the candidates / Q), then the near-tie units' codes
@@ -261,6 +261,7 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
   return pol;
 }
 
+
 // 16-byte streaming load (read once: evict-first in L1 and L2).
 __device__ __forceinline__ uint4 ld_stream16(const void *p) {
   return __ldcs(reinterpret_cast<const uint4 *>(p));
@@ -278,6 +279,17 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 __device__ __forceinline__ double warp_max_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+// sum / max over the 16 lanes of a half warp (mask: the half's lanes)
+__device__ __forceinline__ double half_sum_d(double v, unsigned mask) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(mask, v, o, 16));
+  return v;
+}
+__device__ __forceinline__ double half_max_d(double v, unsigned mask) {
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(mask, v, o, 16));
   return v;
 }
 // max over lanes of non-negative floats (their bit patterns order as integers)
@@ -404,28 +416,29 @@ __device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) 
   return C::f2(C::add2(p.x1[j], p.x2[j])).x;
 }
 
-// Whole row in fp64, in the definition's order, by one warp, x read back from
-// memory: the slow path for rows the fast path cannot settle.
+// Whole row in fp64, in the definition's order, by the 16 lanes of a half
+// warp, x read back from memory: the slow path for rows the fast path cannot
+// settle.
 template <class T, bool INT4, int NOUT, bool ADD>
-__device__ __forceinline__ void exact_row_warp(const KParams &p, int64_t row) {
+__device__ __forceinline__ void exact_row_half(const KParams &p, int64_t row, int lane,
+                                               unsigned mask) {
   constexpr int QI = INT4 ? 7 : 127;
-  const int lane = threadIdx.x & 31;
   const int n = p.n;
   const int64_t base = row * n;
   double ss = 0.0;
-  for (int c = lane; c < n; c += 32) {
+  for (int c = lane; c < n; c += 16) {
     const double a = x_reload<T, ADD>(p, row, c);
     ss = __fma_rn(a, a, ss);
   }
-  const double rms = rms_of(warp_sum_d(ss), n, p.eps);
+  const double rms = rms_of(half_sum_d(ss, mask), n, p.eps);
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     double m = 0.0;
-    for (int c = lane; c < n; c += 32)
+    for (int c = lane; c < n; c += 16)
       m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
-    const float sc = __double2float_rn(__ddiv_rn(warp_max_d(m), static_cast<double>(QI)));
+    const float sc = __double2float_rn(__ddiv_rn(half_max_d(m, mask), static_cast<double>(QI)));
     if (lane == 0) p.scale[o][row] = sc;
-    for (int c = 2 * lane; c < n; c += 64) {  // element pairs: an INT4 byte has one writer
+    for (int c = 2 * lane; c < n; c += 32) {  // element pairs: an INT4 byte has one writer
       const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
       const int q1 =
           c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
@@ -442,9 +455,10 @@ __device__ __forceinline__ void exact_row_warp(const KParams &p, int64_t row) {
 
 // ---------------------------------------------------------------- settle kernel
 
-// Settles the row records the row kernel wrote: one warp per row.  Launched
-// after the row kernel on the same stream (as a programmatic dependent: it
-// waits for the row kernel's completion and memory before reading anything).
+// Settles the row records the row kernel wrote: one half warp (16 lanes) per
+// row, so a bench-sized call's rows are all resident at once.  Launched after
+// the row kernel on the same stream (as a programmatic dependent: it waits for
+// the row kernel's completion and memory before reading anything).
 // U = elements per unit of the row kernel that wrote the records.
 template <class T, bool INT4, int NOUT, bool ADD, int U>
 __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KParams p) {
@@ -452,54 +466,56 @@ __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KPa
   constexpr int QI = INT4 ? 7 : 127;
   constexpr int PAIRS = U / 2;  // element pairs per unit
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int lane = threadIdx.x & 31;
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  if (r >= p.rows) return;
+  const int lane = threadIdx.x & 15;
+  const unsigned mask = (threadIdx.x & 16) ? 0xFFFF0000u : 0x0000FFFFu;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 4) + (threadIdx.x >> 4);
+  if (r >= p.rows) return;  // whole half warps leave together
   const int n = p.n;
   const int tcap = p.tie_cap;
   const int *h = reinterpret_cast<const int *>(p.records + r * p.rec_bytes);
   const int *units = h + 16;
-  // first round of loads, all independent: the header, this lane's candidate
-  // entry and its first two near-tie entries (read ahead of the counts; every
-  // index stays inside the record)
+  // first round of loads, all independent: the header, this lane's two
+  // candidate entries and its first two near-tie entries (read ahead of the
+  // counts; every index stays inside the record)
   const double ss = *reinterpret_cast<const double *>(h);
   const int nc = h[2], nt = h[3], fl = h[4];
-  const uint32_t ce = static_cast<uint32_t>(units[min(lane / U, kCandCap - 1)]);
+  const uint32_t ce0 = static_cast<uint32_t>(units[min(lane / U, kCandCap - 1)]);
+  const uint32_t ce1 = static_cast<uint32_t>(units[min((lane + 16) / U, kCandCap - 1)]);
   const uint32_t te0 = static_cast<uint32_t>(units[kCandCap + min(lane / PAIRS, tcap - 1)]);
-  const uint32_t te1 = static_cast<uint32_t>(units[kCandCap + min((lane + 32) / PAIRS, tcap - 1)]);
+  const uint32_t te1 = static_cast<uint32_t>(units[kCandCap + min((lane + 16) / PAIRS, tcap - 1)]);
   if ((fl & RF_REDO) || nc > kCandCap || nt > tcap) {
-    exact_row_warp<T, INT4, NOUT, ADD>(p, r);
+    exact_row_half<T, INT4, NOUT, ADD>(p, r, lane, mask);
     return;
   }
-  // x, gamma, beta and the smooth scale of column c of output o
-  struct Elem { float x, g, b, s; };
+  // x, G = gamma * smooth and B = beta * smooth (exact in binary32) of column c
+  struct Elem { float x, g, b; };
   auto load = [&](int o, int c) -> Elem {
     Elem e;
     e.x = x_reload<T, ADD>(p, r, c);
-    e.g = C::f1(__ldg(p.gamma + c));
-    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) : 0.f;
-    e.s = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
+    const float sm = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
+    e.g = C::f1(__ldg(p.gamma + c)) * sm;
+    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) * sm : 0.f;
     return e;
   };
   const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
-  // fp64 input: x * rinv * (gamma * smooth) + beta * smooth (exact products)
   auto input64 = [&](const Elem &e) -> double {
-    const double sm = static_cast<double>(e.s);
-    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), __dmul_rn(static_cast<double>(e.g), sm),
-                    __dmul_rn(static_cast<double>(e.b), sm));
+    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), static_cast<double>(e.g),
+                    static_cast<double>(e.b));
   };
   auto unit_of = [](uint32_t hd) { return static_cast<int>(hd & 0x7FFFFFFFu); };
   auto out_of = [](uint32_t hd) { return static_cast<int>(hd >> 31); };
-  // second round: every element this lane needs (one candidate element, two
+  // second round: every element this lane needs (two candidate elements, two
   // element pairs of near-tie units), loaded before any arithmetic
-  const int cc = U * unit_of(ce) + lane % U;
-  const bool has_c = lane < nc * U && cc < n;
-  Elem ec = {0.f, 0.f, 0.f, 0.f};
-  if (has_c) ec = load(out_of(ce), cc);
+  const int cc0 = U * unit_of(ce0) + lane % U, cc1 = U * unit_of(ce1) + (lane + 16) % U;
+  const bool has_c0 = lane < nc * U && cc0 < n, has_c1 = lane + 16 < nc * U && cc1 < n;
+  const Elem zero = {0.f, 0.f, 0.f};
+  Elem ec0 = zero, ec1 = zero;
+  if (has_c0) ec0 = load(out_of(ce0), cc0);
+  if (has_c1) ec1 = load(out_of(ce1), cc1);
   const int ct0 = U * unit_of(te0) + 2 * (lane % PAIRS);
-  const int ct1 = U * unit_of(te1) + 2 * ((lane + 32) % PAIRS);
-  const bool has_t0 = lane < nt * PAIRS, has_t1 = lane + 32 < nt * PAIRS;
-  Elem t00 = {0.f, 0.f, 0.f, 0.f}, t01 = t00, t10 = t00, t11 = t00;
+  const int ct1 = U * unit_of(te1) + 2 * ((lane + 16) % PAIRS);
+  const bool has_t0 = lane < nt * PAIRS, has_t1 = lane + 16 < nt * PAIRS;
+  Elem t00 = zero, t01 = zero, t10 = zero, t11 = zero;
   if (has_t0) {
     t00 = load(out_of(te0), ct0);
     if (ct0 + 1 < n) t01 = load(out_of(te0), ct0 + 1);
@@ -510,15 +526,19 @@ __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KPa
   }
   // exact scales: fp64 maximum over the candidate elements
   double m[2] = {0.0, 0.0};
-  if (has_c) {
-    const double v = fabs(input64(ec));
-    if (out_of(ce) == 0) m[0] = v; else m[1] = v;
+  if (has_c0) {
+    const double v = fabs(input64(ec0));
+    if (out_of(ce0) == 0) m[0] = v; else m[1] = v;
+  }
+  if (has_c1) {
+    const double v = fabs(input64(ec1));
+    if (out_of(ce1) == 0) m[0] = fmax(m[0], v); else m[1] = fmax(m[1], v);
   }
   const double inv_q = 1.0 / static_cast<double>(QI);
   float sc[2] = {0.f, 0.f};
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
-    sc[o] = __double2float_rn(__dmul_rn(warp_max_d(m[o]), inv_q));
+    sc[o] = __double2float_rn(__dmul_rn(half_max_d(m[o], mask), inv_q));
     if (lane == 0) p.scale[o][r] = sc[o];
   }
   // near-tie codes in fp64, one element pair (one INT4 byte) at a time
@@ -537,12 +557,12 @@ __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KPa
   };
   if (has_t0) put(te0, ct0, t00, t01);
   if (has_t1) put(te1, ct1, t10, t11);
-  // more near-tie pairs than two per lane (rare): one pair at a time
-  for (int e = lane + 64; e < nt * PAIRS; e += 32) {
+  // more near-tie pairs than two per lane: one pair at a time
+  for (int e = lane + 32; e < nt * PAIRS; e += 16) {
     const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / PAIRS]);
     const int c = U * unit_of(hd) + 2 * (e % PAIRS);
     const Elem e0 = load(out_of(hd), c);
-    const Elem e1 = c + 1 < n ? load(out_of(hd), c + 1) : Elem{0.f, 0.f, 0.f, 0.f};
+    const Elem e1 = c + 1 < n ? load(out_of(hd), c + 1) : zero;
     put(hd, c, e0, e1);
   }
 }
@@ -762,7 +782,6 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       }
       if (ADD && ok && (p.flags & F_XOUT)) {
         if (MODE != LOAD_SCALAR) {
-          // a plain store: the settle kernel may read it back soon, from L2
           *reinterpret_cast<uint4 *>(p.x_out + row * n + static_cast<int64_t>(u) * 8) =
               make_uint4(xo[0], xo[1], xo[2], xo[3]);
         } else {
@@ -814,8 +833,12 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     }
 
     double ss_row = 0.0;
-    for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
-    ss_row = warp_sum_d(ss_row);
+    if (nslots <= 8) {  // every lane adds the few partial sums itself
+      for (int i = 0; i < nslots; ++i) ss_row = __dadd_rn(ss_row, ss_slots[i]);
+    } else {
+      for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
+      ss_row = warp_sum_d(ss_row);
+    }
     // v = ss/n + eps; 1/sqrt(v) in binary32 for the bulk, in fp64 when needed
     const double v64 = __fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps));
     const float v32 = __double2float_rn(v64);
