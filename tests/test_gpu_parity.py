@@ -311,6 +311,30 @@ def test_zero_and_constant_rows():
     assert q2[123] == 127 and np.count_nonzero(q2) == 1
 
 
+@pytest.mark.parametrize("qdt", ["int8", "int4"])
+def test_rows_of_exact_ties_take_the_exact_path(qdt):
+    # x = 1 everywhere; gamma holds Q once and k + 1/2 (k = 0..Q-1) elsewhere,
+    # so every other input / scale is an exact half-way point in real
+    # arithmetic, moved off it only by the binary32 rounding of the scale:
+    # thousands of near ties per row, more than a row's record holds, so the
+    # row is recomputed whole in fp64.  Row 1 mixes in a plain random row.
+    n, q = 4096, (127 if qdt == "int8" else 7)
+    g = (np.arange(n) % q + 0.5).astype(np.float32)
+    g[17] = q
+    x1 = np.ones((3, n), np.float32)
+    rng = np.random.default_rng(5)
+    x1[1] = rng.standard_normal(n)
+    x1[2] = 0.5
+    w = wl.Workload(name="ties", rows=3, n=n, dtype="bf16", qdtype=qdt, eps=0.0,
+                    mask=None, x1=wl.to_bits(x1, "bf16"), x2=wl.to_bits(np.zeros_like(x1), "bf16"),
+                    gamma=wl.to_bits(g, "bf16"))
+    gpu, _ = run_gpu(w)
+    o = run_oracle(w)
+    # exact in both: codes and scales identical, not just within tolerance
+    assert np.array_equal(gpu["scale1"], o["scale1"])
+    assert np.array_equal(gpu["y1"], o["y1"].view(np.uint8))
+
+
 # ------------------------------------------------------------------ the other entry points
 
 @pytest.mark.parametrize("dt,qdt", [("bf16", "int8"), ("fp16", "int4")])
