@@ -230,6 +230,7 @@ bool vector_ok(const Problem &P) {
 struct Launch {
   KernelFn fn;
   int smem, seg, units;
+  int tail_rows, trec_bytes;  // in-kernel settling (tail_rows > 0) or the settle kernel
 };
 
 int upt_candidate(int mode, int i) {
@@ -237,9 +238,12 @@ int upt_candidate(int mode, int i) {
   return mode == arnq::LOAD_SCALAR ? sca[i] : vec[i];
 }
 
-// Shared memory of one CTA: the exchange slots, then (staged) the input ring.
-int smem_bytes(int cl, int threads, int nout, int stages, int stage_bytes) {
-  const arnq::Layout lay = arnq::make_layout(cl * (threads / 32), nout, stages);
+// Shared memory of one CTA: the exchange slots, the in-kernel row records (tail
+// plans), then (staged) the input ring.
+int smem_bytes(int cl, int threads, int nout, int stages, int stage_bytes, int tail_rows = 0,
+               int trec_bytes = 0) {
+  const arnq::Layout lay =
+      arnq::make_layout(cl * (threads / 32), nout, stages, tail_rows, trec_bytes);
   return lay.ring + stages * stage_bytes;
 }
 
@@ -389,7 +393,39 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
     clusters_fit = want < nc ? want : nc;
     pl->ctas_per_sm = static_cast<int32_t>(ceil_div(clusters_fit * cl, di.sms));
   }
-  const int64_t nclusters = P.rows < clusters_fit ? P.rows : clusters_fit;
+  int64_t nclusters = P.rows < clusters_fit ? P.rows : clusters_fit;
+
+  // one CTA per row: the row kernel settles its own rows from records in its
+  // shared memory, at most tail_rows per CTA.  While those records would
+  // cost resident CTAs, fewer rows per CTA (a larger grid, run in waves).
+  L->tail_rows = 0;
+  L->trec_bytes = 0;
+  if (cl == 1) {
+    const int trec = arnq::tail_rec_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
+    const int per_sm = pl->ctas_per_sm;
+    int64_t rows_cta = ceil_div(P.rows, nclusters);
+    int smem_t = 0, fit = 0;
+    while (true) {
+      smem_t = smem_bytes(1, pl->threads, nout, pl->stages, stage_bytes,
+                          static_cast<int>(rows_cta), trec);
+      fit = 0;
+      if (smem_t <= di.smem_per_block_optin) {
+        st = prepare_kernel(fn, dev, smem_t);
+        if (st != ARNQ_OK) return st;
+        st = occupancy(fn, pl->threads, smem_t, &fit);
+        if (st != ARNQ_OK) return st;
+      }
+      if (fit >= per_sm || rows_cta == 1) break;
+      rows_cta = ceil_div(rows_cta, 2);
+    }
+    if (fit < 1) return ARNQ_ERR_PLAN;
+    if (fit < per_sm) pl->ctas_per_sm = fit;
+    // the resident grid, unless fewer rows per CTA need more CTAs
+    if (rows_cta < ceil_div(P.rows, nclusters)) nclusters = ceil_div(P.rows, rows_cta);
+    L->tail_rows = static_cast<int>(ceil_div(P.rows, nclusters));
+    L->trec_bytes = trec;
+    smem = smem_t;
+  }
   pl->grid = static_cast<int32_t>(nclusters * cl);
   L->fn = fn;
   L->smem = smem;
@@ -398,9 +434,64 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   return ARNQ_OK;
 }
 
+// Plans depend on the device, the shape, the dtypes, the outputs, whether the
+// 16-byte path applies and the requested plan fields, not on the pointers:
+// cached per key, so that repeated calls skip the occupancy queries.
+struct PlanKey {
+  int dev;
+  int64_t rows, n;
+  int dt, qdt, nout, add, vec, beta;
+  arnq_plan req;
+};
+struct PlanEntry {
+  bool used;
+  PlanKey key;
+  arnq_plan plan;
+  Launch L;
+};
+constexpr int kPlanCache = 64;
+PlanEntry g_plans[kPlanCache];
+int g_plan_next = 0;
+
+bool same_key(const PlanKey &a, const PlanKey &b) { return std::memcmp(&a, &b, sizeof a) == 0; }
+
+arnq_status make_plan_cached(const Problem &P, arnq_plan *pl, Launch *L) {
+  PlanKey key;
+  std::memset(&key, 0, sizeof key);  // padding too: keys compare bytewise
+  if (cudaGetDevice(&key.dev) != cudaSuccess) return ARNQ_ERR_CUDA;
+  key.rows = P.rows;
+  key.n = P.n;
+  key.dt = P.dt;
+  key.qdt = P.qdt;
+  key.nout = (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0);
+  key.add = P.add ? 1 : 0;
+  key.vec = vector_ok(P) ? 1 : 0;
+  key.beta = P.beta ? 1 : 0;
+  key.req = *pl;
+  {
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (int i = 0; i < kPlanCache; ++i)
+      if (g_plans[i].used && same_key(g_plans[i].key, key)) {
+        *pl = g_plans[i].plan;
+        *L = g_plans[i].L;
+        return ARNQ_OK;
+      }
+  }
+  arnq_status st = make_plan(P, pl, L);
+  if (st != ARNQ_OK) return st;
+  std::lock_guard<std::mutex> lock(g_mu);
+  PlanEntry &e = g_plans[g_plan_next];
+  g_plan_next = (g_plan_next + 1) % kPlanCache;
+  e.used = true;
+  e.key = key;
+  e.plan = *pl;
+  e.L = *L;
+  return ARNQ_OK;
+}
+
 arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream_t stream) {
   Launch L;
-  arnq_status st = make_plan(P, &plan, &L);
+  arnq_status st = make_plan_cached(P, &plan, &L);
   if (st != ARNQ_OK) return st;
   KParams k;
   std::memset(&k, 0, sizeof k);
@@ -433,24 +524,33 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   k.seg_units = L.seg;
   k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0);
   k.stages = plan.stages;
+  k.tail_rows = L.tail_rows;
+  k.trec_bytes = L.trec_bytes;
   k.eps = P.eps;
   k.inv_n = 1.0 / static_cast<double>(P.n);
 
+  // The row kernel is a programmatic dependent of whatever precedes it on the
+  // stream: its CTAs may become resident while that work finishes, and wait
+  // (griddepcontrol.wait) for it before touching memory.
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.gridDim = dim3(plan.grid, 1, 1);
   cfg.blockDim = dim3(plan.threads, 1, 1);
   cfg.dynamicSmemBytes = L.smem;
   cfg.stream = stream;
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (plan.cluster > 1) {
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = plan.cluster;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = plan.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
   }
   if (cudaLaunchKernelEx(&cfg, L.fn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
+  if (plan.cluster == 1) return ARNQ_OK;  // the row kernel settles its own rows
 
   // the settle kernel: a half warp per row, a programmatic dependent of the row
   // kernel (it may start early and waits for the row kernel's results)

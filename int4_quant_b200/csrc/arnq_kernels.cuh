@@ -94,6 +94,22 @@ __host__ __device__ inline int record_bytes(int tcap) {
   return (64 + (kCandCap + tcap) * 4 + 15) & ~15;
 }
 
+// In-kernel settling (one CTA per row): the records of the CTA's own rows
+// stay in its shared memory, one per row it processes, and the CTA settles
+// them itself after its last row.  Record: a 32-byte header (double ss;
+// int cnt[2] = candidate and near-tie units recorded; int flags), then
+// kCandCap + tie_cap unit entries (unit | output << 31), as in the workspace
+// records of clusters.
+struct TailHead {
+  double ss;
+  int cnt[2];
+  int flags;
+  int pad[3];
+};
+__host__ __device__ inline int tail_rec_bytes(int tcap) {
+  return (static_cast<int>(sizeof(TailHead)) + (kCandCap + tcap) * 4 + 15) & ~15;
+}
+
 // Shared-memory layout, sized by the launch (the host computes the same):
 //   ss    [nslots] doubles: per-warp partial sums (also the exact path's reductions)
 //   wmax  [NOUT][nslots] floats: per-warp binary32 row maxima of |input_k|
@@ -101,13 +117,16 @@ __host__ __device__ inline int record_bytes(int tcap) {
 //   lcnt  [2][2] ints: candidate and near-tie units recorded, by row parity
 //         (in the first CTA of a cluster)
 //   flags [2] ints: RF_* of a row, by row parity
-//   bars  [stages] mbarriers; ring [stages] rows of staged input
+//   bars  [stages] mbarriers
+//   trec  [tail_rows] in-kernel row records of trec_bytes each (one CTA per row)
+//   ring  [stages] rows of staged input
 // nslots = warps per CTA times CTAs per cluster.
 constexpr int kMaxStagesDev = 8;
 struct Layout {
-  int ss, wmax, maxb, amax, flags, bars, ring;
+  int ss, wmax, maxb, amax, flags, bars, trec, ring;
 };
-__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) {
+__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int tail_rows,
+                                              int trec_bytes) {
   Layout L;
   int off = 0;
   L.ss = off;    off += nslots * 8;
@@ -118,6 +137,8 @@ __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages) 
   L.flags = off; off += 2 * 4;
   off = (off + 7) & ~7;
   L.bars = off;  off += stages * 8;
+  off = (off + 15) & ~15;
+  L.trec = off;  off += tail_rows * trec_bytes;
   L.ring = (off + 127) & ~127;
   return L;
 }
@@ -138,6 +159,8 @@ struct KParams {
   int32_t seg_units;          // units per CTA of a cluster
   int32_t flags;
   int32_t stages;             // staged kernel: ring depth
+  int32_t tail_rows;          // one CTA per row: rows per CTA at most (shared-memory records)
+  int32_t trec_bytes;         // bytes per shared-memory record (tail_rec_bytes)
   float eps;
   double inv_n;               // 1 / n
 };
@@ -281,15 +304,14 @@ __device__ __forceinline__ double warp_max_d(double v) {
   for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
   return v;
 }
-// sum / max over the 16 lanes of a half warp (mask: the half's lanes)
-__device__ __forceinline__ double half_sum_d(double v, unsigned mask) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(mask, v, o, 16));
+// sum / max over an aligned group of `width` lanes (a power of two up to 32;
+// mask: the group's lanes)
+__device__ __forceinline__ double group_sum_d(double v, unsigned mask, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(mask, v, o, width));
   return v;
 }
-__device__ __forceinline__ double half_max_d(double v, unsigned mask) {
-#pragma unroll
-  for (int o = 8; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(mask, v, o, 16));
+__device__ __forceinline__ double group_max_d(double v, unsigned mask, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(mask, v, o, width));
   return v;
 }
 // max over lanes of non-negative floats (their bit patterns order as integers)
@@ -416,29 +438,30 @@ __device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) 
   return C::f2(C::add2(p.x1[j], p.x2[j])).x;
 }
 
-// Whole row in fp64, in the definition's order, by the 16 lanes of a half
-// warp, x read back from memory: the slow path for rows the fast path cannot
-// settle.
+// Whole row in fp64, in the definition's order, by an aligned group of
+// `width` lanes (lane = 0 .. width-1, mask: the group's lanes), x read back
+// from memory: the slow path for rows the fast path cannot settle.
 template <class T, bool INT4, int NOUT, bool ADD>
-__device__ __forceinline__ void exact_row_half(const KParams &p, int64_t row, int lane,
-                                               unsigned mask) {
+__device__ __forceinline__ void exact_row_lanes(const KParams &p, int64_t row, int lane, int width,
+                                                unsigned mask) {
   constexpr int QI = INT4 ? 7 : 127;
   const int n = p.n;
   const int64_t base = row * n;
   double ss = 0.0;
-  for (int c = lane; c < n; c += 16) {
+  for (int c = lane; c < n; c += width) {
     const double a = x_reload<T, ADD>(p, row, c);
     ss = __fma_rn(a, a, ss);
   }
-  const double rms = rms_of(half_sum_d(ss, mask), n, p.eps);
+  const double rms = rms_of(group_sum_d(ss, mask, width), n, p.eps);
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
     double m = 0.0;
-    for (int c = lane; c < n; c += 16)
+    for (int c = lane; c < n; c += width)
       m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
-    const float sc = __double2float_rn(__ddiv_rn(half_max_d(m, mask), static_cast<double>(QI)));
+    const float sc =
+        __double2float_rn(__ddiv_rn(group_max_d(m, mask, width), static_cast<double>(QI)));
     if (lane == 0) p.scale[o][row] = sc;
-    for (int c = 2 * lane; c < n; c += 32) {  // element pairs: an INT4 byte has one writer
+    for (int c = 2 * lane; c < n; c += 2 * width) {  // element pairs: an INT4 byte has one writer
       const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
       const int q1 =
           c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
@@ -484,7 +507,7 @@ __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KPa
   const uint32_t te0 = static_cast<uint32_t>(units[kCandCap + min(lane / PAIRS, tcap - 1)]);
   const uint32_t te1 = static_cast<uint32_t>(units[kCandCap + min((lane + 16) / PAIRS, tcap - 1)]);
   if ((fl & RF_REDO) || nc > kCandCap || nt > tcap) {
-    exact_row_half<T, INT4, NOUT, ADD>(p, r, lane, mask);
+    exact_row_lanes<T, INT4, NOUT, ADD>(p, r, lane, 16, mask);
     return;
   }
   // x, G = gamma * smooth and B = beta * smooth (exact in binary32) of column c
@@ -538,7 +561,7 @@ __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KPa
   float sc[2] = {0.f, 0.f};
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {
-    sc[o] = __double2float_rn(__dmul_rn(half_max_d(m[o], mask), inv_q));
+    sc[o] = __double2float_rn(__dmul_rn(group_max_d(m[o], mask, 16), inv_q));
     if (lane == 0) p.scale[o][r] = sc[o];
   }
   // near-tie codes in fp64, one element pair (one INT4 byte) at a time
@@ -567,6 +590,151 @@ __global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KPa
   }
 }
 
+// ---------------------------------------------------------------- in-kernel settling
+
+// Settles one row from its record with an aligned group of g lanes (lane l of
+// g >= 8, gmask: the group's lanes): the exact scales from the candidate
+// units, then the near-tie units' codes, in fp64 from x read back from memory
+// and the parameters (the same arithmetic as settle_kernel).  The loads of the
+// common case (every candidate element, and each lane's first two element
+// pairs of near-tie units) are issued before any arithmetic.
+template <class T, bool INT4, int NOUT, bool ADD, int U>
+__device__ __forceinline__ void settle_row_group(const KParams &p, int64_t r, double ss, int nc,
+                                                 int nt, const int *ent, int l, int g,
+                                                 unsigned gmask) {
+  using C = Cvt<T>;
+  constexpr int QI = INT4 ? 7 : 127;
+  constexpr int PAIRS = U / 2;           // element pairs per unit
+  constexpr int CE = kCandCap * U / 8;   // candidate elements per lane, at most (g >= 8)
+  const int n = p.n;
+  struct Elem { float x, g, b; };
+  const Elem zero = {0.f, 0.f, 0.f};
+  auto load = [&](int o, int c) -> Elem {
+    Elem e;
+    e.x = x_reload<T, ADD>(p, r, c);
+    const float sm = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
+    e.g = C::f1(__ldg(p.gamma + c)) * sm;  // exact: two 16-bit significands
+    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) * sm : 0.f;
+    return e;
+  };
+  auto unit_of = [](uint32_t hd) { return static_cast<int>(hd & 0x7FFFFFFFu); };
+  auto out_of = [](uint32_t hd) { return static_cast<int>(hd >> 31); };
+
+  // candidate elements e = l, l + g, ... of the nc * U
+  Elem ce[CE];
+  int co[CE];
+  bool cv[CE];
+#pragma unroll
+  for (int k = 0; k < CE; ++k) {
+    const int e = l + k * g;
+    ce[k] = zero;
+    co[k] = 0;
+    cv[k] = false;
+    if (e < nc * U) {
+      const uint32_t hd = static_cast<uint32_t>(ent[e / U]);
+      const int c = U * unit_of(hd) + e % U;
+      if (c < n) {
+        co[k] = out_of(hd);
+        cv[k] = true;
+        ce[k] = load(co[k], c);
+      }
+    }
+  }
+  // near-tie element pairs q = l, l + g, ...: the first two now
+  Elem ta[2], tb[2];
+  uint32_t th[2];
+  int tc[2];
+  bool tv[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int q = l + k * g;
+    ta[k] = tb[k] = zero;
+    th[k] = 0u;
+    tc[k] = 0;
+    tv[k] = q < nt * PAIRS;
+    if (tv[k]) {
+      th[k] = static_cast<uint32_t>(ent[kCandCap + q / PAIRS]);
+      tc[k] = U * unit_of(th[k]) + 2 * (q % PAIRS);
+      ta[k] = load(out_of(th[k]), tc[k]);
+      if (tc[k] + 1 < n) tb[k] = load(out_of(th[k]), tc[k] + 1);
+    }
+  }
+
+  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
+  auto input64 = [&](const Elem &e) -> double {
+    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), static_cast<double>(e.g),
+                    static_cast<double>(e.b));
+  };
+  // exact scales: fp64 maximum over the candidate elements
+  double m0 = 0.0, m1 = 0.0;
+#pragma unroll
+  for (int k = 0; k < CE; ++k) {
+    if (cv[k]) {
+      const double v = fabs(input64(ce[k]));
+      if (co[k] == 0) m0 = fmax(m0, v); else m1 = fmax(m1, v);
+    }
+  }
+  const double inv_q = 1.0 / static_cast<double>(QI);
+  float sc[2] = {0.f, 0.f};
+  sc[0] = __double2float_rn(__dmul_rn(group_max_d(m0, gmask, g), inv_q));
+  if (NOUT == 2) sc[1] = __double2float_rn(__dmul_rn(group_max_d(m1, gmask, g), inv_q));
+  if (l == 0) {
+    p.scale[0][r] = sc[0];
+    if (NOUT == 2) p.scale[1][r] = sc[1];
+  }
+  // near-tie codes in fp64, one element pair (one INT4 byte) at a time
+  auto put = [&](uint32_t hd, int c, const Elem &e0, const Elem &e1) {
+    const int o = out_of(hd);
+    const float so = o == 0 ? sc[0] : sc[1];
+    const double rs = so == 0.f ? 0.0 : rcp64(so);
+    const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(e0), rs), QI);
+    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(e1), rs), QI);
+    if (INT4) {
+      p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+    } else {
+      p.y[o][r * n + c] = static_cast<uint8_t>(q0);
+      if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
+    }
+  };
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+    if (tv[k]) put(th[k], tc[k], ta[k], tb[k]);
+  for (int q = l + 2 * g; q < nt * PAIRS; q += g) {  // more than two pairs per lane
+    const uint32_t hd = static_cast<uint32_t>(ent[kCandCap + q / PAIRS]);
+    const int c = U * unit_of(hd) + 2 * (q % PAIRS);
+    const Elem e0 = load(out_of(hd), c);
+    const Elem e1 = c + 1 < n ? load(out_of(hd), c + 1) : zero;
+    put(hd, c, e0, e1);
+  }
+}
+
+// The CTA settles its own rows (local rows 0 .. nrows-1 = global rows row0,
+// row0 + row_step, ...) from the records in its shared memory, after its last
+// row: a group of lanes per row (32, 16 or 8: as many rows at once as the
+// CTA's threads allow).  Rows whose record overflowed, or that the fast path
+// flagged, are recomputed whole in fp64 by their group.
+template <class T, bool INT4, int NOUT, bool ADD, int U>
+__device__ __forceinline__ void tail_settle(const KParams &p, const unsigned char *trec, int nrows,
+                                            int64_t row0, int64_t row_step) {
+  const int nthreads = static_cast<int>(blockDim.x);
+  int g = 32;
+  while (g > 8 && nthreads / g < nrows) g >>= 1;
+  const int groups = nthreads / g;
+  const int wl = static_cast<int>(threadIdx.x) & 31;
+  const int l = wl & (g - 1);
+  const unsigned gmask = g == 32 ? 0xFFFFFFFFu : ((1u << g) - 1u) << (wl & ~(g - 1));
+  for (int i = static_cast<int>(threadIdx.x) / g; i < nrows; i += groups) {
+    const TailHead *h = reinterpret_cast<const TailHead *>(trec + static_cast<size_t>(i) * p.trec_bytes);
+    const int *ent = reinterpret_cast<const int *>(h + 1);
+    const int64_t r = row0 + static_cast<int64_t>(i) * row_step;
+    const int nc = h->cnt[0], nt = h->cnt[1];
+    if ((h->flags & RF_REDO) || nc > kCandCap || nt > p.tie_cap)
+      exact_row_lanes<T, INT4, NOUT, ADD>(p, r, l, g, gmask);
+    else
+      settle_row_group<T, INT4, NOUT, ADD, U>(p, r, h->ss, nc, nt, ent, l, g, gmask);
+  }
+}
+
 // ---------------------------------------------------------------- row kernel
 
 template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD, bool CL>
@@ -579,6 +747,9 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   constexpr float QF = static_cast<float>(QI);
   constexpr int NIN = ADD ? 2 : 1;                  // staged inputs per row
 
+  // Launched as a programmatic dependent: everything before this kernel on
+  // the stream is complete, and its memory visible, only from here on.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   Exchange<CL> ex;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -601,7 +772,10 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   const uint32_t stage_bytes = NIN * static_cast<uint32_t>(p.seg_units) * 16u;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  const Layout lay = make_layout(nslots, NOUT, ring_depth);
+  // one CTA per row: records in shared memory, settled by this CTA after its
+  // last row; a cluster per row: records in the workspace, the settle kernel
+  constexpr bool tail = !CL;
+  const Layout lay = make_layout(nslots, NOUT, ring_depth, tail ? p.tail_rows : 0, p.trec_bytes);
   double *ss_slots = reinterpret_cast<double *>(smem + lay.ss);      // [nslots]
   float *wmax_slots = reinterpret_cast<float *>(smem + lay.wmax);    // [NOUT][nslots]
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
@@ -678,6 +852,16 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   }
   if (tid < 4) lcnt[tid] = 0;
   if (tid < 2) rflags[tid] = 0;
+  auto thead = [&](int64_t i) -> TailHead * {
+    return reinterpret_cast<TailHead *>(smem + lay.trec + static_cast<size_t>(i) * p.trec_bytes);
+  };
+  if (tail) {
+    for (int i = tid; i < p.tail_rows; i += blockDim.x) {
+      TailHead *th = thead(i);
+      th->cnt[0] = th->cnt[1] = 0;
+      th->flags = 0;
+    }
+  }
   if (MODE == LOAD_STAGED && tid == 0) {
     for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -716,14 +900,21 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   };
   // record unit u of output o on list l (0 candidate, 1 near tie) of row r;
   // an overflowing list only counts, and the row goes to the slow path
+  int64_t it = 0;          // rows this CTA has processed
   auto record = [&](int l, int pp, int64_t r, int u, int o) {
+    const int entry = static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
+    if (tail) {
+      TailHead *th = thead(it);
+      const int k = atomicAdd(&th->cnt[l], 1);
+      if (k < (l == 0 ? kCandCap : p.tie_cap))
+        reinterpret_cast<int *>(th + 1)[l == 0 ? k : kCandCap + k] = entry;
+      return;
+    }
     const int k = atomicAdd(ex.lcnt_slot(lcnt, pp * 2 + l), 1);
     if (k >= (l == 0 ? kCandCap : p.tie_cap)) return;
-    header(r)[16 + (l == 0 ? k : kCandCap + k)] =
-        static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
+    header(r)[16 + (l == 0 ? k : kCandCap + k)] = entry;
   };
 
-  int64_t it = 0;
   int stage = 0;          // staged: it % stages, kept incrementally
   uint32_t phase = 0;     // staged: (it / stages) & 1, the mbarrier phase to wait for
   for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
@@ -851,6 +1042,15 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     // binary32 range the bulk arithmetic is not trusted), the previous row's
     // unit counts; this row's counters start at zero
     if (tid == 0 && rank == 0) {
+      const int fl0 =
+          (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
+      if (tail) {
+        TailHead *th = thead(it);
+        th->ss = ss_row;
+        th->flags = fl0;
+      }
+    }
+    if (!tail && tid == 0 && rank == 0) {
       int *h = header(row);
       *reinterpret_cast<double *>(h) = ss_row;
       h[4] = (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
@@ -897,7 +1097,9 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
       const float sa = gm * (1.f / QF);
       const bool normal = sa >= 1.1754943508222875e-38f;
       // 1/s~ would overflow: the slow path
-      if (sa != 0.f && !normal && tid == 0 && rank == 0) header(row)[4] = RF_REDO;
+      if (sa != 0.f && !normal && tid == 0 && rank == 0) {
+        if (tail) thead(it)->flags = RF_REDO; else header(row)[4] = RF_REDO;
+      }
       const float r32 = normal ? __frcp_rn(sa) : 0.f;
       // candidates for the row maximum: within the binary32 error of it
       const float thr = gm - 12.f * kUnit * (gm + maxBg[o]);
@@ -967,6 +1169,16 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
     prev_row = row;
   }
 
+  // the next kernel on the stream may start its set-up (it waits for this
+  // grid's completion before it reads anything)
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  // ---- in-kernel settling of this CTA's rows (rows 0 .. it-1 are complete)
+  if (tail) {
+    __syncthreads();
+    tail_settle<T, INT4, NOUT, ADD, U>(p, smem + lay.trec, static_cast<int>(it), cluster_id,
+                                       nclusters);
+    return;
+  }
   // ---- the last row's unit counts (the settle kernel takes it from here)
   if (prev_row >= 0) {
     const int par = static_cast<int>((it + 1) & 1);  // the last row's parity

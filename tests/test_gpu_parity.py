@@ -215,6 +215,13 @@ PLAN_CASES = [
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=1, cluster=4),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=8, units=2),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=16),
+    # one CTA per row (settled in the row kernel's tail), also with few CTAs
+    # per SM: more rows per CTA, or a grid run in waves
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, units=2),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, ctas_per_sm=1),
+    dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=1, units=1, ctas_per_sm=1),
 ]
 
 
@@ -223,6 +230,8 @@ PLAN_CASES = [
                                    (211, 5120, "fp16", "int4"), (19, 16384, "bf16", "int4")])
 def test_plans(pk, shape):
     rows, n, dt, qdt = shape
+    if pk.get("cluster") == 1 and n == 16384:
+        pytest.skip("a 16384-column row with two outputs does not fit one CTA")
     w = wl.random_case(rows, n, dtype=dt, qdtype=qdt, seed=rows + n, beta=True, smooth1=True,
                        smooth2=True, mask=(True, True), outlier_frac=0.01)
     p = plan(**pk)
@@ -237,6 +246,14 @@ def test_scalar_plans(units, cluster):
     w = wl.random_case(53, 3002, seed=units * 10 + cluster, beta=True, smooth1=True)
     g, _ = run_gpu(w, plan=plan(kernel=A.ARNQ_KERNEL_DIRECT, units=units, cluster=cluster))
     compare(g, run_oracle(w), "int8", f"scalar u{units} c{cluster}")
+
+
+def test_many_rows_per_cta_and_grid_in_waves():
+    # 40000 short rows on one resident CTA per SM: dozens of rows per CTA, each
+    # CTA's records in its shared memory, settled after its last row
+    w = wl.random_case(40000, 256, seed=21, beta=True, smooth1=True)
+    g, _ = run_gpu(w, plan=plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1))
+    compare(g, run_oracle(w), "int8", "40000 rows")
 
 
 def test_bad_plans_are_rejected():
@@ -293,7 +310,13 @@ def test_deterministic_rerun():
         assert np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)), k
 
 
-def test_zero_and_constant_rows():
+# one CTA per row (the row kernel settles its rows) or a cluster per row (the
+# settle kernel does)
+SETTLE_PLANS = [dict(cluster=1), dict(cluster=4)]
+
+
+@pytest.mark.parametrize("pk", SETTLE_PLANS, ids=lambda d: f"cluster{d['cluster']}")
+def test_zero_and_constant_rows(pk):
     n = 4096
     x1 = np.zeros((4, n), np.float32)
     x1[1] = 0.75
@@ -302,7 +325,7 @@ def test_zero_and_constant_rows():
     w = wl.Workload(name="special", rows=4, n=n, dtype="bf16", qdtype="int8", eps=1e-6,
                     mask=None, x1=wl.to_bits(x1, "bf16"), x2=wl.to_bits(np.zeros_like(x1), "bf16"),
                     gamma=wl.to_bits(np.ones(n, np.float32), "bf16"))
-    g, _ = run_gpu(w)
+    g, _ = run_gpu(w, plan=plan(**pk))
     o = run_oracle(w)
     compare(g, o, "int8", "special rows")
     assert g["scale1"][0] == 0.0 and not g["y1"][0].any()
@@ -311,8 +334,9 @@ def test_zero_and_constant_rows():
     assert q2[123] == 127 and np.count_nonzero(q2) == 1
 
 
+@pytest.mark.parametrize("pk", SETTLE_PLANS, ids=lambda d: f"cluster{d['cluster']}")
 @pytest.mark.parametrize("qdt", ["int8", "int4"])
-def test_rows_of_exact_ties_take_the_exact_path(qdt):
+def test_rows_of_exact_ties_take_the_exact_path(qdt, pk):
     # x = 1 everywhere; gamma holds Q once and k + 1/2 (k = 0..Q-1) elsewhere,
     # so every other input / scale is an exact half-way point in real
     # arithmetic, moved off it only by the binary32 rounding of the scale:
@@ -328,7 +352,7 @@ def test_rows_of_exact_ties_take_the_exact_path(qdt):
     w = wl.Workload(name="ties", rows=3, n=n, dtype="bf16", qdtype=qdt, eps=0.0,
                     mask=None, x1=wl.to_bits(x1, "bf16"), x2=wl.to_bits(np.zeros_like(x1), "bf16"),
                     gamma=wl.to_bits(g, "bf16"))
-    gpu, _ = run_gpu(w)
+    gpu, _ = run_gpu(w, plan=plan(**pk))
     o = run_oracle(w)
     # exact in both: codes and scales identical, not just within tolerance
     assert np.array_equal(gpu["scale1"], o["scale1"])
