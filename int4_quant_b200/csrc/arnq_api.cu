@@ -240,10 +240,11 @@ int upt_candidate(int mode, int i) {
 
 // Shared memory of one CTA: the exchange slots, the in-kernel row records (tail
 // plans), then (staged) the input ring.
-int smem_bytes(int cl, int threads, int nout, int stages, int stage_bytes, int tail_rows = 0,
-               int trec_bytes = 0) {
-  const arnq::Layout lay =
-      arnq::make_layout(cl * (threads / 32), nout, stages, tail_rows, trec_bytes);
+int smem_bytes(int mode, int upt, int cl, int threads, int nout, int stages, int stage_bytes,
+               int tail_rows = 0, int trec_bytes = 0) {
+  const arnq::Layout lay = arnq::make_layout(
+      cl * (threads / 32), nout, stages, tail_rows, trec_bytes,
+      arnq::bsm_bytes_for(mode != arnq::LOAD_SCALAR, nout, upt, threads));
   return lay.ring + stages * stage_bytes;
 }
 
@@ -284,14 +285,15 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   if (max_seg == 0) return ARNQ_ERR_PLAN;
 
   // cluster: enough CTAs per row that one CTA's slice fits in registers (and,
-  // staged, two stages of it in shared memory), then more CTAs per row while
-  // the rows are too few to fill the SMs
+  // staged, one stage of it and its B_k in shared memory), then more CTAs per
+  // row while the rows are too few to fill the SMs
   if (pl->cluster == 0) {
     int cl = 1;
     auto too_big = [&](int c) {
       const int64_t seg = ceil_div(units, c);
       if (seg > max_seg) return true;
-      return mode == arnq::LOAD_STAGED && 2 * nin * seg * 16 + 8192 > di.smem_per_block_optin;
+      return mode == arnq::LOAD_STAGED &&
+             nin * seg * 16 + nout * seg * 32 + 8192 > di.smem_per_block_optin;
     };
     while (cl < kMaxCluster && too_big(cl)) cl *= 2;
     while (cl < kMaxCluster && P.rows * cl < di.sms && ceil_div(units, 2 * cl) >= 64) cl *= 2;
@@ -316,7 +318,8 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       if (ceil_div(seg, c) < 32 && best != 0) continue;  // no more than a warp's worth idle
       KernelFn f = lookup(P.dt, P.qdt, nout, P.add, mode, c, cl);
       if (!f) continue;
-      const int sm = smem_bytes(cl, t, nout, mode == arnq::LOAD_STAGED ? 2 : 0, stage_bytes);
+      const int sm = smem_bytes(mode, c, cl, t, nout, mode == arnq::LOAD_STAGED ? 1 : 0,
+                                stage_bytes);
       if (sm > di.smem_per_block_optin) continue;
       st = prepare_kernel(f, dev, sm);
       if (st != ARNQ_OK) return st;
@@ -344,88 +347,129 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
 
   KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units, cl);
   if (!fn) return ARNQ_ERR_PLAN;
-  int smem = smem_bytes(cl, pl->threads, nout, 0, 0);
-  if (mode == arnq::LOAD_STAGED) {
-    if (pl->stages == 0) {
-      // two rows in flight per CTA (measured best on 4096..16384-element rows;
-      // deeper rings cost CTAs per SM), one if two do not fit
-      int s = 2;
-      while (s > 1 && smem_bytes(cl, pl->threads, nout, s, stage_bytes) > di.smem_per_block_optin)
-        --s;
-      pl->stages = s;
+  const int upt = pl->units;
+  const int trec = arnq::tail_rec_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
+
+  // Resident CTAs, grid and (one CTA per row) rows per CTA for a ring depth
+  // `stages`.  One CTA per row keeps the records of its rows in shared memory
+  // and settles them after its last row; while those records do not fit, fewer
+  // CTAs per SM (a persistent grid, more rows each), and only when not even one
+  // CTA fits, fewer rows per CTA (a larger grid, run in waves).
+  struct Eval {
+    int per_sm = 0, smem = 0, tail_rows = 0;
+    int64_t nclusters = 0;
+  };
+  auto evaluate = [&](int stages, Eval *e) -> arnq_status {
+    *e = Eval();
+    const int base = smem_bytes(mode, upt, cl, pl->threads, nout, stages, stage_bytes);
+    if (base > di.smem_per_block_optin) return ARNQ_OK;
+    arnq_status s2 = prepare_kernel(fn, dev, base);
+    if (s2 != ARNQ_OK) return s2;
+    if (cl > 1) {
+      cudaLaunchConfig_t cfg = {};
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = cl;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.gridDim = dim3(cl * 1024, 1, 1);
+      cfg.blockDim = dim3(pl->threads, 1, 1);
+      cfg.dynamicSmemBytes = base;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int nc = 0;
+      if (cudaOccupancyMaxActiveClusters(&nc, fn, &cfg) != cudaSuccess) return ARNQ_ERR_CUDA;
+      if (nc < 1) return ARNQ_OK;
+      int64_t want =
+          pl->ctas_per_sm != 0 ? static_cast<int64_t>(pl->ctas_per_sm) * di.sms / cl : nc;
+      if (want < 1) want = 1;
+      const int64_t fit_clusters = want < nc ? want : nc;
+      e->per_sm = static_cast<int>(ceil_div(fit_clusters * cl, di.sms));
+      e->nclusters = P.rows < fit_clusters ? P.rows : fit_clusters;
+      e->smem = base;
+      return ARNQ_OK;
     }
-    if (pl->stages < 1 || pl->stages > kMaxStages) return ARNQ_ERR_PLAN;
-    smem = smem_bytes(cl, pl->threads, nout, pl->stages, stage_bytes);
-  } else {
-    pl->stages = 0;
-  }
-  if (smem > di.smem_per_block_optin) return ARNQ_ERR_PLAN;
-  st = prepare_kernel(fn, dev, smem);
-  if (st != ARNQ_OK) return st;
-
-  // grid: persistent, as many clusters as fit at once (or one per row)
-  int64_t clusters_fit = 0;
-  if (cl == 1) {
     int per_sm = 0;
-    st = occupancy(fn, pl->threads, smem, &per_sm);
-    if (st != ARNQ_OK) return st;
-    if (per_sm < 1) return ARNQ_ERR_PLAN;
+    s2 = occupancy(fn, pl->threads, base, &per_sm);
+    if (s2 != ARNQ_OK) return s2;
+    if (per_sm < 1) return ARNQ_OK;
     if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
-    pl->ctas_per_sm = per_sm;
-    clusters_fit = static_cast<int64_t>(per_sm) * di.sms;
-  } else {
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = cl;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3(cl * 1024, 1, 1);
-    cfg.blockDim = dim3(pl->threads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int nc = 0;
-    if (cudaOccupancyMaxActiveClusters(&nc, fn, &cfg) != cudaSuccess) return ARNQ_ERR_CUDA;
-    if (nc < 1) return ARNQ_ERR_PLAN;
-    int64_t want = pl->ctas_per_sm != 0 ? static_cast<int64_t>(pl->ctas_per_sm) * di.sms / cl : nc;
-    if (want < 1) want = 1;
-    clusters_fit = want < nc ? want : nc;
-    pl->ctas_per_sm = static_cast<int32_t>(ceil_div(clusters_fit * cl, di.sms));
-  }
-  int64_t nclusters = P.rows < clusters_fit ? P.rows : clusters_fit;
-
-  // one CTA per row: the row kernel settles its own rows from records in its
-  // shared memory, at most tail_rows per CTA.  While those records would
-  // cost resident CTAs, fewer rows per CTA (a larger grid, run in waves).
-  L->tail_rows = 0;
-  L->trec_bytes = 0;
-  if (cl == 1) {
-    const int trec = arnq::tail_rec_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
-    const int per_sm = pl->ctas_per_sm;
-    int64_t rows_cta = ceil_div(P.rows, nclusters);
-    int smem_t = 0, fit = 0;
-    while (true) {
-      smem_t = smem_bytes(1, pl->threads, nout, pl->stages, stage_bytes,
-                          static_cast<int>(rows_cta), trec);
-      fit = 0;
-      if (smem_t <= di.smem_per_block_optin) {
-        st = prepare_kernel(fn, dev, smem_t);
-        if (st != ARNQ_OK) return st;
-        st = occupancy(fn, pl->threads, smem_t, &fit);
-        if (st != ARNQ_OK) return st;
+    auto fit_for = [&](int64_t rows_cta, int *fit, int *sm) -> arnq_status {
+      *fit = 0;
+      *sm = smem_bytes(mode, upt, 1, pl->threads, nout, stages, stage_bytes,
+                       static_cast<int>(rows_cta), trec);
+      if (rows_cta > (1 << 24) || *sm > di.smem_per_block_optin) return ARNQ_OK;
+      arnq_status s3 = prepare_kernel(fn, dev, *sm);
+      if (s3 != ARNQ_OK) return s3;
+      return occupancy(fn, pl->threads, *sm, fit);
+    };
+    for (int iter = 0; iter < 16; ++iter) {  // per_sm only decreases
+      const int64_t g = static_cast<int64_t>(per_sm) * di.sms;
+      const int64_t grid = P.rows < g ? P.rows : g;
+      const int64_t rows_cta = ceil_div(P.rows, grid);
+      int fit = 0, sm = 0;
+      s2 = fit_for(rows_cta, &fit, &sm);
+      if (s2 != ARNQ_OK) return s2;
+      if (fit >= per_sm) {
+        e->per_sm = per_sm;
+        e->nclusters = grid;
+        e->tail_rows = static_cast<int>(ceil_div(P.rows, grid));
+        e->smem = sm;
+        return ARNQ_OK;
       }
-      if (fit >= per_sm || rows_cta == 1) break;
+      if (fit < 1) break;
+      per_sm = fit;
+    }
+    // one resident CTA cannot hold all its rows' records: fewer rows per CTA
+    int64_t rows_cta = ceil_div(P.rows, static_cast<int64_t>(di.sms));
+    while (true) {
+      int fit = 0, sm = 0;
+      s2 = fit_for(rows_cta, &fit, &sm);
+      if (s2 != ARNQ_OK) return s2;
+      if (fit >= 1) {
+        e->per_sm = 1;
+        e->nclusters = ceil_div(P.rows, rows_cta);
+        e->tail_rows = static_cast<int>(ceil_div(P.rows, e->nclusters));
+        e->smem = sm;
+        return ARNQ_OK;
+      }
+      if (rows_cta == 1) return ARNQ_OK;
       rows_cta = ceil_div(rows_cta, 2);
     }
-    if (fit < 1) return ARNQ_ERR_PLAN;
-    if (fit < per_sm) pl->ctas_per_sm = fit;
-    // the resident grid, unless fewer rows per CTA need more CTAs
-    if (rows_cta < ceil_div(P.rows, nclusters)) nclusters = ceil_div(P.rows, rows_cta);
-    L->tail_rows = static_cast<int>(ceil_div(P.rows, nclusters));
-    L->trec_bytes = trec;
-    smem = smem_t;
+  };
+
+  Eval best;
+  if (mode == arnq::LOAD_STAGED) {
+    // ring depth: the one (of 1 and 2) that keeps the most CTAs, i.e. rows in
+    // flight, on an SM; two on a tie (measured on 4096-column rows: five CTAs
+    // with one stage beat four with two)
+    if (pl->stages != 0 && (pl->stages < 1 || pl->stages > kMaxStages)) return ARNQ_ERR_PLAN;
+    int best_s = 0;
+    for (int s = 1; s <= kMaxStages; ++s) {
+      if (pl->stages != 0 ? s != pl->stages : s > 2) continue;
+      Eval e;
+      st = evaluate(s, &e);
+      if (st != ARNQ_OK) return st;
+      if (e.per_sm > 0 && e.per_sm >= best.per_sm) {
+        best = e;
+        best_s = s;
+      }
+    }
+    if (best_s == 0) return ARNQ_ERR_PLAN;
+    pl->stages = best_s;
+  } else {
+    pl->stages = 0;
+    st = evaluate(0, &best);
+    if (st != ARNQ_OK) return st;
+    if (best.per_sm == 0) return ARNQ_ERR_PLAN;
   }
+  st = prepare_kernel(fn, dev, best.smem);
+  if (st != ARNQ_OK) return st;
+  pl->ctas_per_sm = best.per_sm;
+  const int64_t nclusters = best.nclusters;
+  const int smem = best.smem;
+  L->tail_rows = cl == 1 ? best.tail_rows : 0;
+  L->trec_bytes = cl == 1 ? trec : 0;
   pl->grid = static_cast<int32_t>(nclusters * cl);
   L->fn = fn;
   L->smem = smem;

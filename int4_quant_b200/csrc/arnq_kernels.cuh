@@ -119,14 +119,21 @@ __host__ __device__ inline int tail_rec_bytes(int tcap) {
 //   flags [2] ints: RF_* of a row, by row parity
 //   bars  [stages] mbarriers
 //   trec  [tail_rows] in-kernel row records of trec_bytes each (one CTA per row)
+//   bsm   16-byte units: B_k = beta * smooth_k of every thread's units,
+//         [NOUT][UPT][2][threads] float4 (bsm_bytes_for)
 //   ring  [stages] rows of staged input
 // nslots = warps per CTA times CTAs per cluster.
 constexpr int kMaxStagesDev = 8;
+// shared memory holding B_k for a CTA of `threads` threads, `upt` 16-byte units
+// each (0 for 2-element units, whose B_k stay in registers)
+__host__ __device__ inline int bsm_bytes_for(bool vector_units, int nout, int upt, int threads) {
+  return vector_units ? nout * upt * threads * 32 : 0;
+}
 struct Layout {
-  int ss, wmax, maxb, amax, flags, bars, trec, ring;
+  int ss, wmax, maxb, amax, flags, bars, trec, bsm, ring;
 };
 __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int tail_rows,
-                                              int trec_bytes) {
+                                              int trec_bytes, int bsm_bytes) {
   Layout L;
   int off = 0;
   L.ss = off;    off += nslots * 8;
@@ -139,6 +146,8 @@ __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, 
   L.bars = off;  off += stages * 8;
   off = (off + 15) & ~15;
   L.trec = off;  off += tail_rows * trec_bytes;
+  off = (off + 15) & ~15;
+  L.bsm = off;   off += bsm_bytes;
   L.ring = (off + 127) & ~127;
   return L;
 }
@@ -737,9 +746,10 @@ __device__ __forceinline__ void tail_settle(const KParams &p, const unsigned cha
 
 // ---------------------------------------------------------------- row kernel
 
+// The row kernel's body; the __global__ entry points below differ only in
+// their register budget.
 template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD, bool CL>
-__global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
-    rows_kernel(const __grid_constant__ KParams p) {
+__device__ __forceinline__ void rows_body(const KParams &p) {
   using C = Cvt<T>;
   constexpr int U = (MODE == LOAD_SCALAR) ? 2 : 8;  // elements per unit
   constexpr int W = U / 2;                          // element pairs per unit
@@ -775,7 +785,14 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   // one CTA per row: records in shared memory, settled by this CTA after its
   // last row; a cluster per row: records in the workspace, the settle kernel
   constexpr bool tail = !CL;
-  const Layout lay = make_layout(nslots, NOUT, ring_depth, tail ? p.tail_rows : 0, p.trec_bytes);
+  // 16-byte units keep B_k in shared memory (registers go to x and G_k)
+  constexpr bool BSM = (W == 4);
+  const Layout lay = make_layout(nslots, NOUT, ring_depth, tail ? p.tail_rows : 0, p.trec_bytes,
+                                 bsm_bytes_for(BSM, NOUT, UPT, static_cast<int>(blockDim.x)));
+  float4 *bsm = reinterpret_cast<float4 *>(smem + lay.bsm);
+  auto bsm_at = [&](int o, int k, int j) -> float4 & {
+    return bsm[((o * UPT + k) * 2 + j) * static_cast<int>(blockDim.x) + tid];
+  };
   double *ss_slots = reinterpret_cast<double *>(smem + lay.ss);      // [nslots]
   float *wmax_slots = reinterpret_cast<float *>(smem + lay.wmax);    // [NOUT][nslots]
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
@@ -842,7 +859,28 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
         maxB[o] = fmaxf(maxB[o], fmaxf(fabsf(B[o][k][i].x), fabsf(B[o][k][i].y)));
       }
     }
+    if (BSM) {  // read back only by this thread
+#pragma unroll
+      for (int o = 0; o < NOUT; ++o)
+#pragma unroll
+        for (int j = 0; j < W / 2; ++j)
+          bsm_at(o, k, j) = make_float4(B[o][k][2 * j].x, B[o][k][2 * j].y, B[o][k][2 * j + 1].x,
+                                        B[o][k][2 * j + 1].y);
+    }
   }
+  // B_k of unit k, output o: from shared memory (16-byte units) or registers
+  auto b_of = [&](int o, int k, float2 (&bk)[W]) {
+#pragma unroll
+    for (int i = 0; i < W; ++i) bk[i] = B[o][k][i];
+    if (BSM) {
+#pragma unroll
+      for (int j = 0; j < W / 2; ++j) {
+        const float4 b = bsm_at(o, k, j);
+        bk[2 * j] = make_float2(b.x, b.y);
+        bk[2 * j + 1] = make_float2(b.z, b.w);
+      }
+    }
+  };
 
   // ---- set-up exchange: the row-wide bound on |B_k|; shared state; staged ring
 #pragma unroll
@@ -1071,9 +1109,12 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
 #pragma unroll
       for (int k = 0; k < UPT; ++k) {
         float mk = 0.f;
+        float2 bk[W];
+        b_of(o, k, bk);
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
+          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], bk[i]);
+          if (NOUT == 1) xf[k][i] = in;  // one output: pass 3 quantizes this input
           mk = fmaxf(mk, fmaxf(fabsf(in.x), fabsf(in.y)));
         }
         mu[o][k] = mk;
@@ -1122,9 +1163,15 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
         if (u >= seg_end) continue;
         uint32_t bits[2 * W];  // low bits: the code (two's complement)
         float dmax = 0.f;      // largest |t - RNE(t)| of the unit
+        float2 bk[W];
+#pragma unroll
+        for (int i = 0; i < W; ++i) bk[i] = make_float2(0.f, 0.f);
+        if (NOUT == 2) b_of(o, k, bk);
 #pragma unroll
         for (int i = 0; i < W; ++i) {
-          const float2 in = __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], B[o][k][i]);
+          // the same binary32 input as in pass 2: kept (one output) or recomputed
+          const float2 in =
+              NOUT == 1 ? xf[k][i] : __ffma2_rn(__fmul2_rn(xf[k][i], rinv2), G[o][k][i], bk[i]);
           const float2 t = __fmul2_rn(in, r2);
           const float2 m = __fadd2_rn(t, make_float2(kMagic, kMagic));
           const float2 rr = __fadd2_rn(m, make_float2(-kMagic, -kMagic));  // RNE(t), exact
@@ -1191,6 +1238,20 @@ __global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
   }
   // no CTA leaves while a peer may still touch its shared memory
   if (CL) ex.sync();
+}
+
+template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD, bool CL>
+__global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
+    rows_kernel(const __grid_constant__ KParams p) {
+  rows_body<T, INT4, MODE, UPT, NOUT, ADD, CL>(p);
+}
+
+// 16-byte units, four per thread, one output: at most 96 registers, so that
+// five 128-thread CTAs (five rows in flight) fit an SM's 64K registers.
+constexpr int kRegsUpt4 = 96;
+template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD, bool CL>
+__global__ void __maxnreg__(kRegsUpt4) rows_kernel_r96(const __grid_constant__ KParams p) {
+  rows_body<T, INT4, MODE, UPT, NOUT, ADD, CL>(p);
 }
 
 }  // namespace arnq

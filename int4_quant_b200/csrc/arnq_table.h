@@ -24,17 +24,24 @@ inline int table_index(int nout, bool add, int mode, int slot, bool cl) {
          (cl ? 1 : 0);
 }
 
+// Four 16-byte units per thread with one output use the 96-register entry
+// point (five CTAs per SM); every other variant the launch-bounds one.
+template <class T, bool I4, int MODE, int NOUT, bool ADD, bool CL>
+constexpr KernelFn upt4_kernel() {
+  if constexpr (NOUT == 1) return rows_kernel_r96<T, I4, MODE, 4, NOUT, ADD, CL>;
+  else return rows_kernel<T, I4, MODE, 4, NOUT, ADD, CL>;
+}
+
 template <class T, bool I4, int NOUT, bool ADD, bool CL>
 void fill_na(KernelFn *t) {
   t[table_index(NOUT, ADD, LOAD_VEC, 0, CL)] = rows_kernel<T, I4, LOAD_VEC, 1, NOUT, ADD, CL>;
   t[table_index(NOUT, ADD, LOAD_VEC, 1, CL)] = rows_kernel<T, I4, LOAD_VEC, 2, NOUT, ADD, CL>;
-  t[table_index(NOUT, ADD, LOAD_VEC, 2, CL)] = rows_kernel<T, I4, LOAD_VEC, 4, NOUT, ADD, CL>;
+  t[table_index(NOUT, ADD, LOAD_VEC, 2, CL)] = upt4_kernel<T, I4, LOAD_VEC, NOUT, ADD, CL>();
   t[table_index(NOUT, ADD, LOAD_STAGED, 0, CL)] =
       rows_kernel<T, I4, LOAD_STAGED, 1, NOUT, ADD, CL>;
   t[table_index(NOUT, ADD, LOAD_STAGED, 1, CL)] =
       rows_kernel<T, I4, LOAD_STAGED, 2, NOUT, ADD, CL>;
-  t[table_index(NOUT, ADD, LOAD_STAGED, 2, CL)] =
-      rows_kernel<T, I4, LOAD_STAGED, 4, NOUT, ADD, CL>;
+  t[table_index(NOUT, ADD, LOAD_STAGED, 2, CL)] = upt4_kernel<T, I4, LOAD_STAGED, NOUT, ADD, CL>();
   t[table_index(NOUT, ADD, LOAD_SCALAR, 0, CL)] =
       rows_kernel<T, I4, LOAD_SCALAR, 1, NOUT, ADD, CL>;
   t[table_index(NOUT, ADD, LOAD_SCALAR, 1, CL)] =

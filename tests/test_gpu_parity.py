@@ -248,12 +248,15 @@ def test_scalar_plans(units, cluster):
     compare(g, run_oracle(w), "int8", f"scalar u{units} c{cluster}")
 
 
-def test_many_rows_per_cta_and_grid_in_waves():
-    # 40000 short rows on one resident CTA per SM: dozens of rows per CTA, each
-    # CTA's records in its shared memory, settled after its last row
-    w = wl.random_case(40000, 256, seed=21, beta=True, smooth1=True)
-    g, _ = run_gpu(w, plan=plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1))
-    compare(g, run_oracle(w), "int8", "40000 rows")
+@pytest.mark.parametrize("rows,n", [(40000, 256), (300000, 64)])
+def test_many_rows_per_cta(rows, n):
+    # one resident CTA per SM: hundreds of rows per CTA, each CTA's records in
+    # its shared memory, settled after its last row; at 300000 rows one CTA
+    # cannot hold all its rows' records, so the grid grows (run in waves)
+    w = wl.random_case(rows, n, seed=21, beta=True, smooth1=True)
+    p = plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1)
+    g, _ = run_gpu(w, plan=p)
+    compare(g, run_oracle(w), "int8", f"{rows} rows")
 
 
 def test_bad_plans_are_rejected():
