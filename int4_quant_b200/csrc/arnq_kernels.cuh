@@ -13,9 +13,12 @@
 // A CTA (or, for rows too long for one CTA or too few rows to fill the SMs, a
 // thread-block cluster of CTAs sharing a row through distributed shared memory)
 // takes one row at a time; each thread keeps its elements of x and its folded
-// parameters in registers.  Persistent grid: cluster c handles rows c,
-// c + nclusters, ...  Two barriers per row: after the sum of squares and after
-// the row maximum.
+// parameters G_k in registers (B_k of 16-byte units in shared memory, read
+// back by the thread that wrote it).  Persistent grid: cluster c handles rows
+// c, c + nclusters, ...  Two barriers per row: after the sum of squares and
+// after the row maximum.  The kernel is launched as a programmatic dependent
+// (it waits for the preceding work before touching memory, and lets the next
+// kernel start its set-up after its last row).
 //
 // Arithmetic of the fast path, binary32 two lanes at a time with the sm_100
 // packed instructions (add/mul/fma.rn.f32x2):
@@ -30,26 +33,29 @@
 // The result must be what an fp64 evaluation of the definition gives, with the
 // scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
 // code = RNE(input_k / scale_k).  The fast path writes its codes and, for
-// each row, a record in the workspace: the row's fp64 sum of squares and the
-// few units (8 or 2 elements) that the binary32 arithmetic cannot settle:
+// each row, a record: the row's fp64 sum of squares and the few units (8 or
+// 2 elements) that the binary32 arithmetic cannot settle:
 //  * candidate units: holding an element within the binary32 error bound of
 //    the row maximum (the true maximum is among them);
 //  * near-tie units: holding a code whose binary32 quotient t lies within tau
 //    of a half-way point, where |t - t_exact| <= tau covers the binary32
 //    error and the distance between s~ and the exact scale.
-// A second, small kernel (settle_kernel, 16 lanes per row, launched as a
-// programmatic dependent of the first) settles the records: x read back from
-// xOut or the inputs, the parameters from memory, the exact scale RN32(max
-// fp64 |input| over the candidates / Q), then the near-tie units' codes
-// recomputed in fp64.  A record holds only unit indices: storing more from
-// the fast path costs it register spills.  These
+// The records are settled from x read back from xOut or the inputs and the
+// parameters from memory: the exact scale RN32(max fp64 |input| over the
+// candidates / Q), then the near-tie units' codes recomputed in fp64.  With
+// one CTA per row, each CTA keeps its rows' records in shared memory and
+// settles them itself after its last row (tail_settle, a group of 8 to 32
+// lanes per row); a row shared by a cluster has its record in the workspace,
+// settled by a second, small kernel (settle_kernel, 16 lanes per row, launched
+// as a programmatic dependent).  A record holds only unit indices: storing
+// more from the fast path costs it register spills.  These
 // fp64 evaluations use 1/Rms and 1/scale from Newton steps (a few fp64 ulp)
 // instead of divisions: the decisions they settle sit at distances of about
 // the binary32 rounding of the scale (~1e-7 relative) from a half-way point,
 // many orders above fp64 rounding.  A row whose record overflows (many equal
 // maxima, many exact ties) or whose sum of squares or scale leaves the normal
-// binary32 range is recomputed whole by its warp of settle_kernel, in fp64
-// with IEEE divisions in the definition's order.
+// binary32 range is recomputed whole by its lanes, in fp64 with IEEE
+// divisions in the definition's order.
 // Nothing here is a contraction: no tensor cores.
 #pragma once
 
@@ -276,8 +282,7 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity)
 }
 
 // 1-D bulk copy global -> this CTA's shared memory, completing on an mbarrier.
-// dst, src 16-byte aligned; bytes a multiple of 16.  Evict-first in L2: every
-// input byte is read exactly once.
+// dst, src 16-byte aligned; bytes a multiple of 16; `policy` an L2 cache policy.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
                                          uint32_t bar, uint64_t policy) {
   asm volatile(
@@ -287,9 +292,12 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
       : "memory");
 }
 
-__device__ __forceinline__ uint64_t policy_evict_first() {
+// L2 policy of the staged input copies: normal eviction (measured faster than
+// evict-first on the 8192 x 4096 workload, where x1, x2 and the outputs
+// together exceed L2).
+__device__ __forceinline__ uint64_t policy_evict_normal() {
   uint64_t pol;
-  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  asm volatile("createpolicy.fractional.L2::evict_normal.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
 
@@ -924,7 +932,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     if (ADD) bulk_g2s(dst + seg_bytes, p.x2 + off, seg_bytes, bar, policy);
   };
   if (MODE == LOAD_STAGED && tid == 0 && seg_len > 0) {
-    policy = policy_evict_first();
+    policy = policy_evict_normal();
     for (int s = 0; s < stages; ++s) {
       const int64_t row = cluster_id + s * nclusters;
       if (row < p.rows) issue(row, s);
