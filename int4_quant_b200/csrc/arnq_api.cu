@@ -396,9 +396,12 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
     if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
     auto fit_for = [&](int64_t rows_cta, int *fit, int *sm) -> arnq_status {
       *fit = 0;
+      *sm = 0;
+      // (records alone beyond a CTA's shared memory: no fit, and no int overflow below)
+      if (rows_cta * static_cast<int64_t>(trec) > di.smem_per_block_optin) return ARNQ_OK;
       *sm = smem_bytes(mode, upt, 1, pl->threads, nout, stages, stage_bytes,
                        static_cast<int>(rows_cta), trec);
-      if (rows_cta > (1 << 24) || *sm > di.smem_per_block_optin) return ARNQ_OK;
+      if (*sm > di.smem_per_block_optin) return ARNQ_OK;
       arnq_status s3 = prepare_kernel(fn, dev, *sm);
       if (s3 != ARNQ_OK) return s3;
       return occupancy(fn, pl->threads, *sm, fit);
