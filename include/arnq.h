@@ -45,6 +45,14 @@
  * as x1 or x2 (in-place residual update); any other overlap between an
  * output and an input is undefined.
  *
+ * Launches: one kernel per call when each row is handled by one CTA, two
+ * (the row kernel, then a small settle kernel) when a thread-block cluster
+ * shares each row.  The row kernel is launched as a programmatic dependent
+ * launch (cudaLaunchAttributeProgrammaticStreamSerialization): its CTAs may
+ * become resident while the preceding kernel on the stream finishes, but
+ * they read and write no memory before that kernel has completed and its
+ * writes are visible, so stream order holds as for a plain launch.
+ *
  * Errors: every argument check happens on the host before anything is
  * launched; a failing call writes nothing and returns the status.  A launch
  * failure returns ARNQ_ERR_CUDA (cudaGetLastError() holds the CUDA error).
