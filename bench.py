@@ -2,7 +2,7 @@
 """Benchmark of the fused add + RMSNorm + dynamic-quant operator on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload c2] [--no-cpu-baseline]
+                    [--workload c2] [--no-cpu-baseline] [--no-workloads]
 
 A step is one call of the operator (arnq_run) over one
 batch of the workload: by default the 8192 x 4096 bf16 configuration
@@ -21,7 +21,13 @@ Also printed, on the same JSON line: rows/s, the roofline of the kernel
 measured copy bandwidth), the end-to-end figure through the public call with
 host buffers (H2D copies, the call, D2H of the outputs, all inside the timed
 region), SM clocks sampled by NVML during the timed region, and the CPU
-oracle's throughput on a bounded sample (rank 0, one GPU only).
+oracle's throughput on a bounded sample (rank 0, one GPU only).  The
+`workloads` object carries the other configurations measured in the same
+run: the large ones (>= 80 % roofline class) as device time per call of calls
+back to back, the small, latency-bound ones as device time per call from a
+CUDA graph of back-to-back calls (L2-cold and L2-hot) and as host time per
+call.  The timed loops call arnq_run through ctypes with arguments marshalled
+once, so that the host keeps ahead of the device.
 
 --impl reference times the CPU oracle (the only other implementation of the
 operator; there is no runnable reference library) on the host cores.
@@ -266,10 +272,9 @@ def run_reference(args, w, on1, on2):
 # ---------------------------------------------------------------- our arm
 
 def launches_per_call(plan):
-    """Kernels one arnq_run call launches: the row kernel, which settles its own
-    rows when each row has one CTA; with a cluster per row, also the settle
-    kernel."""
-    return 1 if plan.cluster == 1 else 2
+    """Kernels one arnq_run call launches: the row kernel alone, whether a row
+    has one CTA or a cluster (each row is settled inside the kernel)."""
+    return 1
 
 
 def max_over_ranks(value_ms, dist, device):
@@ -287,6 +292,173 @@ def job_gbs(bytes_per_step, steps, world, total_ms):
     return bytes_per_step * steps * world / (total_ms / 1e3) / 1e9
 
 
+def outputs_of(w):
+    """(y1 produced, y2 produced) for a workload, by the outputMask rules."""
+    on1 = w.mask is None or w.mask[0]
+    on2 = (w.mask is not None and w.mask[1]) or (w.mask is None and w.smooth1 is not None
+                                                 and w.smooth2 is not None)
+    return on1, on2
+
+
+def sets_for(w, on1, on2, min_bytes=None, cap=2048):
+    """Buffer sets to rotate so that a call's inputs have left L2 before they are
+    read again: at least 3, and enough that the sets together move min_bytes."""
+    if min_bytes is None:
+        return 3
+    per = workload_bytes(w, on1, on2)
+    return int(min(cap, max(3, -(-min_bytes // per))))
+
+
+class DeviceRun:
+    """One workload resident on the device: `nsets` rotated buffer sets, the
+    parameters, a zeroed workspace, and the arnq_run arguments of every set
+    marshalled once (ctypes), so that a timed loop spends its host time in
+    the library's own launch path."""
+
+    def __init__(self, w, dev, stream, nsets=3):
+        import ctypes
+        import torch
+        from int4_quant_b200 import _abi as A
+        import int4_quant_b200 as q
+        self.w, self.dev, self.stream, self.A = w, dev, stream, A
+        self.on1, self.on2 = outputs_of(w)
+        TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}[w.dtype]
+        self.dt_code = A.ARNQ_BF16 if w.dtype == "bf16" else A.ARNQ_FP16
+        self.q_code = A.ARNQ_INT8 if w.qdtype == "int8" else A.ARNQ_INT4
+        self.mc = q.mask_code(w.mask)
+
+        def to_dev(bits):
+            if bits is None:
+                return None
+            t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
+            return t.to(dev).view(TDT)
+
+        cb = w.n if w.qdtype == "int8" else w.n // 2
+        self.params = [to_dev(a) for a in (w.gamma, w.beta, w.smooth1, w.smooth2)]
+        x1d, x2d = to_dev(w.x1), to_dev(w.x2)
+        self.sets = []
+        for i in range(nsets):
+            self.sets.append(dict(
+                x1=x1d if i == 0 else x1d.clone(), x2=x2d if i == 0 else x2d.clone(),
+                y1=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if self.on1 else None,
+                s1=torch.empty((w.rows,), dtype=torch.float32, device=dev) if self.on1 else None,
+                y2=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if self.on2 else None,
+                s2=torch.empty((w.rows,), dtype=torch.float32, device=dev) if self.on2 else None,
+                xo=torch.empty((w.rows, w.n), dtype=TDT, device=dev)))
+        st, self.ws_bytes = A.arnq_workspace_size(w.rows, w.n, self.dt_code, self.q_code, self.mc,
+                                                  w.smooth1 is not None, w.smooth2 is not None)
+        if st != A.ARNQ_OK:
+            raise A.ArnqError(st, "arnq_workspace_size")
+        self.ws = torch.zeros(self.ws_bytes, dtype=torch.uint8, device=dev)
+        self.fn = A.lib().arnq_run
+        self.args = [self._args(s, stream) for s in self.sets]
+        st, self.plan = A.arnq_make_plan(self.sets[0]["x1"], self.sets[0]["x2"], *self.params,
+                                         w.rows, w.n, self.dt_code, self.mc, self.q_code,
+                                         self.sets[0]["y1"], self.sets[0]["y2"],
+                                         self.sets[0]["xo"])
+        if st != A.ARNQ_OK:
+            raise A.ArnqError(st, "arnq_make_plan")
+        self.bytes = workload_bytes(w, self.on1, self.on2)
+
+    def _args(self, s, stream):
+        import ctypes
+        A = self.A
+        p = A._ptr
+        return (p(s["x1"]), p(s["x2"]), *[p(t) for t in self.params], self.w.rows, self.w.n,
+                self.dt_code, ctypes.c_float(self.w.eps), self.mc, self.q_code, p(s["y1"]),
+                p(s["s1"]), p(s["y2"]), p(s["s2"]), p(s["xo"]), p(self.ws), self.ws_bytes,
+                A._stream(stream))
+
+    def launch(self, i, args=None):
+        st = self.fn(*(args or self.args)[i % len(self.sets)])
+        if st:
+            raise self.A.ArnqError(st, "arnq_run")
+
+    def status(self):
+        """(code, row, counters) of the workspace status block (synchronizes)."""
+        h = self.ws[:32].cpu().numpy().view(np.int32)
+        return int(h[0]), int(h[2:4].view(np.int64)[0]), [int(v) for v in h[4:7]]
+
+    def check_status(self):
+        code, row, ctr = self.status()
+        if code != 0 or any(ctr):
+            raise RuntimeError(f"{self.w.name}: device status {code} (row {row}), counters {ctr}")
+
+    def timed(self, steps, warmup):
+        """Mean device time of one call over `steps` calls back to back (one CUDA
+        event pair on the launching stream: the calls are programmatic
+        dependents of one another, and an event between two would separate
+        them), after `warmup` calls."""
+        import torch
+        for i in range(warmup):
+            self.launch(i)
+        torch.cuda.synchronize(self.dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(self.stream)
+        for i in range(steps):
+            self.launch(i)
+        e1.record(self.stream)
+        torch.cuda.synchronize(self.dev)
+        return e0.elapsed_time(e1) / steps
+
+    def graph_timed(self, calls, replays=20):
+        """Device time of one call when `calls` calls (rotating the buffer sets)
+        run back to back from a CUDA graph: no host enqueue in the way, as a
+        decode loop captured in a graph sees it.  Returns the median over
+        replays of (replay time / calls) in ms."""
+        import torch
+        side = torch.cuda.Stream(self.dev)
+        args = [self._args(s, side) for s in self.sets]
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(side):
+            for i in range(3):
+                self.launch(i, args)
+        torch.cuda.synchronize(self.dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            for i in range(calls):
+                self.launch(i, args)
+        g.replay()
+        torch.cuda.synchronize(self.dev)
+        out = []
+        for _ in range(replays):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(self.stream)
+            g.replay()
+            e1.record(self.stream)
+            torch.cuda.synchronize(self.dev)
+            out.append(e0.elapsed_time(e1) / calls)
+        del g
+        return statistics.median(out)
+
+    def host_us(self, calls=2000):
+        """Host time of one call of arnq_run (argument checks, plan lookup and
+        launch), from Python through ctypes, calls issued back to back."""
+        import torch
+        for i in range(10):
+            self.launch(i)
+        t0 = time.perf_counter()
+        for i in range(calls):
+            self.launch(i)
+        t1 = time.perf_counter()
+        torch.cuda.synchronize(self.dev)
+        return (t1 - t0) / calls * 1e6
+
+
+def workload_entry(run, ms, peak, how):
+    """One line of the `workloads` object: a call's time, throughput, roofline."""
+    gbs = run.bytes / (ms / 1e3) / 1e9
+    return {"us_per_call": ms * 1e3, "gbs": gbs, "frac": gbs / peak,
+            "rows_per_s": run.w.rows / (ms / 1e3), "bytes_per_call": run.bytes,
+            "plan": run.plan.as_dict(), "timing": how}
+
+
+SMALL = ("c1", "c5a", "c5b", "c5c")     # latency-bound: device time per call from a graph
+LARGE = ("c2", "c3", "c4", "c5d")       # the >= 80 % roofline class
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -296,6 +468,8 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the other workloads' lines (the `workloads` object)")
     ap.add_argument("--sets", type=int, default=3, help="rotated buffer sets")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -303,9 +477,7 @@ def main():
 
     from int4_quant_b200 import workloads as wl
     w = wl.CONFIGS[args.workload]()
-    on1 = w.mask is None or w.mask[0]
-    on2 = (w.mask is not None and w.mask[1]) or (w.mask is None and w.smooth1 is not None
-                                                 and w.smooth2 is not None)
+    on1, on2 = outputs_of(w)
     if args.impl == "reference":
         return run_reference(args, w, on1, on2)
 
@@ -327,46 +499,9 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
 
     A.lib()
-    TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}[w.dtype]
-    dt_code = A.ARNQ_BF16 if w.dtype == "bf16" else A.ARNQ_FP16
-    q_code = A.ARNQ_INT8 if w.qdtype == "int8" else A.ARNQ_INT4
-    mc = q.mask_code(w.mask)
-
-    def to_dev(bits):
-        if bits is None:
-            return None
-        t = torch.from_numpy(np.ascontiguousarray(bits).view(np.int16))
-        return t.to(dev).view(TDT)
-
-    cb = w.n if w.qdtype == "int8" else w.n // 2
-    params = [to_dev(a) for a in (w.gamma, w.beta, w.smooth1, w.smooth2)]
-    x1h, x2h = w.x1, w.x2
-    sets = []
-    for _ in range(args.sets):
-        sets.append(dict(
-            x1=to_dev(x1h), x2=to_dev(x2h),
-            y1=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if on1 else None,
-            s1=torch.empty((w.rows,), dtype=torch.float32, device=dev) if on1 else None,
-            y2=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev) if on2 else None,
-            s2=torch.empty((w.rows,), dtype=torch.float32, device=dev) if on2 else None,
-            xo=torch.empty((w.rows, w.n), dtype=TDT, device=dev)))
-    ws_bytes = A.arnq_workspace_size(w.rows, w.n, dt_code, q_code, mc, w.smooth1 is not None,
-                                     w.smooth2 is not None)[1]
-    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
-    sptr = stream.cuda_stream
-
-    def launch(s):
-        st = A.arnq_run(s["x1"], s["x2"], params[0], params[1], params[2], params[3], w.rows, w.n,
-                        dt_code, w.eps, mc, q_code, s["y1"], s["s1"], s["y2"], s["s2"], s["xo"], ws,
-                        ws_bytes, sptr)
-        if st != A.ARNQ_OK:
-            raise A.ArnqError(st, "arnq_run")
-
-    st, plan = A.arnq_make_plan(sets[0]["x1"], sets[0]["x2"], *params, w.rows, w.n, dt_code, mc,
-                                q_code, sets[0]["y1"], sets[0]["y2"], sets[0]["xo"])
-    if st != A.ARNQ_OK:
-        raise A.ArnqError(st, "arnq_make_plan")
+    run = DeviceRun(w, dev, stream, nsets=args.sets)
+    plan = run.plan
 
     def barrier():
         torch.cuda.synchronize(dev)
@@ -376,7 +511,7 @@ def main():
 
     # ---- warm-up
     for i in range(args.warmup):
-        launch(sets[i % args.sets])
+        run.launch(i)
     barrier()
 
     # ---- timed region: exactly K steps, back to back on the stream (one event
@@ -385,23 +520,21 @@ def main():
     K = args.steps
     ev0 = torch.cuda.Event(enable_timing=True)
     ev1 = torch.cuda.Event(enable_timing=True)
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(local, period=0.0005)
     clocks.start()
     barrier()
     ev0.record(stream)
     for i in range(K):
-        launch(sets[i % args.sets])
+        run.launch(i)
     ev1.record(stream)
     barrier()
     clocks.stop()
     total_ms = ev0.elapsed_time(ev1)
-    wsh = ws[:16].cpu().numpy().view(np.int32)
-    if wsh[0] != 0:
-        raise RuntimeError(f"kernel reported device status {wsh[0]}")
+    run.check_status()
     local_ms = total_ms
     total_ms = max_over_ranks(total_ms, dist, dev)
 
-    nbytes = workload_bytes(w, on1, on2)
+    nbytes = run.bytes
     value = job_gbs(nbytes, K, world, total_ms)
     rows_per_s = w.rows * K * world / (total_ms / 1e3)
     # this rank's mean duration of one call (its kernels run back to back)
@@ -411,17 +544,18 @@ def main():
 
     # ---- end to end through the public call, host buffers, copies timed
     e2e_steps = max(1, args.e2e_steps)
-    x1p = torch.from_numpy(np.ascontiguousarray(x1h).view(np.int16)).view(TDT).pin_memory()
-    x2p = torch.from_numpy(np.ascontiguousarray(x2h).view(np.int16)).view(TDT).pin_memory()
+    TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}[w.dtype]
+    x1p = torch.from_numpy(np.ascontiguousarray(w.x1).view(np.int16)).view(TDT).pin_memory()
+    x2p = torch.from_numpy(np.ascontiguousarray(w.x2).view(np.int16)).view(TDT).pin_memory()
     outs_h = {}
-    s0 = sets[0]
-    for k, t in (("y1", s0["y1"]), ("s1", s0["s1"]), ("y2", s0["y2"]), ("s2", s0["s2"]),
-                 ("xo", s0["xo"])):
+    ge = run.sets[0]
+    params = run.params
+    for k in ("y1", "s1", "y2", "s2", "xo"):
+        t = ge[k]
         if t is not None:
             outs_h[k] = torch.empty(t.shape, dtype=t.dtype).pin_memory()
     h2d = x1p.numel() * 2 * 2
     d2h = sum(t.numel() * t.element_size() for t in outs_h.values())
-    ge = s0
 
     def e2e_step():
         ge["x1"].copy_(x1p, non_blocking=True)
@@ -447,6 +581,49 @@ def main():
     e2e_ms = e_start.elapsed_time(e_end)
     e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     e2e_value = job_gbs(nbytes, e2e_steps, world, e2e_ms)
+    headline_plan = plan.as_dict()
+    del run
+    torch.cuda.empty_cache()
+
+    # ---- the other workloads, in the same run (this rank alone; device time of
+    # one call).  Large ones: K' calls back to back, 3 rotated sets (each call's
+    # inputs have left L2 when they come round again).  Small ones (latency):
+    # a CUDA graph of back-to-back calls, on L2-cold rotated sets and on one
+    # L2-hot set; plus the host time of one call.
+    workloads = None
+    wl_clocks = ClockSampler(local, period=0.002)
+    if not args.no_workloads:
+        workloads = {}
+        wl_clocks.start()
+        for name in LARGE:
+            if name == args.workload:
+                continue
+            wr = DeviceRun(wl.CONFIGS[name](), dev, stream, nsets=3)
+            ms = wr.timed(steps=200, warmup=20)
+            wr.check_status()
+            workloads[name] = workload_entry(wr, ms, peak, "200 calls back to back, 3 sets")
+            workloads[name]["workload"] = wr.w.name
+            del wr
+            torch.cuda.empty_cache()
+        for name in SMALL:
+            ww = wl.CONFIGS[name]()
+            o1, o2 = outputs_of(ww)
+            nsets = sets_for(ww, o1, o2, min_bytes=300 << 20)
+            wr = DeviceRun(ww, dev, stream, nsets=nsets)
+            cold = wr.graph_timed(calls=nsets)
+            wr.check_status()
+            e = workload_entry(wr, cold, peak, f"CUDA graph of {nsets} calls on {nsets} rotated "
+                                                f"sets (L2-cold), median of 20 replays")
+            hot_run = DeviceRun(ww, dev, stream, nsets=1)
+            hot = hot_run.graph_timed(calls=256)
+            hot_run.check_status()
+            e["hot_us_per_call"] = hot * 1e3
+            e["host_us_per_call"] = hot_run.host_us()
+            e["workload"] = ww.name
+            workloads[name] = e
+            del wr, hot_run
+            torch.cuda.empty_cache()
+        wl_clocks.stop()
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -479,7 +656,7 @@ def main():
             "smooth1": w.smooth1 is not None, "smooth2": w.smooth2 is not None, "eps": w.eps,
             "l2": f"{args.sets} rotated buffer sets, inputs {2 * w.rows * w.n * 2 / 1e6:.0f} MB "
                   f"per set (> 126 MB L2)",
-            "plan": plan.as_dict(),
+            "plan": headline_plan,
             "parallelism": f"replicas x{world} (rows independent; no collective)",
         },
         "rows_per_s": rows_per_s,
@@ -491,11 +668,10 @@ def main():
             "peak": peak,
             "unit": "GB/s",
             "frac": achieved / peak,
-            "traffic": recorded_traffic(w.name, plan.as_dict()),
+            "traffic": recorded_traffic(w.name, headline_plan),
             "peak_kind": peak_kind,
-            "kernel": ("arnq::rows_kernel (one arnq_run call; rows settled in the kernel's tail)"
-                       if plan.cluster == 1 else
-                       "arnq::rows_kernel + arnq::settle_kernel (one arnq_run call)"),
+            "kernel": "arnq::rows_kernel (one launch per arnq_run call; rows settled in the "
+                      "kernel, one row behind)",
             "mean_call_us": mean_launch_ms * 1e3,
             "launches_per_call": launches_per_call(plan),
         },
@@ -505,6 +681,8 @@ def main():
                 "ms_per_step": e2e_ms / e2e_steps},
         "gpu_launches": K * launches_per_call(plan),
         "clocks": clocks.summary(),
+        "workloads": workloads,
+        "workloads_clocks": wl_clocks.summary() if workloads is not None else None,
     }
     print(json.dumps(line), flush=True)
     return 0

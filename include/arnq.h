@@ -26,7 +26,8 @@
  *     rounded half-to-even and clamped to [-Q, Q].  A row whose scale is 0
  *     (all inputs 0) gets scale 0 and all codes 0.
  *   - INT4 codes are two's-complement nibbles packed two per byte, the even
- *     column in the low nibble; an INT4 row of n codes occupies n/2 bytes.
+ *     column in the low nibble; an INT4 row of n codes occupies n/2 bytes
+ *     (or n/8 int32 words of eight codes: see arnq_qdtype).
  *   - Results are deterministic: the same inputs and the same plan give the
  *     same bits on every run ("Deterministic compute" in the Constraints
  *     section).  Sums are fixed-order trees; there are no float atomics.
@@ -34,7 +35,8 @@
  * Layout: every tensor is dense row-major ("ND" in the Constraints section).
  *   x1, x2, xOut : [rows, n] of dtype (bf16 or fp16)
  *   gamma, beta, smooth1, smooth2 : [n] of dtype
- *   y1, y2 : [rows, n] int8, or [rows, n/2] bytes of packed INT4
+ *   y1, y2 : [rows, n] int8, [rows, n/2] bytes of packed INT4, or
+ *            [rows, n/8] int32 words of eight INT4 codes
  *   scale1, scale2 : [rows] binary32
  *
  * Ownership: the caller owns every buffer.  All tensor pointers are DEVICE
@@ -45,20 +47,20 @@
  * as x1 or x2 (in-place residual update); any other overlap between an
  * output and an input is undefined.
  *
- * Launches: one kernel per call when each row is handled by one CTA, two
- * (the row kernel, then a small settle kernel) when a thread-block cluster
- * shares each row.  The row kernel is launched as a programmatic dependent
- * launch (cudaLaunchAttributeProgrammaticStreamSerialization): its CTAs may
- * become resident while the preceding kernel on the stream finishes, but
- * they read and write no memory before that kernel has completed and its
- * writes are visible, so stream order holds as for a plain launch.
+ * Launches: one kernel per call, whether a row is handled by one CTA or by a
+ * thread-block cluster.  It is launched as a programmatic dependent launch
+ * (cudaLaunchAttributeProgrammaticStreamSerialization): its CTAs may become
+ * resident while the preceding kernel on the stream finishes, but they read
+ * and write no memory before that kernel has completed and its writes are
+ * visible, so stream order holds as for a plain launch.
  *
  * Errors: every argument check happens on the host before anything is
  * launched; a failing call writes nothing and returns the status.  A launch
  * failure returns ARNQ_ERR_CUDA (cudaGetLastError() holds the CUDA error).
- * Kernels that wait on asynchronous copies do so with a time limit; if a wait
- * expires the kernel stops early and records ARNQ_ERR_DEVICE_TIMEOUT in the
- * workspace's status block (see arnq_workspace_status).
+ * Kernels that wait on asynchronous copies do so with a time limit (1 s
+ * unless a plan sets wait_limit_us); if a wait expires the kernel stops early
+ * and records ARNQ_ERR_DEVICE_TIMEOUT in the workspace's status block (see
+ * arnq_workspace_status).
  */
 #ifndef ARNQ_H
 #define ARNQ_H
@@ -80,19 +82,32 @@ typedef enum arnq_status {
   ARNQ_OK = 0,
   ARNQ_ERR_NULL_PTR = 1,        /* a required input, or a selected output, is NULL        */
   ARNQ_ERR_EMPTY = 2,           /* rows == 0 or n == 0: empty tensors are not supported    */
-  ARNQ_ERR_SHAPE = 3,           /* INT4 with odd n; n above ARNQ_MAX_N; negative sizes     */
+  ARNQ_ERR_SHAPE = 3,           /* n not a multiple of 2 (INT4) or 8 (INT4_INT32); n above
+                                   ARNQ_MAX_N; negative sizes                              */
   ARNQ_ERR_DTYPE = 4,           /* unknown dtype or qdtype                                 */
   ARNQ_ERR_MASK = 5,            /* outputMask / smooth-scale combination the page forbids  */
   ARNQ_ERR_EPS = 6,             /* epsilon negative or not finite                          */
-  ARNQ_ERR_ALIGN = 7,           /* a 16-bit tensor not 2-byte aligned, a scale not 4-byte  */
+  ARNQ_ERR_ALIGN = 7,           /* a 16-bit tensor not 2-byte aligned, a scale (or an
+                                   INT4_INT32 output) not 4-byte aligned                   */
   ARNQ_ERR_WORKSPACE = 8,       /* workspace NULL or smaller than arnq_workspace_size()    */
   ARNQ_ERR_CUDA = 9,            /* a CUDA call failed (launch, attribute, device query)    */
   ARNQ_ERR_PLAN = 10,           /* an explicit plan that cannot run this problem           */
-  ARNQ_ERR_DEVICE_TIMEOUT = 11  /* reported through the workspace status block only        */
+  ARNQ_ERR_DEVICE_TIMEOUT = 11, /* reported through the workspace status block only        */
+  ARNQ_ERR_WORKSPACE_STATE = 12 /* status block only: the workspace was not zero-filled    */
 } arnq_status;
 
 typedef enum arnq_dtype { ARNQ_BF16 = 0, ARNQ_FP16 = 1 } arnq_dtype;
-typedef enum arnq_qdtype { ARNQ_INT8 = 0, ARNQ_INT4 = 1 } arnq_qdtype;
+/* Code types of y1 and y2 ("aclnnAddRmsNormDynamicQuantV2", Formula: y1Out is
+ * INT8 or INT4; the page fixes no INT4 container):
+ *   ARNQ_INT8        int8 [rows, n]
+ *   ARNQ_INT4        bytes [rows, n/2], two codes a byte, even column in the
+ *                    low nibble (n even)
+ *   ARNQ_INT4_INT32  int32 [rows, n/8], eight codes a 32-bit word, column
+ *                    8w + k of a row in bits 4k .. 4k+3 of its word w (n a
+ *                    multiple of 8; y 4-byte aligned).  On a little-endian
+ *                    device its bytes are those of ARNQ_INT4.
+ * INT4 codes are two's-complement nibbles in [-7, 7]. */
+typedef enum arnq_qdtype { ARNQ_INT8 = 0, ARNQ_INT4 = 1, ARNQ_INT4_INT32 = 2 } arnq_qdtype;
 
 /* outputMask encoding: ARNQ_MASK_ABSENT means "outputMaskOptional not given";
  * otherwise bit 0 is outputMask[0] (y1) and bit 1 is outputMask[1] (y2). */
@@ -120,14 +135,16 @@ ARNQ_API arnq_status arnq_selected_outputs(int out_mask, int has_smooth1, int ha
                                   int *y2_on);
 
 /* Workspace bytes arnq_run needs for this problem (first phase of the pages'
- * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize"):
- * 256 + rows * R, R = 80 + 4 * (12 + ceil(n * nout / 256)) rounded up to a
- * multiple of 16, nout = outputs produced.  The workspace holds a 16-byte status block, which the kernels
- * write only on error, and one record per row that the call writes and reads
- * back (the row's fp64 sum of squares and the few units the binary32
- * arithmetic cannot settle).  The caller allocates it on the device and
- * zero-fills the status block once; it may be reused for any number of calls
- * on one stream (not by calls that overlap).  Validates the same arguments as
+ * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize"): 256 for
+ * every valid problem.  The workspace holds the status block (bytes 0-15, see
+ * arnq_workspace_status), which the kernels write only on error, and three
+ * row hand-out counters (bytes 16-27) that every call leaves at zero; the
+ * per-row bookkeeping of the exact scales stays in on-chip shared memory.
+ * The caller allocates it on the device (8-byte aligned) and zero-fills all
+ * 256 bytes once; it may then be reused for any number of calls on one
+ * stream (not by calls that overlap).  A call that finds the counters not at
+ * zero records ARNQ_ERR_WORKSPACE_STATE in the status block (its outputs are
+ * then unreliable) and leaves them at zero.  Validates the same arguments as
  * arnq_run (except pointers).  Host only. */
 ARNQ_API arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdtype qdt,
                                 int out_mask, int has_smooth1, int has_smooth2, size_t *bytes);
@@ -171,8 +188,9 @@ ARNQ_API arnq_status arnq_rms_norm_dynamic_quant(const void *x, const void *gamm
                                         void *stream);
 
 /* Status block at the start of the workspace.  code is 0 (ARNQ_OK) until a
- * kernel records an error; the library never clears it.  row is the first
- * row the failing kernel did not finish.  Read it with a device-to-host copy
+ * kernel records an error (ARNQ_ERR_DEVICE_TIMEOUT, ARNQ_ERR_WORKSPACE_STATE);
+ * the library never clears it.  row is the first row the failing kernel did
+ * not finish (-1 when no row applies).  Read it with a device-to-host copy
  * after synchronizing the stream; zero it to re-arm. */
 typedef struct arnq_workspace_status {
   int32_t code;
@@ -199,13 +217,27 @@ typedef struct arnq_plan {
   int32_t units;         /* units per thread: 1, 2, 4 (16-byte) or 1, 4, 8 (pairs) */
   int32_t stages;        /* staged kernel: rows in flight per CTA (1..8)        */
   int32_t ctas_per_sm;   /* resident CTAs per SM the grid is sized for         */
-  int32_t grid;          /* CTAs launched (output; multiple of cluster)        */
+  int32_t grid;          /* CTAs launched (multiple of cluster); 0 = as many
+                            clusters as cover the rows with equal row counts */
   int32_t vector;        /* output: 1 if 16-byte vector loads are used         */
+  int32_t wait_limit_us; /* bounded device waits give up after this many us;
+                            0 = 1 s                                          */
+  int32_t test_hold_bytes; /* testing only (staged kernel): the first copy's
+                            barrier of every CTA expects this many bytes more
+                            than its copies bring, so that wait runs out and
+                            the call records ARNQ_ERR_DEVICE_TIMEOUT; at most
+                            65536; 0 in normal use                           */
+  int32_t schedule;      /* 1: rows dealt out to CTAs in turn; 2: the last
+                            quarter of the rows handed out one at a time to
+                            whichever CTA is free (staged kernel, one CTA per
+                            row, at least two rows per CTA); 0 = choose      */
 } arnq_plan;
 
 /* Fills *plan with the plan arnq_run would use for these arguments (pointers
  * are only inspected for alignment).  Fields of *plan that are nonzero on
- * entry are kept as requested.  Queries the current device. */
+ * entry are kept as requested.  Queries the current device.  A requested grid
+ * larger than the resident clusters runs in waves; one with more clusters
+ * than rows leaves the extra clusters idle. */
 ARNQ_API arnq_status arnq_make_plan(const void *x1, const void *x2, const void *gamma, const void *beta,
                            const void *smooth1, const void *smooth2, int64_t rows, int64_t n,
                            arnq_dtype dt, int out_mask, arnq_qdtype qdt, const void *y1,
@@ -223,27 +255,31 @@ ARNQ_API arnq_status arnq_run_planned(const void *x1, const void *x2, const void
 /* ---- no-allocation variant ----------------------------------------------
  *
  * The paper has no counterpart: the pages' two-phase call always takes a
- * caller-allocated workspace.  This entry point is arnq_run with the workspace
- * replaced by a file-scope device array inside the library
- * (ARNQ_STATIC_SCRATCH_BYTES = 4 MiB per device; arnq_workspace_size tells
- * whether a problem fits: about 21000 rows of 4096 columns, one output),
- * so a caller that cannot allocate
- * (no allocator at hand, a fixed memory budget) still gets the operator.
+ * caller-allocated workspace.  Some callers cannot allocate device memory at
+ * the point of the call: code running under a fixed memory budget, a caller
+ * with no allocator at hand (a plain C host program that owns no CUDA
+ * allocator, or one whose framework's caching allocator must not be bypassed),
+ * or a caller that would otherwise have to allocate and free around every
+ * call.  This entry point is arnq_run with the workspace replaced by a
+ * file-scope device array inside the library, ARNQ_STATIC_SCRATCH_BYTES per
+ * device, held by every GPU that loads the library until the process exits.
  * It allocates nothing: no cudaMalloc / cudaFree and no allocating library
  * routine.  Arguments and results are those of arnq_run; in addition
  *   - ARNQ_ERR_WORKSPACE if the problem needs more scratch than
- *     ARNQ_STATIC_SCRATCH_BYTES (arnq_workspace_size larger than the array);
+ *     ARNQ_STATIC_SCRATCH_BYTES (arnq_workspace_size larger than the array;
+ *     no valid problem does today: it needs 256 bytes);
  *   - ARNQ_ERR_CUDA if the array's device address cannot be obtained
- *     (cudaGetSymbolAddress fails) or its set-up fails.
- * The status block at the start of the array must be zero when a kernel
- * starts: every call clears it first (an async memset on `stream`).  The first
- * call on each device does set-up (looks up the array's address and zeroes
- * it, synchronously): make it before any stream capture.  The array is shared
- * by every call on a device: calls that overlap (other streams, other host
+ *     (cudaGetSymbolAddress fails).
+ * Every call looks up the array's address for the current device (so a device
+ * reset between calls does no harm) and clears the status block at its start
+ * with an async memset on `stream` before the kernel.  The first call on a
+ * device may load the library's device code: make it before any stream
+ * capture.  The array is shared by every call on a device and keeps the last
+ * call's contents: calls that overlap on the GPU (other streams, other host
  * threads) race on it; serialise them.  A device-side timeout status lands in
  * the array and is not readable from the host: use arnq_run with a workspace
  * where that status matters. */
-#define ARNQ_STATIC_SCRATCH_BYTES (4 << 20)
+#define ARNQ_STATIC_SCRATCH_BYTES 4096
 ARNQ_API arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *gamma,
                                     const void *beta, const void *smooth1, const void *smooth2,
                                     int64_t rows, int64_t n, arnq_dtype dt, float eps,

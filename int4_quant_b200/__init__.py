@@ -17,7 +17,20 @@ from . import _abi
 from ._abi import ArnqError  # noqa: F401
 
 _DT = {"torch.bfloat16": _abi.ARNQ_BF16, "torch.float16": _abi.ARNQ_FP16}
-_QDT = {"int8": _abi.ARNQ_INT8, "int4": _abi.ARNQ_INT4}
+_QDT = {"int8": _abi.ARNQ_INT8, "int4": _abi.ARNQ_INT4, "int4_int32": _abi.ARNQ_INT4_INT32}
+
+
+def _codes_like(lead, n, qdtype):
+    """(shape, torch dtype) of a quantized output: int8 [..., n], packed uint8
+    [..., n/2], or int32 [..., n/8] words of eight INT4 codes."""
+    import torch
+    if qdtype == "int8":
+        return lead + (n,), torch.int8
+    if qdtype == "int4_int32":
+        return lead + (n // 8,), torch.int32
+    if qdtype == "int4":
+        return lead + (n // 2,), torch.uint8
+    raise ValueError(f"unknown qdtype {qdtype!r}")
 _workspaces = {}
 
 
@@ -68,9 +81,11 @@ def add_rms_norm_dynamic_quant(x1, x2, gamma, beta=None, smooth1=None, smooth2=N
 
     x1, x2: [..., n] bf16 or fp16; gamma, beta, smooth1, smooth2: [n] same dtype.
     Returns (y1, scale1, y2, scale2, x_out); an output that is not selected is
-    None.  y is int8 [..., n] or, for qdtype="int4", uint8 [..., n/2] holding
-    two codes per byte (even column in the low nibble).  `out` may pass
-    preallocated tensors under the same keys.
+    None.  y is int8 [..., n]; for qdtype="int4", uint8 [..., n/2] holding
+    two codes per byte (even column in the low nibble); for
+    qdtype="int4_int32", int32 [..., n/8] holding eight codes per word (column
+    8w + k in bits 4k..4k+3).  `out` may pass preallocated tensors under the
+    same keys.
     """
     import torch
     _check(x1, "x1")
@@ -87,8 +102,7 @@ def add_rms_norm_dynamic_quant(x1, x2, gamma, beta=None, smooth1=None, smooth2=N
     if st != _abi.ARNQ_OK:
         raise ArnqError(st, "arnq_selected_outputs")
     lead = tuple(x1.shape[:-1])
-    cshape = lead + ((n,) if qdtype == "int8" else (n // 2,))
-    cdt = torch.int8 if qdtype == "int8" else torch.uint8
+    cshape, cdt = _codes_like(lead, n, qdtype)
     out = dict(out or {})
 
     def alloc(key, shape, dtype, on):
@@ -130,9 +144,8 @@ def rms_norm_dynamic_quant(x, gamma, beta=None, smooth=None, *, eps: float = 1e-
     n = x.shape[-1]
     rows = x.numel() // n if n else 0
     lead = tuple(x.shape[:-1])
-    cshape = lead + ((n,) if qdtype == "int8" else (n // 2,))
-    y = torch.empty(cshape, dtype=torch.int8 if qdtype == "int8" else torch.uint8,
-                    device=x.device)
+    cshape, cdt = _codes_like(lead, n, qdtype)
+    y = torch.empty(cshape, dtype=cdt, device=x.device)
     scale = torch.empty(lead, dtype=torch.float32, device=x.device)
     st, nbytes = _abi.arnq_workspace_size(rows, n, _DT[str(dt)], _QDT[qdtype],
                                           _abi.ARNQ_MASK_ABSENT, smooth is not None, False)

@@ -18,28 +18,18 @@ namespace {
 using arnq::KParams;
 using arnq::KernelFn;
 
-// workspace: the status block (padded to kRecordBase), then one record per row
-size_t workspace_bytes_for(int64_t rows, int64_t n, int nout) {
-  const int rec = arnq::record_bytes(arnq::tie_cap(static_cast<int>(n), nout));
-  return static_cast<size_t>(arnq::kRecordBase) +
-         static_cast<size_t>(rows) * static_cast<size_t>(rec);
-}
+// workspace: the status block only (the row records live in shared memory),
+// whatever the problem
+size_t workspace_bytes_for() { return static_cast<size_t>(arnq::kStatusBytes); }
 constexpr int kMaxStages = arnq::kMaxStagesDev;
 constexpr int kMaxCluster = 16;
-constexpr int kSettleRowsPerBlock = 16;  // settle kernel: 16 lanes per row, 256 threads
 
 // ---------------------------------------------------------------- kernel table
 
 struct KernelTable {
   KernelFn fn[2][2][arnq::kTableSize];  // [dtype][qdtype][...]
-  arnq::SettleFn settle[2][2][arnq::kSettleSize];
   KernelTable() {
     std::memset(fn, 0, sizeof fn);
-    std::memset(settle, 0, sizeof settle);
-    arnq::fill_settle_bf16_int8(settle[0][0]);
-    arnq::fill_settle_bf16_int4(settle[0][1]);
-    arnq::fill_settle_fp16_int8(settle[1][0]);
-    arnq::fill_settle_fp16_int4(settle[1][1]);
     arnq::fill_table_bf16_int8(fn[0][0]);
     arnq::fill_table_bf16_int4(fn[0][1]);
     arnq::fill_table_fp16_int8(fn[1][0]);
@@ -56,12 +46,12 @@ const KernelTable &kernel_table() {
   return table;
 }
 
-arnq::SettleFn lookup_settle(int dt, int qdt, int nout, bool add, bool vec) {
-  if (nout < 1 || nout > 2) return nullptr;
-  return kernel_table().settle[dt][qdt][arnq::settle_index(nout, add, vec)];
-}
-
+// The eight-codes-per-word INT4 container has the byte layout of packed INT4
+// on a little-endian device (code 8w + k in bits 4k..4k+3 of word w is the
+// low nibble of byte 4w + k/2 for even k, the high nibble for odd k): the
+// INT4 kernels write it.
 KernelFn lookup(int dt, int qdt, int nout, bool add, int mode, int upt, int cluster) {
+  if (qdt == ARNQ_INT4_INT32) qdt = ARNQ_INT4;
   const KernelTable &table = kernel_table();
   const int s = arnq::upt_slot(mode, upt);
   if (s < 0 || nout < 1 || nout > 2) return nullptr;
@@ -166,12 +156,13 @@ arnq_status selected(int out_mask, int has_s1, int has_s2, int *on1, int *on2) {
 
 arnq_status check_shape(int64_t rows, int64_t n, int dt, int qdt, float eps) {
   if (dt != ARNQ_BF16 && dt != ARNQ_FP16) return ARNQ_ERR_DTYPE;
-  if (qdt != ARNQ_INT8 && qdt != ARNQ_INT4) return ARNQ_ERR_DTYPE;
+  if (qdt != ARNQ_INT8 && qdt != ARNQ_INT4 && qdt != ARNQ_INT4_INT32) return ARNQ_ERR_DTYPE;
   if (rows < 0 || n < 0) return ARNQ_ERR_SHAPE;
   if (rows > INT32_MAX) return ARNQ_ERR_SHAPE;  // row indices are 32-bit in the kernels' lists
   if (rows == 0 || n == 0) return ARNQ_ERR_EMPTY;
   if (n > ARNQ_MAX_N) return ARNQ_ERR_SHAPE;
   if (qdt == ARNQ_INT4 && (n % 2) != 0) return ARNQ_ERR_SHAPE;
+  if (qdt == ARNQ_INT4_INT32 && (n % 8) != 0) return ARNQ_ERR_SHAPE;
   if (!(eps >= 0.0f) || !std::isfinite(eps)) return ARNQ_ERR_EPS;
   return ARNQ_OK;
 }
@@ -201,9 +192,9 @@ arnq_status validate(Problem &P, int out_mask, const void *workspace, size_t wor
   for (const void *q : h16)
     if (q && !aligned(q, 2)) return ARNQ_ERR_ALIGN;
   if ((P.on1 && !aligned(P.scale1, 4)) || (P.on2 && !aligned(P.scale2, 4))) return ARNQ_ERR_ALIGN;
-  if (!workspace ||
-      workspace_bytes < workspace_bytes_for(P.rows, P.n, (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0)))
-    return ARNQ_ERR_WORKSPACE;
+  if (P.qdt == ARNQ_INT4_INT32 && ((P.on1 && !aligned(P.y1, 4)) || (P.on2 && !aligned(P.y2, 4))))
+    return ARNQ_ERR_ALIGN;
+  if (!workspace || workspace_bytes < workspace_bytes_for()) return ARNQ_ERR_WORKSPACE;
   if (!aligned(workspace, 8)) return ARNQ_ERR_ALIGN;
   return ARNQ_OK;
 }
@@ -230,7 +221,8 @@ bool vector_ok(const Problem &P) {
 struct Launch {
   KernelFn fn;
   int smem, seg, units;
-  int tail_rows, trec_bytes;  // in-kernel settling (tail_rows > 0) or the settle kernel
+  int rec_bytes;     // bytes of one row record (three live in shared memory)
+  int64_t dyn_base;  // first row handed out by the workspace counter (rows: none)
 };
 
 int upt_candidate(int mode, int i) {
@@ -238,12 +230,12 @@ int upt_candidate(int mode, int i) {
   return mode == arnq::LOAD_SCALAR ? sca[i] : vec[i];
 }
 
-// Shared memory of one CTA: the exchange slots, the in-kernel row records (tail
-// plans), then (staged) the input ring.
+// Shared memory of one CTA: the exchange slots, three row records, B_k of
+// 16-byte units, then (staged) the input ring.
 int smem_bytes(int mode, int upt, int cl, int threads, int nout, int stages, int stage_bytes,
-               int tail_rows = 0, int trec_bytes = 0) {
+               int rec_bytes) {
   const arnq::Layout lay = arnq::make_layout(
-      cl * (threads / 32), nout, stages, tail_rows, trec_bytes,
+      cl * (threads / 32), nout, stages, rec_bytes,
       arnq::bsm_bytes_for(mode != arnq::LOAD_SCALAR, nout, upt, threads));
   return lay.ring + stages * stage_bytes;
 }
@@ -256,10 +248,21 @@ arnq_status occupancy(KernelFn fn, int threads, int smem, int *per_sm) {
   return ARNQ_OK;
 }
 
+// Requested plan fields that no plan can take (checked before any device query).
+arnq_status check_plan_fields(const arnq_plan &q) {
+  if (q.wait_limit_us < 0 || q.test_hold_bytes < 0 || q.test_hold_bytes > 65536 || q.grid < 0 ||
+      q.ctas_per_sm < 0 || q.schedule < 0 || q.schedule > 2 || q.stages < 0 || q.threads < 0 ||
+      q.units < 0 || q.cluster < 0)
+    return ARNQ_ERR_PLAN;
+  return ARNQ_OK;
+}
+
 arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
+  arnq_status st = check_plan_fields(*pl);
+  if (st != ARNQ_OK) return st;
   DeviceInfo di;
   int dev = 0;
-  arnq_status st = device_info(&di, &dev);
+  st = device_info(&di, &dev);
   if (st != ARNQ_OK) return st;
   const bool vec = vector_ok(P);
   const int nout = (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0);
@@ -304,6 +307,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   const int seg = static_cast<int>(ceil_div(units, cl));
   if (seg > max_seg) return ARNQ_ERR_PLAN;
   const int stage_bytes = nin * seg * 16;
+  const int rec = arnq::rec_slot_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
 
   // units per thread: of the variants whose threads hold a slice, the one with
   // the most CTAs (rows in flight) per SM, then the most units per thread
@@ -319,7 +323,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       KernelFn f = lookup(P.dt, P.qdt, nout, P.add, mode, c, cl);
       if (!f) continue;
       const int sm = smem_bytes(mode, c, cl, t, nout, mode == arnq::LOAD_STAGED ? 1 : 0,
-                                stage_bytes);
+                                stage_bytes, rec);
       if (sm > di.smem_per_block_optin) continue;
       st = prepare_kernel(f, dev, sm);
       if (st != ARNQ_OK) return st;
@@ -348,23 +352,24 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   KernelFn fn = lookup(P.dt, P.qdt, nout, P.add, mode, pl->units, cl);
   if (!fn) return ARNQ_ERR_PLAN;
   const int upt = pl->units;
-  const int trec = arnq::tail_rec_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
 
-  // Resident CTAs, grid and (one CTA per row) rows per CTA for a ring depth
-  // `stages`.  One CTA per row keeps the records of its rows in shared memory
-  // and settles them after its last row; while those records do not fit, fewer
-  // CTAs per SM (a persistent grid, more rows each), and only when not even one
-  // CTA fits, fewer rows per CTA (a larger grid, run in waves).
+  // Resident clusters (CTAs when cl == 1) and the grid for a ring depth
+  // `stages`: every resident slot gets a cluster (more rows in flight beat
+  // equal row counts: on 8192 x 4096, 740 CTAs took 44.3 us a call, the 683
+  // that give every CTA 12 rows 46.2 us), no more clusters than rows.  A
+  // requested grid is kept.
   struct Eval {
-    int per_sm = 0, smem = 0, tail_rows = 0;
+    int per_sm = 0, smem = 0;
     int64_t nclusters = 0;
   };
   auto evaluate = [&](int stages, Eval *e) -> arnq_status {
     *e = Eval();
-    const int base = smem_bytes(mode, upt, cl, pl->threads, nout, stages, stage_bytes);
-    if (base > di.smem_per_block_optin) return ARNQ_OK;
-    arnq_status s2 = prepare_kernel(fn, dev, base);
+    const int sm = smem_bytes(mode, upt, cl, pl->threads, nout, stages, stage_bytes, rec);
+    if (sm > di.smem_per_block_optin) return ARNQ_OK;
+    arnq_status s2 = prepare_kernel(fn, dev, sm);
     if (s2 != ARNQ_OK) return s2;
+    int64_t slots = 0;
+    int per_sm = 0;
     if (cl > 1) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -374,7 +379,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       attr[0].val.clusterDim.z = 1;
       cfg.gridDim = dim3(cl * 1024, 1, 1);
       cfg.blockDim = dim3(pl->threads, 1, 1);
-      cfg.dynamicSmemBytes = base;
+      cfg.dynamicSmemBytes = sm;
       cfg.attrs = attr;
       cfg.numAttrs = 1;
       int nc = 0;
@@ -383,62 +388,26 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       int64_t want =
           pl->ctas_per_sm != 0 ? static_cast<int64_t>(pl->ctas_per_sm) * di.sms / cl : nc;
       if (want < 1) want = 1;
-      const int64_t fit_clusters = want < nc ? want : nc;
-      e->per_sm = static_cast<int>(ceil_div(fit_clusters * cl, di.sms));
-      e->nclusters = P.rows < fit_clusters ? P.rows : fit_clusters;
-      e->smem = base;
-      return ARNQ_OK;
-    }
-    int per_sm = 0;
-    s2 = occupancy(fn, pl->threads, base, &per_sm);
-    if (s2 != ARNQ_OK) return s2;
-    if (per_sm < 1) return ARNQ_OK;
-    if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
-    auto fit_for = [&](int64_t rows_cta, int *fit, int *sm) -> arnq_status {
-      *fit = 0;
-      *sm = 0;
-      // (records alone beyond a CTA's shared memory: no fit, and no int overflow below)
-      if (rows_cta * static_cast<int64_t>(trec) > di.smem_per_block_optin) return ARNQ_OK;
-      *sm = smem_bytes(mode, upt, 1, pl->threads, nout, stages, stage_bytes,
-                       static_cast<int>(rows_cta), trec);
-      if (*sm > di.smem_per_block_optin) return ARNQ_OK;
-      arnq_status s3 = prepare_kernel(fn, dev, *sm);
-      if (s3 != ARNQ_OK) return s3;
-      return occupancy(fn, pl->threads, *sm, fit);
-    };
-    for (int iter = 0; iter < 16; ++iter) {  // per_sm only decreases
-      const int64_t g = static_cast<int64_t>(per_sm) * di.sms;
-      const int64_t grid = P.rows < g ? P.rows : g;
-      const int64_t rows_cta = ceil_div(P.rows, grid);
-      int fit = 0, sm = 0;
-      s2 = fit_for(rows_cta, &fit, &sm);
+      slots = want < nc ? want : nc;
+      per_sm = static_cast<int>(ceil_div(slots * cl, di.sms));
+    } else {
+      s2 = occupancy(fn, pl->threads, sm, &per_sm);
       if (s2 != ARNQ_OK) return s2;
-      if (fit >= per_sm) {
-        e->per_sm = per_sm;
-        e->nclusters = grid;
-        e->tail_rows = static_cast<int>(ceil_div(P.rows, grid));
-        e->smem = sm;
-        return ARNQ_OK;
-      }
-      if (fit < 1) break;
-      per_sm = fit;
+      if (per_sm < 1) return ARNQ_OK;
+      if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
+      slots = static_cast<int64_t>(per_sm) * di.sms;
     }
-    // one resident CTA cannot hold all its rows' records: fewer rows per CTA
-    int64_t rows_cta = ceil_div(P.rows, static_cast<int64_t>(di.sms));
-    while (true) {
-      int fit = 0, sm = 0;
-      s2 = fit_for(rows_cta, &fit, &sm);
-      if (s2 != ARNQ_OK) return s2;
-      if (fit >= 1) {
-        e->per_sm = 1;
-        e->nclusters = ceil_div(P.rows, rows_cta);
-        e->tail_rows = static_cast<int>(ceil_div(P.rows, e->nclusters));
-        e->smem = sm;
-        return ARNQ_OK;
-      }
-      if (rows_cta == 1) return ARNQ_OK;
-      rows_cta = ceil_div(rows_cta, 2);
+    int64_t nclusters;
+    if (pl->grid != 0) {
+      if (pl->grid % cl != 0) return ARNQ_ERR_PLAN;
+      nclusters = pl->grid / cl;
+    } else {
+      nclusters = P.rows < slots ? P.rows : slots;
     }
+    e->per_sm = per_sm;
+    e->nclusters = nclusters;
+    e->smem = sm;
+    return ARNQ_OK;
   };
 
   Eval best;
@@ -471,9 +440,23 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   pl->ctas_per_sm = best.per_sm;
   const int64_t nclusters = best.nclusters;
   const int smem = best.smem;
-  L->tail_rows = cl == 1 ? best.tail_rows : 0;
-  L->trec_bytes = cl == 1 ? trec : 0;
   pl->grid = static_cast<int32_t>(nclusters * cl);
+  L->rec_bytes = rec;
+  // Row hand-out (staged kernel, one CTA per row, at least two rows per CTA):
+  // the first three quarters of each CTA's share dealt out in turn, the rest
+  // handed out by the workspace counter as CTAs become free (CTAs of one call
+  // run at different speeds: on 8192 x 4096, CTAs with the same eleven rows
+  // ended their loops anywhere from 32 to 40 us).
+  L->dyn_base = P.rows;
+  const bool can_dyn = mode == arnq::LOAD_STAGED && cl == 1 && P.rows >= 2 * nclusters &&
+                       P.rows < (int64_t(1) << 30);
+  if (pl->schedule == 2 && !can_dyn) return ARNQ_ERR_PLAN;
+  if (pl->schedule == 0) pl->schedule = can_dyn ? 2 : 1;
+  if (pl->schedule == 2) {
+    int64_t per = 3 * P.rows / (4 * nclusters);
+    if (per < 1) per = 1;
+    L->dyn_base = per * nclusters;
+  }
   L->fn = fn;
   L->smem = smem;
   L->seg = seg;
@@ -562,19 +545,24 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   }
   k.x_out = static_cast<uint16_t *>(P.x_out);
   k.status = static_cast<int32_t *>(workspace);
-  k.records = static_cast<unsigned char *>(workspace) + arnq::kRecordBase;
+  k.sched = static_cast<int32_t *>(workspace) + 4;
   k.tie_cap = arnq::tie_cap(static_cast<int>(P.n), (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0));
-  k.rec_bytes = arnq::record_bytes(k.tie_cap);
+  k.rec_bytes = L.rec_bytes;
+  k.dyn_base = L.dyn_base;
   k.rows = P.rows;
   k.n = static_cast<int32_t>(P.n);
   k.units = L.units;
   k.seg_units = L.seg;
   k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0);
   k.stages = plan.stages;
-  k.tail_rows = L.tail_rows;
-  k.trec_bytes = L.trec_bytes;
   k.eps = P.eps;
   k.inv_n = 1.0 / static_cast<double>(P.n);
+  k.wait_limit_ns = plan.wait_limit_us > 0
+                        ? static_cast<uint64_t>(plan.wait_limit_us) * 1000ull
+                        : static_cast<uint64_t>(arnq::kWaitLimitNs);
+  k.test_hold_tx = plan.kernel == ARNQ_KERNEL_STAGED && plan.test_hold_bytes > 0
+                       ? static_cast<uint32_t>(plan.test_hold_bytes)
+                       : 0u;
 
   // The row kernel is a programmatic dependent of whatever precedes it on the
   // stream: its CTAs may become resident while that work finishes, and wait
@@ -597,22 +585,6 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
     cfg.numAttrs = 2;
   }
   if (cudaLaunchKernelEx(&cfg, L.fn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
-  if (plan.cluster == 1) return ARNQ_OK;  // the row kernel settles its own rows
-
-  // the settle kernel: a half warp per row, a programmatic dependent of the row
-  // kernel (it may start early and waits for the row kernel's results)
-  arnq::SettleFn sfn = lookup_settle(P.dt, P.qdt, slot, P.add, plan.vector != 0);
-  if (!sfn) return ARNQ_ERR_PLAN;
-  cudaLaunchConfig_t sc = {};
-  cudaLaunchAttribute sattr[1];
-  sattr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  sattr[0].val.programmaticStreamSerializationAllowed = 1;
-  sc.gridDim = dim3(static_cast<unsigned>(ceil_div(P.rows, kSettleRowsPerBlock)), 1, 1);
-  sc.blockDim = dim3(16 * kSettleRowsPerBlock, 1, 1);
-  sc.stream = stream;
-  sc.attrs = sattr;
-  sc.numAttrs = 1;
-  if (cudaLaunchKernelEx(&sc, sfn, k) != cudaSuccess) return ARNQ_ERR_CUDA;
   return ARNQ_OK;
 }
 
@@ -631,21 +603,16 @@ Problem problem(const void *x1, const void *x2, const void *gamma, const void *b
 // ---------------------------------------------------------------- static scratch
 
 // The no-allocation entry point's scratch: one array per device, in the
-// library's own device memory.  Its address is looked up once per device.
+// library's own device memory (zero when the library's device code is loaded).
+// Host code cannot use the symbol as a device address: the address is looked
+// up on every call, with the current device, so that it is never stale (a
+// device reset between calls reloads the module at another address).
 static __device__ __align__(256) unsigned char g_static_scratch[ARNQ_STATIC_SCRATCH_BYTES];
-void *g_scratch_addr[kMaxDevices];
 
 arnq_status static_scratch(void **out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ARNQ_ERR_CUDA;
-  std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return ARNQ_ERR_CUDA;
-    if (cudaMemset(p, 0, ARNQ_STATIC_SCRATCH_BYTES) != cudaSuccess) return ARNQ_ERR_CUDA;
-    g_scratch_addr[dev] = p;
-  }
-  *out = g_scratch_addr[dev];
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return ARNQ_ERR_CUDA;
+  *out = p;
   return ARNQ_OK;
 }
 
@@ -656,6 +623,8 @@ arnq_status run_common(Problem P, int out_mask, void *workspace, size_t workspac
   arnq_plan pl;
   std::memset(&pl, 0, sizeof pl);
   if (plan) pl = *plan;
+  st = check_plan_fields(pl);
+  if (st != ARNQ_OK) return st;
   return launch(P, pl, workspace, static_cast<cudaStream_t>(stream));
 }
 
@@ -670,7 +639,9 @@ const char *arnq_status_string(arnq_status s) {
     case ARNQ_OK: return "ARNQ_OK";
     case ARNQ_ERR_NULL_PTR: return "ARNQ_ERR_NULL_PTR: a required input or a selected output is NULL";
     case ARNQ_ERR_EMPTY: return "ARNQ_ERR_EMPTY: empty tensors are not supported";
-    case ARNQ_ERR_SHAPE: return "ARNQ_ERR_SHAPE: unsupported shape (odd n for INT4, n too large, negative size)";
+    case ARNQ_ERR_SHAPE:
+      return "ARNQ_ERR_SHAPE: unsupported shape (n not a multiple of 2 for INT4 or 8 for "
+             "INT4_INT32, n too large, negative size)";
     case ARNQ_ERR_DTYPE: return "ARNQ_ERR_DTYPE: unknown dtype or qdtype";
     case ARNQ_ERR_MASK: return "ARNQ_ERR_MASK: outputMask / smooth-scale combination not allowed";
     case ARNQ_ERR_EPS: return "ARNQ_ERR_EPS: epsilon must be finite and >= 0";
@@ -679,6 +650,8 @@ const char *arnq_status_string(arnq_status s) {
     case ARNQ_ERR_CUDA: return "ARNQ_ERR_CUDA: a CUDA call failed";
     case ARNQ_ERR_PLAN: return "ARNQ_ERR_PLAN: the launch plan cannot run this problem";
     case ARNQ_ERR_DEVICE_TIMEOUT: return "ARNQ_ERR_DEVICE_TIMEOUT: a kernel gave up waiting for a copy";
+    case ARNQ_ERR_WORKSPACE_STATE:
+      return "ARNQ_ERR_WORKSPACE_STATE: the workspace was not zero-filled before its first call";
   }
   return "ARNQ: unknown status";
 }
@@ -696,7 +669,7 @@ arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdt
   int on1 = 0, on2 = 0;
   st = selected(out_mask, has_smooth1 != 0, has_smooth2 != 0, &on1, &on2);
   if (st != ARNQ_OK) return st;
-  *bytes = workspace_bytes_for(rows, n, on1 + on2);
+  *bytes = workspace_bytes_for();
   return ARNQ_OK;
 }
 
@@ -783,9 +756,8 @@ arnq_status arnq_run_static_scratch(const void *x1, const void *x2, const void *
   void *scratch = nullptr;
   st = static_scratch(&scratch);
   if (st != ARNQ_OK) return st;
-  // the status block must start at zero (the row records need no clearing:
-  // each is written before it is read)
-  if (cudaMemsetAsync(scratch, 0, arnq::kRecordBase, static_cast<cudaStream_t>(stream)) !=
+  // the status block must start at zero (the kernel writes it only on error)
+  if (cudaMemsetAsync(scratch, 0, arnq::kStatusBytes, static_cast<cudaStream_t>(stream)) !=
       cudaSuccess)
     return ARNQ_ERR_CUDA;
   return run_common(P, out_mask, scratch, ARNQ_STATIC_SCRATCH_BYTES, stream, nullptr);

@@ -14,48 +14,44 @@
 // thread-block cluster of CTAs sharing a row through distributed shared memory)
 // takes one row at a time; each thread keeps its elements of x and its folded
 // parameters G_k in registers (B_k of 16-byte units in shared memory, read
-// back by the thread that wrote it).  Persistent grid: cluster c handles rows
-// c, c + nclusters, ...  Two barriers per row: after the sum of squares and
-// after the row maximum.  The kernel is launched as a programmatic dependent
-// (it waits for the preceding work before touching memory, and lets the next
-// kernel start its set-up after its last row).
+// back by the thread that wrote it).  Persistent grid: a CTA takes rows c,
+// c + G, ... and then (staged kernel, one CTA per row) rows handed out one at
+// a time by a counter in the workspace.  Three barriers per row: after the
+// sum of squares, after the binary32 row maxima and after the exact row
+// maxima.  The kernel is launched as a programmatic dependent (it waits for
+// the preceding work before touching memory, and lets the next kernel start
+// its set-up after its last row).
 //
-// Arithmetic of the fast path, binary32 two lanes at a time with the sm_100
-// packed instructions (add/mul/fma.rn.f32x2):
+// The result is what an fp64 evaluation of the definition gives, with the
+// scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
+// code = RNE(input_k / scale_k).  Per row:
 //   x = RN16(x1 + x2)            add.rn.{bf16,f16}x2 -- the correctly rounded
-//                                sum, which equals rounding the binary32 sum
+//                                sum, which equals rounding the binary32 sum;
+//                                written as xOut and kept in registers
 //   ss = sum x^2                 fp64 (each x^2 is exact)
 //   1/Rms                        binary32 from ss (within a few ulp)
-//   input_k = x*rinv*G_k + B_k   G_k = gamma*smooth_k, B_k = beta*smooth_k, exact
-//                                products of two 16-bit values
-//   s~_k = max|input_k| / Q      approximate scale
-//   code = RNE(input_k / s~_k)   rounded half-to-even by adding 1.5*2^23
-// The result must be what an fp64 evaluation of the definition gives, with the
-// scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
-// code = RNE(input_k / scale_k).  The fast path writes its codes and, for
-// each row, a record: the row's fp64 sum of squares and the few units (8 or
-// 2 elements) that the binary32 arithmetic cannot settle:
-//  * candidate units: holding an element within the binary32 error bound of
-//    the row maximum (the true maximum is among them);
-//  * near-tie units: holding a code whose binary32 quotient t lies within tau
-//    of a half-way point, where |t - t_exact| <= tau covers the binary32
-//    error and the distance between s~ and the exact scale.
-// The records are settled from x read back from xOut or the inputs and the
-// parameters from memory: the exact scale RN32(max fp64 |input| over the
-// candidates / Q), then the near-tie units' codes recomputed in fp64.  With
-// one CTA per row, each CTA keeps its rows' records in shared memory and
-// settles them itself after its last row (tail_settle, a group of 8 to 32
-// lanes per row); a row shared by a cluster has its record in the workspace,
-// settled by a second, small kernel (settle_kernel, 16 lanes per row, launched
-// as a programmatic dependent).  A record holds only unit indices: storing
-// more from the fast path costs it register spills.  These
-// fp64 evaluations use 1/Rms and 1/scale from Newton steps (a few fp64 ulp)
-// instead of divisions: the decisions they settle sit at distances of about
-// the binary32 rounding of the scale (~1e-7 relative) from a half-way point,
-// many orders above fp64 rounding.  A row whose record overflows (many equal
-// maxima, many exact ties) or whose sum of squares or scale leaves the normal
-// binary32 range is recomputed whole by its lanes, in fp64 with IEEE
-// divisions in the definition's order.
+//   input_k = x*rinv*G_k + B_k   binary32, packed f32x2 (add/mul/fma.rn.f32x2);
+//                                G_k = gamma*smooth_k, B_k = beta*smooth_k,
+//                                exact products of two 16-bit values
+//   max_k                        binary32 row maximum, then exact: the threads
+//                                holding a candidate unit (an element within
+//                                the binary32 error bound of that maximum; the
+//                                true maximum is among them) evaluate its
+//                                elements in fp64, and the fp64 maxima meet
+//                                at the third barrier
+//   scale_k = RN32(max_k / Q)    exact
+//   code = RNE(input_k * RN32(1/scale_k))  binary32, rounded half to even by
+//                                adding 1.5*2^23; a code whose quotient lies
+//                                within tau of a half-way point (tau bounds the
+//                                binary32 error) is recomputed by its thread in
+//                                fp64 as input_k / scale_k (about 1e-3 of the
+//                                codes)
+// The fp64 inputs use 1/Rms from Newton steps (a few fp64 ulp): the decisions
+// they settle sit many orders of magnitude above fp64 rounding.  A row whose
+// ss/n + eps leaves the normal binary32 range is computed whole in fp64, in
+// the definition's order with IEEE divisions; one whose 1/scale is not a
+// normal binary32 number gets all its codes in fp64.  Every thread handles
+// its own elements: no global memory is read twice.
 // Nothing here is a contraction: no tensor cores.
 #pragma once
 
@@ -75,56 +71,64 @@ enum : int {
 enum : int { LOAD_VEC = 0, LOAD_SCALAR = 1, LOAD_STAGED = 2 };
 
 // status codes the kernels record in the workspace status block
-enum : int { DEV_TIMEOUT = 11 };
+enum : int {
+  DEV_TIMEOUT = 11,   // a bounded wait ran out
+  DEV_SCHED = 12      // the row hand-out counters were not zero when the call started
+};
 
-// A bounded wait gives up after this long (nanoseconds of %globaltimer).
+// A bounded wait gives up after this long (nanoseconds of %globaltimer)
+// unless the launch asks for another limit.
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 
 // row flags exchanged at the first barrier of the next row
 enum : int { RF_REDO = 1, RF_ABORT = 2 };
 
-// Row records, in the workspace after the status block (kRecordBase bytes):
-// one per row, record_bytes(tie_cap) each:
-//   header (64 B): double ss; int ncand, ntie, flags (RF_REDO); pad
-//   units [kCandCap + tie_cap] ints: unit | output << 31; candidates first,
-//     then near ties.
-// A near tie needs |t - RNE(t)| > 0.5 - tau, about 2 tau ~ 1e-3 of the codes
-// or fewer; tie_cap leaves several times that for a row of n columns and
-// nout outputs, so rows overflow (and go to the slow path) only by design:
-// many exact ties.
-constexpr int kRecordBase = 256;
-constexpr int kCandCap = 4;     // candidate units per row
-__host__ __device__ inline int tie_cap(int n, int nout) { return 12 + (n * nout + 255) / 256; }
-// (a multiple of 16 bytes: the header's double must stay 8-byte aligned)
-__host__ __device__ inline int record_bytes(int tcap) {
-  return (64 + (kCandCap + tcap) * 4 + 15) & ~15;
-}
+// The workspace holds only the status block (kStatusBytes: the status at
+// bytes 0-15, the row hand-out counters at 16-27).
+constexpr int kStatusBytes = 256;
 
-// In-kernel settling (one CTA per row): the records of the CTA's own rows
-// stay in its shared memory, one per row it processes, and the CTA settles
-// them itself after its last row.  Record: a 32-byte header (double ss;
-// int cnt[2] = candidate and near-tie units recorded; int flags), then
-// kCandCap + tie_cap unit entries (unit | output << 31), as in the workspace
-// records of clusters.
-struct TailHead {
+// Row records.  The binary32 fast path leaves a few units (8 or 2 elements)
+// per row that it cannot settle: candidate units, holding an element within
+// the binary32 error bound of the row maximum (the true maximum is among
+// them), and near-tie units, holding a code whose binary32 quotient lies
+// within tau of a half-way point.  The thread that holds such a unit appends
+// it to the row's record together with the unit's G_k and B_k; one row later
+// one warp (the settling warp) copies the recorded units' x from xOut (or
+// x1, x2) into the record with cp.async, and one row later again settles the
+// row from the record alone: the exact scale RN32(max fp64 |input| over the
+// candidates / Q), then the near-tie codes in fp64 -- with no load on its
+// critical path.  Three records live in the shared memory of the row's CTA
+// (of the cluster's first CTA): the row being processed, the one whose x is
+// on its way, and the one being settled.
+//   header (32 B): double ss; int cnt[2] (candidate, near-tie entries); int flags
+//   ue  [cap] ints: unit | output << 31, candidates first (cap = kCandCap + tie_cap)
+//   ent [cap][24] 32-bit words: x (16 bytes: eight 16-bit values, or x1 then
+//       x2 when xOut is not written; 32 bytes reserved), G_k (8 floats), B_k
+//       (8 floats); pair units (2 elements) use the first words of each part
+// A row whose near-tie list overflows (many exact ties) or whose arithmetic
+// leaves the normal binary32 range is recomputed whole, in fp64.
+constexpr int kCandCap = 4;
+__host__ __device__ inline int tie_cap(int n, int nout) { return 12 + (n * nout + 255) / 256; }
+struct RecHead {
   double ss;
   int cnt[2];
   int flags;
   int pad[3];
 };
-__host__ __device__ inline int tail_rec_bytes(int tcap) {
-  return (static_cast<int>(sizeof(TailHead)) + (kCandCap + tcap) * 4 + 15) & ~15;
+__host__ __device__ inline int rec_ue_bytes(int tcap) { return ((kCandCap + tcap) * 4 + 15) & ~15; }
+__host__ __device__ inline int rec_slot_bytes(int tcap) {
+  return static_cast<int>(sizeof(RecHead)) + rec_ue_bytes(tcap) + (kCandCap + tcap) * 96;
 }
 
 // Shared-memory layout, sized by the launch (the host computes the same):
 //   ss    [nslots] doubles: per-warp partial sums (also the exact path's reductions)
 //   wmax  [NOUT][nslots] floats: per-warp binary32 row maxima of |input_k|
 //   maxb  [NOUT][nslots] floats: set-up reduction of the bound on |B_k|
-//   lcnt  [2][2] ints: candidate and near-tie units recorded, by row parity
-//         (in the first CTA of a cluster)
 //   flags [2] ints: RF_* of a row, by row parity
 //   bars  [stages] mbarriers
-//   trec  [tail_rows] in-kernel row records of trec_bytes each (one CTA per row)
+//   recs  [3] row records of rec_bytes each (used in the cluster's first CTA)
+//   srow  [stages] int64: staged kernel, the row each stage holds (-1: none)
+//   take  16 bytes: the copy-issuing thread's row hand-out state (TakeState)
 //   bsm   16-byte units: B_k = beta * smooth_k of every thread's units,
 //         [NOUT][UPT][2][threads] float4 (bsm_bytes_for)
 //   ring  [stages] rows of staged input
@@ -136,22 +140,28 @@ __host__ __device__ inline int bsm_bytes_for(bool vector_units, int nout, int up
   return vector_units ? nout * upt * threads * 32 : 0;
 }
 struct Layout {
-  int ss, wmax, maxb, amax, flags, bars, trec, bsm, ring;
+  int ss, wmax, maxb, flags, bars, srow, take, recs, bsm, ring;
 };
-__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int tail_rows,
-                                              int trec_bytes, int bsm_bytes) {
+struct TakeState {
+  int64_t nxt;   // next row dealt out in turn
+  int ndyn;      // rows taken from the counter
+  int dry;       // the counter ran out: take nothing more
+};
+__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int rec_bytes,
+                                              int bsm_bytes) {
   Layout L;
   int off = 0;
   L.ss = off;    off += nslots * 8;
   L.wmax = off;  off += nout * nslots * 4;
   L.maxb = off;  off += nout * nslots * 4;
   off = (off + 7) & ~7;
-  L.amax = off;  off += 4 * 4;
   L.flags = off; off += 2 * 4;
   off = (off + 7) & ~7;
   L.bars = off;  off += stages * 8;
+  L.srow = off;  off += stages * 8;
+  L.take = off;  off += 16;
   off = (off + 15) & ~15;
-  L.trec = off;  off += tail_rows * trec_bytes;
+  L.recs = off;  off += 3 * rec_bytes;
   off = (off + 15) & ~15;
   L.bsm = off;   off += bsm_bytes;
   L.ring = (off + 127) & ~127;
@@ -165,19 +175,23 @@ struct KParams {
   float *scale[2];            // per output slot
   uint16_t *x_out;
   int32_t *status;            // workspace status block
-  unsigned char *records;     // workspace row records (rec_bytes per row)
-  int32_t tie_cap;            // near-tie units a record holds
-  int32_t rec_bytes;          // bytes per record
+  int32_t *sched;             // workspace: tickets handed out, CTAs done, rows handed out
+                              // (all zero between calls)
+  int64_t dyn_base;           // staged, one CTA per row: rows from here on are handed
+                              // out by the counter (rows = none)
   int64_t rows;
   int32_t n;                  // row length in elements
   int32_t units;              // units per row: ceil(n / U)
   int32_t seg_units;          // units per CTA of a cluster
   int32_t flags;
   int32_t stages;             // staged kernel: ring depth
-  int32_t tail_rows;          // one CTA per row: rows per CTA at most (shared-memory records)
-  int32_t trec_bytes;         // bytes per shared-memory record (tail_rec_bytes)
+  int32_t tie_cap;            // near-tie entries a record holds
+  int32_t rec_bytes;          // bytes of one record (rec_slot_bytes)
   float eps;
   double inv_n;               // 1 / n
+  uint64_t wait_limit_ns;     // bounded waits give up after this long
+  uint32_t test_hold_tx;      // testing only: extra bytes the first staged copy's
+                              // barrier expects (never delivered); 0 in normal use
 };
 
 struct Bf16 {};
@@ -271,13 +285,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the given phase parity of an mbarrier, at most kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Waits for the given phase parity of an mbarrier, at most limit_ns.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_timer_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (global_timer_ns() - t0 > kWaitLimitNs) return false;
+    if (global_timer_ns() - t0 > limit_ns) return false;
   }
 }
 
@@ -290,6 +305,20 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
       "[%0], [%1], %2, [%3], %4;" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
+}
+
+// 16-byte copy global -> shared (cp.async, through L2 only); completes for
+// the issuing thread at cp.async.wait_group
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 // L2 policy of the staged input copies: normal eviction (measured faster than
@@ -319,16 +348,6 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 __device__ __forceinline__ double warp_max_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-  return v;
-}
-// sum / max over an aligned group of `width` lanes (a power of two up to 32;
-// mask: the group's lanes)
-__device__ __forceinline__ double group_sum_d(double v, unsigned mask, int width) {
-  for (int o = width >> 1; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(mask, v, o, width));
-  return v;
-}
-__device__ __forceinline__ double group_max_d(double v, unsigned mask, int width) {
-  for (int o = width >> 1; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(mask, v, o, width));
   return v;
 }
 // max over lanes of non-negative floats (their bit patterns order as integers)
@@ -369,14 +388,6 @@ __device__ __forceinline__ double rsqrt64(double v) {
   }
   return r;
 }
-// 1/s in fp64 to a few ulp, for a normal binary32 s: r' = r + r(1 - s r).
-__device__ __forceinline__ double rcp64(float s) {
-  const double d = static_cast<double>(s);
-  double r = static_cast<double>(__frcp_rn(s));
-#pragma unroll
-  for (int i = 0; i < 2; ++i) r = __fma_rn(r, __fma_rn(-d, r, 1.0), r);
-  return r;
-}
 // round half to even, clamped to [-qmax, qmax]
 __device__ __forceinline__ int code_of_t(double t, int qmax) {
   return min(max(__double2int_rn(t), -qmax), qmax);
@@ -401,6 +412,199 @@ __device__ __forceinline__ double input_of(const KParams &p, int o, int c, float
 __device__ __forceinline__ int code_of(double in, float scale, int qmax) {
   if (scale == 0.f) return 0;
   return code_of_t(__ddiv_rn(in, static_cast<double>(scale)), qmax);
+}
+
+// ---------------------------------------------------------------- exact codes
+
+// RNE(in / sc) clamped to [-qmax, qmax], for an fp64 input `in`, a positive
+// normal binary32 scale sc and an approximation t of in / sc that is off by
+// less than 1/2: the only rounding boundary within reach is the half-integer
+// h = floor(t) + 1/2, and the sign of in - h*sc decides on which side of it
+// in / sc lies.  h*sc is exact in fp64 (a half-integer of at most 9 bits
+// times a 24-bit significand), so the fused multiply-add computes that sign
+// exactly: the code is correctly rounded, exact ties to even included, with
+// no division.
+__device__ __forceinline__ int code_exact(double in, float sc, float t, int qmax) {
+  const float h = floorf(t) + 0.5f;
+  const double e = __fma_rn(-static_cast<double>(h), static_cast<double>(sc), in);
+  const int lo = static_cast<int>(h - 0.5f);  // floor(t)
+  int q;
+  if (e > 0.0) q = lo + 1;
+  else if (e < 0.0) q = lo;
+  else q = (lo & 1) ? lo + 1 : lo;  // an exact tie: to even
+  return min(max(q, -qmax), qmax);
+}
+
+// ---------------------------------------------------------------- whole rows in fp64
+
+// x of column c of a row, read back from memory: xOut when written, else the
+// inputs (then unchanged: an in-place update always writes xOut).
+template <class T, bool ADD>
+__device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) {
+  using C = Cvt<T>;
+  const int64_t j = row * p.n + c;
+  if (!ADD) return C::f1(p.x1[j]);
+  if (p.flags & F_XOUT) return C::f1(p.x_out[j]);
+  return C::f2(C::add2(p.x1[j], p.x2[j])).x;
+}
+
+// Whole row in fp64, in the definition's order with IEEE divisions, by the 32
+// lanes of a warp, x read back from memory: the slow path for rows the fast
+// path cannot settle (a near-tie list that overflowed, or ss/n + eps or the
+// scale outside the normal binary32 range).  Called, not inlined: rare, and
+// its division sequences would take registers from the row loop.
+template <class T, bool INT4, int NOUT, bool ADD>
+__device__ __noinline__ void exact_row_warp(const KParams &p, int64_t row, int lane) {
+  constexpr int QI = INT4 ? 7 : 127;
+  const int n = p.n;
+  const int64_t base = row * n;
+  double ss = 0.0;
+  for (int c = lane; c < n; c += 32) {
+    const double a = x_reload<T, ADD>(p, row, c);
+    ss = __fma_rn(a, a, ss);
+  }
+  const double rms = rms_of(warp_sum_d(ss), n, p.eps);
+  for (int o = 0; o < NOUT; ++o) {
+    double m = 0.0;
+    for (int c = lane; c < n; c += 32)
+      m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
+    const float sc = __double2float_rn(__ddiv_rn(warp_max_d(m), static_cast<double>(QI)));
+    if (lane == 0) p.scale[o][row] = sc;
+    for (int c = 2 * lane; c < n; c += 64) {  // element pairs: an INT4 byte has one writer
+      const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
+      const int q1 =
+          c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
+                    : 0;
+      if (INT4) {
+        p.y[o][row * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+      } else {
+        p.y[o][base + c] = static_cast<uint8_t>(q0);
+        if (c + 1 < n) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- settling a record
+
+__device__ __forceinline__ int *rec_ue(RecHead *h) { return reinterpret_cast<int *>(h + 1); }
+__device__ __forceinline__ uint32_t *rec_ent(RecHead *h, int tcap, int ent) {
+  return reinterpret_cast<uint32_t *>(reinterpret_cast<unsigned char *>(h + 1) +
+                                      rec_ue_bytes(tcap)) + ent * 24;
+}
+
+// Copies the recorded units' x of row r into the record h (16-byte units:
+// cp.async, one commit group per call, waited for by the same warp at the
+// row's settle).  Rows the slow path takes need nothing.
+template <bool ADD, int U>
+__device__ __forceinline__ void prefetch_record(const KParams &p, RecHead *h, int64_t r, int lane) {
+  if (U == 8) {
+    const int nc = min(h->cnt[0], kCandCap), nt = min(h->cnt[1], p.tie_cap);
+    const int *ue = rec_ue(h);
+    for (int q = lane; q < kCandCap + nt; q += 32) {
+      if (q >= nc && q < kCandCap) continue;
+      const int u = static_cast<int>(static_cast<uint32_t>(ue[q]) & 0x7FFFFFFFu);
+      const int64_t j = r * p.n + static_cast<int64_t>(u) * 8;
+      uint32_t *dst = rec_ent(h, p.tie_cap, q);
+      if (!ADD) {
+        cp_async16(dst, p.x1 + j);
+      } else if (p.flags & F_XOUT) {
+        cp_async16(dst, p.x_out + j);
+      } else {
+        cp_async16(dst, p.x1 + j);
+        cp_async16(dst + 4, p.x2 + j);
+      }
+    }
+  }
+  cp_async_commit();
+}
+
+// Settles row r from its record h (in this CTA's shared memory, or the
+// cluster's first CTA's) with one warp, then clears the record's counters.
+// The record holds every value needed (x copied in by prefetch_record, whose
+// group the caller has waited for; G_k and B_k from the recording threads):
+// the candidates' fp64 maximum gives the exact scale RN32(max / Q); each
+// near-tie unit's codes are then decided exactly from their fp64 inputs
+// (code_exact).  Pair units (U == 2: misaligned or ragged rows) read x from
+// memory here.
+template <class T, bool INT4, int NOUT, bool ADD, int U>
+__device__ __forceinline__ void settle_record(const KParams &p, RecHead *h, int64_t r, int lane) {
+  using C = Cvt<T>;
+  constexpr int QI = INT4 ? 7 : 127;
+  constexpr int PAIRS = U / 2;
+  const int n = p.n;
+  const int nc = h->cnt[0], nt = h->cnt[1];
+  if ((h->flags & RF_REDO) || nc > kCandCap || nt > p.tie_cap) {
+    exact_row_warp<T, INT4, NOUT, ADD>(p, r, lane);
+  } else {
+    const int *ue = rec_ue(h);
+    const double ri = rsqrt64(__fma_rn(h->ss, p.inv_n, static_cast<double>(p.eps)));
+    // fp64 input of element e of entry ent (column c)
+    auto in64 = [&](int ent, int e, int c) -> double {
+      const uint32_t *v = rec_ent(h, p.tie_cap, ent);
+      float x;
+      if (U == 8) {
+        const int wd = e >> 1;
+        const float2 a = C::f2(ADD && !(p.flags & F_XOUT) ? C::add2(v[wd], v[4 + wd]) : v[wd]);
+        x = (e & 1) ? a.y : a.x;
+      } else {
+        x = x_reload<T, ADD>(p, r, c);
+      }
+      return __fma_rn(__dmul_rn(static_cast<double>(x), ri),
+                      static_cast<double>(__uint_as_float(v[8 + e])),
+                      static_cast<double>(__uint_as_float(v[16 + e])));
+    };
+    // exact scales: fp64 maximum over the candidate elements (one a lane)
+    double m0 = 0.0, m1 = 0.0;
+    if (lane < nc * U) {
+      const int ent = lane / U, e = lane % U;
+      const uint32_t hd = static_cast<uint32_t>(ue[ent]);
+      const int c = U * static_cast<int>(hd & 0x7FFFFFFFu) + e;
+      if (c < n) {
+        const double v = fabs(in64(ent, e, c));
+        if ((hd >> 31) == 0) m0 = v; else m1 = v;
+      }
+    }
+    float sc[2], r32[2];
+    sc[0] = __double2float_rn(__dmul_rn(warp_max_d(m0), 1.0 / static_cast<double>(QI)));
+    sc[1] = NOUT == 2 ? __double2float_rn(__dmul_rn(warp_max_d(m1), 1.0 / static_cast<double>(QI)))
+                      : 0.f;
+#pragma unroll
+    for (int o = 0; o < 2; ++o) r32[o] = sc[o] >= 1.1754943508222875e-38f ? __frcp_rn(sc[o]) : 0.f;
+    if (lane == 0) {
+      p.scale[0][r] = sc[0];
+      if (NOUT == 2) p.scale[1][r] = sc[1];
+    }
+    // near-tie codes, one element pair (one INT4 byte) a lane
+    for (int q = lane; q < nt * PAIRS; q += 32) {
+      const int ent = kCandCap + q / PAIRS;
+      const uint32_t hd = static_cast<uint32_t>(ue[ent]);
+      const int o = static_cast<int>(hd >> 31);
+      const int e = 2 * (q % PAIRS);
+      const int c = U * static_cast<int>(hd & 0x7FFFFFFFu) + e;
+      const float so = o ? sc[1] : sc[0], ro = o ? r32[1] : r32[0];
+      int q2[2] = {0, 0};
+#pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        if (so != 0.f && c + h2 < n) {
+          const double v = in64(ent, e + h2, c + h2);
+          q2[h2] = ro != 0.f ? code_exact(v, so, __double2float_rn(v) * ro, QI) : code_of(v, so, QI);
+        }
+      }
+      if (INT4) {
+        p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q2[0] & 0xF) | ((q2[1] & 0xF) << 4));
+      } else {
+        p.y[o][r * n + c] = static_cast<uint8_t>(q2[0]);
+        if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q2[1]);
+      }
+    }
+  }
+  __syncwarp();
+  if (lane == 0) {
+    h->cnt[0] = 0;
+    h->cnt[1] = 0;
+    h->flags = 0;
+  }
 }
 
 // ---------------------------------------------------------------- exchange
@@ -438,319 +642,12 @@ struct Exchange {
       atomicOr(flags + par, bits);
     }
   }
-  // the row's record counters live in the first CTA of the cluster
-  __device__ __forceinline__ int *lcnt_slot(int *lcnt, int i) {
-    return CL ? cluster.map_shared_rank(lcnt, 0) + i : lcnt + i;
+  // the row records live in the first CTA of the cluster
+  __device__ __forceinline__ unsigned char *first_cta(unsigned char *q) {
+    if constexpr (CL) return cluster.map_shared_rank(q, 0);
+    return q;
   }
 };
-
-// x of column c of a row, read back from memory: xOut when written, else the
-// inputs (then unchanged: an in-place update always writes xOut).
-template <class T, bool ADD>
-__device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) {
-  using C = Cvt<T>;
-  const int64_t j = row * p.n + c;
-  if (!ADD) return C::f1(p.x1[j]);
-  if (p.flags & F_XOUT) return C::f1(p.x_out[j]);
-  return C::f2(C::add2(p.x1[j], p.x2[j])).x;
-}
-
-// Whole row in fp64, in the definition's order, by an aligned group of
-// `width` lanes (lane = 0 .. width-1, mask: the group's lanes), x read back
-// from memory: the slow path for rows the fast path cannot settle.
-template <class T, bool INT4, int NOUT, bool ADD>
-__device__ __forceinline__ void exact_row_lanes(const KParams &p, int64_t row, int lane, int width,
-                                                unsigned mask) {
-  constexpr int QI = INT4 ? 7 : 127;
-  const int n = p.n;
-  const int64_t base = row * n;
-  double ss = 0.0;
-  for (int c = lane; c < n; c += width) {
-    const double a = x_reload<T, ADD>(p, row, c);
-    ss = __fma_rn(a, a, ss);
-  }
-  const double rms = rms_of(group_sum_d(ss, mask, width), n, p.eps);
-#pragma unroll
-  for (int o = 0; o < NOUT; ++o) {
-    double m = 0.0;
-    for (int c = lane; c < n; c += width)
-      m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
-    const float sc =
-        __double2float_rn(__ddiv_rn(group_max_d(m, mask, width), static_cast<double>(QI)));
-    if (lane == 0) p.scale[o][row] = sc;
-    for (int c = 2 * lane; c < n; c += 2 * width) {  // element pairs: an INT4 byte has one writer
-      const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
-      const int q1 =
-          c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
-                    : 0;
-      if (INT4) {
-        p.y[o][row * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
-      } else {
-        p.y[o][base + c] = static_cast<uint8_t>(q0);
-        if (c + 1 < n) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- settle kernel
-
-// Settles the row records the row kernel wrote: one half warp (16 lanes) per
-// row, so a bench-sized call's rows are all resident at once.  Launched after
-// the row kernel on the same stream (as a programmatic dependent: it waits for
-// the row kernel's completion and memory before reading anything).
-// U = elements per unit of the row kernel that wrote the records.
-template <class T, bool INT4, int NOUT, bool ADD, int U>
-__global__ void __launch_bounds__(256) settle_kernel(const __grid_constant__ KParams p) {
-  using C = Cvt<T>;
-  constexpr int QI = INT4 ? 7 : 127;
-  constexpr int PAIRS = U / 2;  // element pairs per unit
-  asm volatile("griddepcontrol.wait;" ::: "memory");
-  const int lane = threadIdx.x & 15;
-  const unsigned mask = (threadIdx.x & 16) ? 0xFFFF0000u : 0x0000FFFFu;
-  const int64_t r = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 4) + (threadIdx.x >> 4);
-  if (r >= p.rows) return;  // whole half warps leave together
-  const int n = p.n;
-  const int tcap = p.tie_cap;
-  const int *h = reinterpret_cast<const int *>(p.records + r * p.rec_bytes);
-  const int *units = h + 16;
-  // first round of loads, all independent: the header, this lane's two
-  // candidate entries and its first two near-tie entries (read ahead of the
-  // counts; every index stays inside the record)
-  const double ss = *reinterpret_cast<const double *>(h);
-  const int nc = h[2], nt = h[3], fl = h[4];
-  const uint32_t ce0 = static_cast<uint32_t>(units[min(lane / U, kCandCap - 1)]);
-  const uint32_t ce1 = static_cast<uint32_t>(units[min((lane + 16) / U, kCandCap - 1)]);
-  const uint32_t te0 = static_cast<uint32_t>(units[kCandCap + min(lane / PAIRS, tcap - 1)]);
-  const uint32_t te1 = static_cast<uint32_t>(units[kCandCap + min((lane + 16) / PAIRS, tcap - 1)]);
-  if ((fl & RF_REDO) || nc > kCandCap || nt > tcap) {
-    exact_row_lanes<T, INT4, NOUT, ADD>(p, r, lane, 16, mask);
-    return;
-  }
-  // x, G = gamma * smooth and B = beta * smooth (exact in binary32) of column c
-  struct Elem { float x, g, b; };
-  auto load = [&](int o, int c) -> Elem {
-    Elem e;
-    e.x = x_reload<T, ADD>(p, r, c);
-    const float sm = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
-    e.g = C::f1(__ldg(p.gamma + c)) * sm;
-    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) * sm : 0.f;
-    return e;
-  };
-  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
-  auto input64 = [&](const Elem &e) -> double {
-    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), static_cast<double>(e.g),
-                    static_cast<double>(e.b));
-  };
-  auto unit_of = [](uint32_t hd) { return static_cast<int>(hd & 0x7FFFFFFFu); };
-  auto out_of = [](uint32_t hd) { return static_cast<int>(hd >> 31); };
-  // second round: every element this lane needs (two candidate elements, two
-  // element pairs of near-tie units), loaded before any arithmetic
-  const int cc0 = U * unit_of(ce0) + lane % U, cc1 = U * unit_of(ce1) + (lane + 16) % U;
-  const bool has_c0 = lane < nc * U && cc0 < n, has_c1 = lane + 16 < nc * U && cc1 < n;
-  const Elem zero = {0.f, 0.f, 0.f};
-  Elem ec0 = zero, ec1 = zero;
-  if (has_c0) ec0 = load(out_of(ce0), cc0);
-  if (has_c1) ec1 = load(out_of(ce1), cc1);
-  const int ct0 = U * unit_of(te0) + 2 * (lane % PAIRS);
-  const int ct1 = U * unit_of(te1) + 2 * ((lane + 16) % PAIRS);
-  const bool has_t0 = lane < nt * PAIRS, has_t1 = lane + 16 < nt * PAIRS;
-  Elem t00 = zero, t01 = zero, t10 = zero, t11 = zero;
-  if (has_t0) {
-    t00 = load(out_of(te0), ct0);
-    if (ct0 + 1 < n) t01 = load(out_of(te0), ct0 + 1);
-  }
-  if (has_t1) {
-    t10 = load(out_of(te1), ct1);
-    if (ct1 + 1 < n) t11 = load(out_of(te1), ct1 + 1);
-  }
-  // exact scales: fp64 maximum over the candidate elements
-  double m[2] = {0.0, 0.0};
-  if (has_c0) {
-    const double v = fabs(input64(ec0));
-    if (out_of(ce0) == 0) m[0] = v; else m[1] = v;
-  }
-  if (has_c1) {
-    const double v = fabs(input64(ec1));
-    if (out_of(ce1) == 0) m[0] = fmax(m[0], v); else m[1] = fmax(m[1], v);
-  }
-  const double inv_q = 1.0 / static_cast<double>(QI);
-  float sc[2] = {0.f, 0.f};
-#pragma unroll
-  for (int o = 0; o < NOUT; ++o) {
-    sc[o] = __double2float_rn(__dmul_rn(group_max_d(m[o], mask, 16), inv_q));
-    if (lane == 0) p.scale[o][r] = sc[o];
-  }
-  // near-tie codes in fp64, one element pair (one INT4 byte) at a time
-  auto put = [&](uint32_t hd, int c, const Elem &e0, const Elem &e1) {
-    const int o = out_of(hd);
-    const float so = o == 0 ? sc[0] : sc[1];
-    const double rs = so == 0.f ? 0.0 : rcp64(so);
-    const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(e0), rs), QI);
-    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(e1), rs), QI);
-    if (INT4) {
-      p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
-    } else {
-      p.y[o][r * n + c] = static_cast<uint8_t>(q0);
-      if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
-    }
-  };
-  if (has_t0) put(te0, ct0, t00, t01);
-  if (has_t1) put(te1, ct1, t10, t11);
-  // more near-tie pairs than two per lane: one pair at a time
-  for (int e = lane + 32; e < nt * PAIRS; e += 16) {
-    const uint32_t hd = static_cast<uint32_t>(units[kCandCap + e / PAIRS]);
-    const int c = U * unit_of(hd) + 2 * (e % PAIRS);
-    const Elem e0 = load(out_of(hd), c);
-    const Elem e1 = c + 1 < n ? load(out_of(hd), c + 1) : zero;
-    put(hd, c, e0, e1);
-  }
-}
-
-// ---------------------------------------------------------------- in-kernel settling
-
-// Settles one row from its record with an aligned group of g lanes (lane l of
-// g >= 8, gmask: the group's lanes): the exact scales from the candidate
-// units, then the near-tie units' codes, in fp64 from x read back from memory
-// and the parameters (the same arithmetic as settle_kernel).  The loads of the
-// common case (every candidate element, and each lane's first two element
-// pairs of near-tie units) are issued before any arithmetic.
-template <class T, bool INT4, int NOUT, bool ADD, int U>
-__device__ __forceinline__ void settle_row_group(const KParams &p, int64_t r, double ss, int nc,
-                                                 int nt, const int *ent, int l, int g,
-                                                 unsigned gmask) {
-  using C = Cvt<T>;
-  constexpr int QI = INT4 ? 7 : 127;
-  constexpr int PAIRS = U / 2;           // element pairs per unit
-  constexpr int CE = kCandCap * U / 8;   // candidate elements per lane, at most (g >= 8)
-  const int n = p.n;
-  struct Elem { float x, g, b; };
-  const Elem zero = {0.f, 0.f, 0.f};
-  auto load = [&](int o, int c) -> Elem {
-    Elem e;
-    e.x = x_reload<T, ADD>(p, r, c);
-    const float sm = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
-    e.g = C::f1(__ldg(p.gamma + c)) * sm;  // exact: two 16-bit significands
-    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) * sm : 0.f;
-    return e;
-  };
-  auto unit_of = [](uint32_t hd) { return static_cast<int>(hd & 0x7FFFFFFFu); };
-  auto out_of = [](uint32_t hd) { return static_cast<int>(hd >> 31); };
-
-  // candidate elements e = l, l + g, ... of the nc * U
-  Elem ce[CE];
-  int co[CE];
-  bool cv[CE];
-#pragma unroll
-  for (int k = 0; k < CE; ++k) {
-    const int e = l + k * g;
-    ce[k] = zero;
-    co[k] = 0;
-    cv[k] = false;
-    if (e < nc * U) {
-      const uint32_t hd = static_cast<uint32_t>(ent[e / U]);
-      const int c = U * unit_of(hd) + e % U;
-      if (c < n) {
-        co[k] = out_of(hd);
-        cv[k] = true;
-        ce[k] = load(co[k], c);
-      }
-    }
-  }
-  // near-tie element pairs q = l, l + g, ...: the first two now
-  Elem ta[2], tb[2];
-  uint32_t th[2];
-  int tc[2];
-  bool tv[2];
-#pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int q = l + k * g;
-    ta[k] = tb[k] = zero;
-    th[k] = 0u;
-    tc[k] = 0;
-    tv[k] = q < nt * PAIRS;
-    if (tv[k]) {
-      th[k] = static_cast<uint32_t>(ent[kCandCap + q / PAIRS]);
-      tc[k] = U * unit_of(th[k]) + 2 * (q % PAIRS);
-      ta[k] = load(out_of(th[k]), tc[k]);
-      if (tc[k] + 1 < n) tb[k] = load(out_of(th[k]), tc[k] + 1);
-    }
-  }
-
-  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
-  auto input64 = [&](const Elem &e) -> double {
-    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), static_cast<double>(e.g),
-                    static_cast<double>(e.b));
-  };
-  // exact scales: fp64 maximum over the candidate elements
-  double m0 = 0.0, m1 = 0.0;
-#pragma unroll
-  for (int k = 0; k < CE; ++k) {
-    if (cv[k]) {
-      const double v = fabs(input64(ce[k]));
-      if (co[k] == 0) m0 = fmax(m0, v); else m1 = fmax(m1, v);
-    }
-  }
-  const double inv_q = 1.0 / static_cast<double>(QI);
-  float sc[2] = {0.f, 0.f};
-  sc[0] = __double2float_rn(__dmul_rn(group_max_d(m0, gmask, g), inv_q));
-  if (NOUT == 2) sc[1] = __double2float_rn(__dmul_rn(group_max_d(m1, gmask, g), inv_q));
-  if (l == 0) {
-    p.scale[0][r] = sc[0];
-    if (NOUT == 2) p.scale[1][r] = sc[1];
-  }
-  // near-tie codes in fp64, one element pair (one INT4 byte) at a time
-  auto put = [&](uint32_t hd, int c, const Elem &e0, const Elem &e1) {
-    const int o = out_of(hd);
-    const float so = o == 0 ? sc[0] : sc[1];
-    const double rs = so == 0.f ? 0.0 : rcp64(so);
-    const int q0 = so == 0.f ? 0 : code_of_t(__dmul_rn(input64(e0), rs), QI);
-    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code_of_t(__dmul_rn(input64(e1), rs), QI);
-    if (INT4) {
-      p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
-    } else {
-      p.y[o][r * n + c] = static_cast<uint8_t>(q0);
-      if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
-    }
-  };
-#pragma unroll
-  for (int k = 0; k < 2; ++k)
-    if (tv[k]) put(th[k], tc[k], ta[k], tb[k]);
-  for (int q = l + 2 * g; q < nt * PAIRS; q += g) {  // more than two pairs per lane
-    const uint32_t hd = static_cast<uint32_t>(ent[kCandCap + q / PAIRS]);
-    const int c = U * unit_of(hd) + 2 * (q % PAIRS);
-    const Elem e0 = load(out_of(hd), c);
-    const Elem e1 = c + 1 < n ? load(out_of(hd), c + 1) : zero;
-    put(hd, c, e0, e1);
-  }
-}
-
-// The CTA settles its own rows (local rows 0 .. nrows-1 = global rows row0,
-// row0 + row_step, ...) from the records in its shared memory, after its last
-// row: a group of lanes per row (32, 16 or 8: as many rows at once as the
-// CTA's threads allow).  Rows whose record overflowed, or that the fast path
-// flagged, are recomputed whole in fp64 by their group.
-template <class T, bool INT4, int NOUT, bool ADD, int U>
-__device__ __forceinline__ void tail_settle(const KParams &p, const unsigned char *trec, int nrows,
-                                            int64_t row0, int64_t row_step) {
-  const int nthreads = static_cast<int>(blockDim.x);
-  int g = 32;
-  while (g > 8 && nthreads / g < nrows) g >>= 1;
-  const int groups = nthreads / g;
-  const int wl = static_cast<int>(threadIdx.x) & 31;
-  const int l = wl & (g - 1);
-  const unsigned gmask = g == 32 ? 0xFFFFFFFFu : ((1u << g) - 1u) << (wl & ~(g - 1));
-  for (int i = static_cast<int>(threadIdx.x) / g; i < nrows; i += groups) {
-    const TailHead *h = reinterpret_cast<const TailHead *>(trec + static_cast<size_t>(i) * p.trec_bytes);
-    const int *ent = reinterpret_cast<const int *>(h + 1);
-    const int64_t r = row0 + static_cast<int64_t>(i) * row_step;
-    const int nc = h->cnt[0], nt = h->cnt[1];
-    if ((h->flags & RF_REDO) || nc > kCandCap || nt > p.tie_cap)
-      exact_row_lanes<T, INT4, NOUT, ADD>(p, r, l, g, gmask);
-    else
-      settle_row_group<T, INT4, NOUT, ADD, U>(p, r, h->ss, nc, nt, ent, l, g, gmask);
-  }
-}
 
 // ---------------------------------------------------------------- row kernel
 
@@ -790,12 +687,9 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   const uint32_t stage_bytes = NIN * static_cast<uint32_t>(p.seg_units) * 16u;
 
   extern __shared__ __align__(128) unsigned char smem[];
-  // one CTA per row: records in shared memory, settled by this CTA after its
-  // last row; a cluster per row: records in the workspace, the settle kernel
-  constexpr bool tail = !CL;
   // 16-byte units keep B_k in shared memory (registers go to x and G_k)
   constexpr bool BSM = (W == 4);
-  const Layout lay = make_layout(nslots, NOUT, ring_depth, tail ? p.tail_rows : 0, p.trec_bytes,
+  const Layout lay = make_layout(nslots, NOUT, ring_depth, p.rec_bytes,
                                  bsm_bytes_for(BSM, NOUT, UPT, static_cast<int>(blockDim.x)));
   float4 *bsm = reinterpret_cast<float4 *>(smem + lay.bsm);
   auto bsm_at = [&](int o, int k, int j) -> float4 & {
@@ -804,10 +698,67 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   double *ss_slots = reinterpret_cast<double *>(smem + lay.ss);      // [nslots]
   float *wmax_slots = reinterpret_cast<float *>(smem + lay.wmax);    // [NOUT][nslots]
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
-  int *lcnt = reinterpret_cast<int *>(smem + lay.amax);                // [2 parity][2 lists]
   int *rflags = reinterpret_cast<int *>(smem + lay.flags);           // [2]
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
+  int64_t *srow = reinterpret_cast<int64_t *>(smem + lay.srow);
   unsigned char *ring = smem + lay.ring;
+
+  // ---- the first rows' copies go out before anything else (the parameter
+  // loads and the set-up exchange overlap them).  The other threads wait on
+  // the barriers only after the set-up exchange below.
+  // staged: row `row` goes to stage s, x1 then x2; the barrier expects `hold`
+  // bytes more than the copies bring (testing only: then the wait runs out)
+  uint64_t policy = 0;
+  auto issue = [&](int64_t row, int s, uint32_t hold) {
+    const uint32_t bar = smem_addr(&bars[s]);
+    const uint32_t dst = smem_addr(ring + static_cast<size_t>(s) * stage_bytes);
+    const int64_t off = row * n + static_cast<int64_t>(seg_begin) * 8;
+    mbar_arrive_expect_tx(bar, NIN * seg_bytes + hold);
+    bulk_g2s(dst, p.x1 + off, seg_bytes, bar, policy);
+    if (ADD) bulk_g2s(dst + seg_bytes, p.x2 + off, seg_bytes, bar, policy);
+  };
+  if (MODE == LOAD_STAGED && tid == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // The rows a CTA (cluster) takes, in order, as the thread that issues the
+  // copies sees them: rows below p.dyn_base are dealt out in turn (c, c + G,
+  // ...); the others are handed out one at a time by the workspace counter,
+  // so that CTAs that run faster take more of them.  A ticket is fetched one
+  // take ahead: its latency overlaps a row.  -1: no more rows.
+  // The hand-out state lives in shared memory (registers are scarce), all but
+  // the prefetched ticket, whose load is waited for only at the next take.
+  const bool dyn = MODE == LOAD_STAGED && !CL && p.dyn_base < p.rows;
+  TakeState *ts = reinterpret_cast<TakeState *>(smem + lay.take);
+  int ticket = 0;
+  auto take = [&]() -> int64_t {
+    const int64_t nx = ts->nxt;
+    if (nx < p.dyn_base) {
+      ts->nxt = nx + nclusters;
+      if (dyn && nx + nclusters >= p.dyn_base) ticket = atomicAdd(p.sched, 1);  // the first ticket
+      return nx < p.rows ? nx : -1;
+    }
+    if (!dyn || ts->dry) return -1;
+    const int64_t r = p.dyn_base + ticket;
+    if (r >= p.rows || r < p.dyn_base) {
+      ts->dry = 1;
+      return -1;
+    }
+    ticket = atomicAdd(p.sched, 1);
+    ts->ndyn += 1;
+    return r;
+  };
+  if (MODE == LOAD_STAGED && tid == 0) {
+    ts->nxt = cluster_id;
+    ts->ndyn = 0;
+    ts->dry = 0;
+    policy = policy_evict_normal();
+    for (int s = 0; s < stages; ++s) {
+      const int64_t row = take();
+      srow[s] = row;
+      if (row >= 0 && seg_len > 0) issue(row, s, s == 0 ? p.test_hold_tx : 0u);
+    }
+  }
 
   // ---- folded parameters for this thread's units: input_k = x*rinv*G_k + B_k
   float2 G[NOUT][UPT][W], B[NOUT][UPT][W];
@@ -896,21 +847,17 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     const float v = warp_max_nonneg(maxB[o]);
     if (lane == 0) ex.publish(maxb_slots, o * nslots + my_slot, v);
   }
-  if (tid < 4) lcnt[tid] = 0;
   if (tid < 2) rflags[tid] = 0;
-  auto thead = [&](int64_t i) -> TailHead * {
-    return reinterpret_cast<TailHead *>(smem + lay.trec + static_cast<size_t>(i) * p.trec_bytes);
+  // the record of row iteration i: slot i % 3, in the shared memory of the
+  // cluster's first CTA
+  unsigned char *const recs = ex.first_cta(smem + lay.recs);
+  auto slot = [&](int64_t i) -> RecHead * {
+    return reinterpret_cast<RecHead *>(recs + static_cast<int>(i % 3) * p.rec_bytes);
   };
-  if (tail) {
-    for (int i = tid; i < p.tail_rows; i += blockDim.x) {
-      TailHead *th = thead(i);
-      th->cnt[0] = th->cnt[1] = 0;
-      th->flags = 0;
-    }
-  }
-  if (MODE == LOAD_STAGED && tid == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  if (rank == 0 && tid < 3) {
+    RecHead *h = reinterpret_cast<RecHead *>(smem + lay.recs + tid * p.rec_bytes);
+    h->cnt[0] = h->cnt[1] = 0;
+    h->flags = 0;
   }
   ex.sync();
   float maxBg[NOUT];  // bound on |B_k| over the whole row
@@ -921,53 +868,81 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     maxBg[o] = warp_max_nonneg(m);
   }
 
-  // staged: row `row` goes to stage s, x1 then x2
-  uint64_t policy = 0;
-  auto issue = [&](int64_t row, int s) {
-    const uint32_t bar = smem_addr(&bars[s]);
-    const uint32_t dst = smem_addr(ring + static_cast<size_t>(s) * stage_bytes);
-    const int64_t off = row * n + static_cast<int64_t>(seg_begin) * 8;
-    mbar_arrive_expect_tx(bar, NIN * seg_bytes);
-    bulk_g2s(dst, p.x1 + off, seg_bytes, bar, policy);
-    if (ADD) bulk_g2s(dst + seg_bytes, p.x2 + off, seg_bytes, bar, policy);
-  };
-  if (MODE == LOAD_STAGED && tid == 0 && seg_len > 0) {
-    policy = policy_evict_normal();
-    for (int s = 0; s < stages; ++s) {
-      const int64_t row = cluster_id + s * nclusters;
-      if (row < p.rows) issue(row, s);
+  // the codes of unit u (8 or 2 elements, low bits of bits[]) of row `row`
+  auto store_codes = [&](uint8_t *y, int64_t row, int u, const uint32_t (&bits)[2 * W]) {
+    if (MODE != LOAD_SCALAR) {
+      if (INT4) {  // 8 codes -> 4 bytes, even column in the low nibble
+        uint32_t w = 0;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) w |= (bits[e] & 0xFu) << (4 * e);
+        __stcs(reinterpret_cast<unsigned int *>(y + row * (n / 2) + static_cast<int64_t>(u) * 4),
+               w);
+      } else {     // 8 codes -> 8 bytes
+        const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
+                                        __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
+        const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
+                                        __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
+        __stcs(reinterpret_cast<uint2 *>(y + row * n + static_cast<int64_t>(u) * 8),
+               make_uint2(lo, hi));
+      }
+    } else {
+      if (INT4) {
+        y[row * (n / 2) + u] = static_cast<uint8_t>((bits[0] & 0xFu) | ((bits[1] & 0xFu) << 4));
+      } else {
+        const int64_t j = row * n + 2 * static_cast<int64_t>(u);
+        y[j] = static_cast<uint8_t>(bits[0] & 0xFFu);
+        if (2 * u + 1 < n) y[j + 1] = static_cast<uint8_t>(bits[1] & 0xFFu);
+      }
     }
-  }
+  };
 
-  // ---- row records
-  int64_t prev_row = -1;
-  auto header = [&](int64_t r) -> int * {
-    return reinterpret_cast<int *>(p.records + r * p.rec_bytes);
-  };
-  // record unit u of output o on list l (0 candidate, 1 near tie) of row r;
-  // an overflowing list only counts, and the row goes to the slow path
-  int64_t it = 0;          // rows this CTA has processed
-  auto record = [&](int l, int pp, int64_t r, int u, int o) {
-    const int entry = static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
-    if (tail) {
-      TailHead *th = thead(it);
-      const int k = atomicAdd(&th->cnt[l], 1);
-      if (k < (l == 0 ? kCandCap : p.tie_cap))
-        reinterpret_cast<int *>(th + 1)[l == 0 ? k : kCandCap + k] = entry;
-      return;
-    }
-    const int k = atomicAdd(ex.lcnt_slot(lcnt, pp * 2 + l), 1);
+  // ---- row records: unit u of output o on list l (0 candidate, 1 near tie) of
+  // the current row, with its G_k and B_k; an overflowing list only counts,
+  // and the row goes to the slow path
+  int64_t it = 0;          // rows this CTA (cluster) has processed
+  auto record = [&](int l, int u, int o, const float2 (&gk)[W], const float2 (&bk)[W]) {
+    RecHead *h = slot(it);
+    const int k = atomicAdd(&h->cnt[l], 1);
     if (k >= (l == 0 ? kCandCap : p.tie_cap)) return;
-    header(r)[16 + (l == 0 ? k : kCandCap + k)] = entry;
+    const int ent = l == 0 ? k : kCandCap + k;
+    rec_ue(h)[ent] = static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
+    float *v = reinterpret_cast<float *>(rec_ent(h, p.tie_cap, ent));
+    if (W == 4) {
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        reinterpret_cast<float4 *>(v + 8)[j] = make_float4(gk[2 * j].x, gk[2 * j].y,
+                                                           gk[2 * j + 1].x, gk[2 * j + 1].y);
+        reinterpret_cast<float4 *>(v + 16)[j] = make_float4(bk[2 * j].x, bk[2 * j].y,
+                                                            bk[2 * j + 1].x, bk[2 * j + 1].y);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < W; ++i) {
+        reinterpret_cast<float2 *>(v + 8)[i] = gk[i];
+        reinterpret_cast<float2 *>(v + 16)[i] = bk[i];
+      }
+    }
   };
+  // the settling warp: the last warp of the cluster's first CTA
+  const bool settler = rank == 0 && warp == nwarps - 1;
 
-  int stage = 0;          // staged: it % stages, kept incrementally
-  uint32_t phase = 0;     // staged: (it / stages) & 1, the mbarrier phase to wait for
-  for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
+  int stage = 0;           // staged: it % stages, kept incrementally
+  uint32_t phase = 0;      // staged: (it / stages) & 1, the mbarrier phase to wait for
+  int64_t prev_row = -1;   // the row of the previous iteration
+  int64_t prev2_row = -1;  // and of the one before
+  for (;; ++it) {
+    int64_t row;
+    if (MODE == LOAD_STAGED) {
+      row = srow[stage];
+      if (row < 0) break;
+    } else {
+      row = cluster_id + it * nclusters;
+      if (row >= p.rows) break;
+    }
     const int par = static_cast<int>(it & 1);
     bool timed_out = false;
     if (MODE == LOAD_STAGED && seg_len > 0) {
-      timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), phase);
+      timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), phase, p.wait_limit_ns);
     }
 
     // ---- pass 1: x = RN16(x1 + x2) (or x1), xOut, sum of squares (fp64)
@@ -1053,19 +1028,19 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
           if (seg_len > 0) {
             for (int s = 0; s < stages; ++s) {
               const int64_t it2 = it + s;  // the ring's outstanding iterations
-              if (cluster_id + it2 * nclusters >= p.rows) break;
+              if (srow[it2 % stages] < 0) break;
               mbar_wait_bounded(smem_addr(&bars[it2 % stages]),
-                                static_cast<uint32_t>((it2 / stages) & 1));
+                                static_cast<uint32_t>((it2 / stages) & 1), p.wait_limit_ns);
             }
           }
         }
-        prev_row = -1;
         break;
       }
-      // every thread has read this stage: refill it
-      if (tid == 0 && seg_len > 0) {
-        const int64_t nrow = row + static_cast<int64_t>(stages) * nclusters;
-        if (nrow < p.rows) issue(nrow, stage);
+      // every thread has read this stage (and its row): refill it
+      if (tid == 0) {
+        const int64_t nrow = take();
+        srow[stage] = nrow;
+        if (nrow >= 0 && seg_len > 0) issue(nrow, stage, 0u);
       }
     }
 
@@ -1076,7 +1051,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
       ss_row = warp_sum_d(ss_row);
     }
-    // v = ss/n + eps; 1/sqrt(v) in binary32 for the bulk, in fp64 when needed
+    // v = ss/n + eps; 1/sqrt(v) in binary32 for the bulk
     const double v64 = __fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps));
     const float v32 = __double2float_rn(v64);
     float2 rinv2;
@@ -1085,28 +1060,11 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       rinv2 = make_float2(r, r);
     }
     // the record: this row's sum of squares and flags (outside the normal
-    // binary32 range the bulk arithmetic is not trusted), the previous row's
-    // unit counts; this row's counters start at zero
+    // binary32 range the bulk arithmetic is not trusted: the slow path)
     if (tid == 0 && rank == 0) {
-      const int fl0 =
-          (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
-      if (tail) {
-        TailHead *th = thead(it);
-        th->ss = ss_row;
-        th->flags = fl0;
-      }
-    }
-    if (!tail && tid == 0 && rank == 0) {
-      int *h = header(row);
-      *reinterpret_cast<double *>(h) = ss_row;
-      h[4] = (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
-      if (prev_row >= 0) {
-        int *hp = header(prev_row);
-        hp[2] = lcnt[(par ^ 1) * 2 + 0];
-        hp[3] = lcnt[(par ^ 1) * 2 + 1];
-      }
-      lcnt[par * 2 + 0] = 0;
-      lcnt[par * 2 + 1] = 0;
+      RecHead *h = slot(it);
+      h->ss = ss_row;
+      h->flags = (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
     }
 
     // ---- pass 2: binary32 maxima of |input_k|, per unit and over the row
@@ -1136,7 +1094,8 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     if (tid == 0) rflags[par ^ 1] = 0;
 
     // ---- pass 3: quantize with the approximate scale s~ = max / Q (rounded half
-    // to even via the 1.5*2^23 trick); queue the codes near a half-way point
+    // to even via the 1.5*2^23 trick); record the candidate units and the
+    // units with a code near a half-way point
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
       float gm = 0.f;
@@ -1146,19 +1105,12 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       const float sa = gm * (1.f / QF);
       const bool normal = sa >= 1.1754943508222875e-38f;
       // 1/s~ would overflow: the slow path
-      if (sa != 0.f && !normal && tid == 0 && rank == 0) {
-        if (tail) thead(it)->flags = RF_REDO; else header(row)[4] = RF_REDO;
-      }
+      if (sa != 0.f && !normal && tid == 0 && rank == 0) slot(it)->flags = RF_REDO;
       const float r32 = normal ? __frcp_rn(sa) : 0.f;
-      // candidates for the row maximum: within the binary32 error of it
-      const float thr = gm - 12.f * kUnit * (gm + maxBg[o]);
-      if (gm > 0.f) {  // about one unit per row
-#pragma unroll
-        for (int k = 0; k < UPT; ++k) {
-          const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
-          if (mu[o][k] >= thr && u < seg_end) record(0, par, row, u, o);
-        }
-      }
+      // candidates for the row maximum: every binary32 input is within
+      // 3u|input| + 12u max|B| of its value scaled by the row's common 1/Rms
+      // error: the true maximum's unit is at or above thr
+      const float thr = gm - 12.f * kUnit * gm - 24.f * kUnit * maxBg[o];
       // |t - t_exact| <= tau: the binary32 error of t (12u(Q + |B| r) + 2uQ) plus
       // the distance between s~ and the exact scale (10uQ + 6u maxB r)
       const float tau = 24.f * kUnit * QF + 18.f * kUnit * maxBg[o] * r32;
@@ -1169,6 +1121,11 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       for (int k = 0; k < UPT; ++k) {
         const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
         if (u >= seg_end) continue;
+        if (gm > 0.f && mu[o][k] >= thr) {  // about one unit a row
+          float2 bk[W];
+          b_of(o, k, bk);
+          record(0, u, o, G[o][k], bk);
+        }
         uint32_t bits[2 * W];  // low bits: the code (two's complement)
         float dmax = 0.f;      // largest |t - RNE(t)| of the unit
         float2 bk[W];
@@ -1188,68 +1145,78 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
           bits[2 * i + 1] = __float_as_uint(m.y);
           dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
         }
-        if (MODE != LOAD_SCALAR) {
-          if (INT4) {  // 8 codes -> 4 bytes, even column in the low nibble
-            uint32_t w = 0;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) w |= (bits[e] & 0xFu) << (4 * e);
-            __stcs(reinterpret_cast<unsigned int *>(y + row * (n / 2) +
-                                                    static_cast<int64_t>(u) * 4), w);
-          } else {     // 8 codes -> 8 bytes
-            const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
-                                            __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
-            const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
-                                            __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
-            __stcs(reinterpret_cast<uint2 *>(y + row * n + static_cast<int64_t>(u) * 8),
-                   make_uint2(lo, hi));
-          }
-        } else {
-          if (INT4) {
-            y[row * (n / 2) + u] =
-                static_cast<uint8_t>((bits[0] & 0xFu) | ((bits[1] & 0xFu) << 4));
-          } else {
-            const int64_t j = row * n + 2 * static_cast<int64_t>(u);
-            y[j] = static_cast<uint8_t>(bits[0] & 0xFFu);
-            if (2 * u + 1 < n) y[j + 1] = static_cast<uint8_t>(bits[1] & 0xFFu);
-          }
-        }
+        store_codes(y, row, u, bits);
         // some code of the unit is near a half-way point (rare): record the unit
-        if (dmax > lim) record(1, par, row, u, o);
+        if (dmax > lim) {
+          if (NOUT == 1) b_of(o, k, bk);
+          record(1, u, o, G[o][k], bk);
+        }
       }
     }
     if (MODE == LOAD_STAGED && ++stage == stages) {
       stage = 0;
       phase ^= 1u;
     }
+    // ---- the settling warp, while the next row's copy is in flight: the
+    // previous row's record is complete (two barriers have passed since):
+    // fetch its units' x; the row before that has its x in place: settle it
+    if (settler) {
+      if (it >= 1) prefetch_record<ADD, U>(p, slot(it - 1), prev_row, lane);
+      if (it >= 2) {
+        cp_async_wait<1>();
+        __syncwarp();
+        settle_record<T, INT4, NOUT, ADD, U>(p, slot(it - 2), prev2_row, lane);
+      }
+    }
+    prev2_row = prev_row;
     prev_row = row;
   }
 
   // the next kernel on the stream may start its set-up (it waits for this
   // grid's completion before it reads anything)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // ---- in-kernel settling of this CTA's rows (rows 0 .. it-1 are complete)
-  if (tail) {
-    __syncthreads();
-    tail_settle<T, INT4, NOUT, ADD, U>(p, smem + lay.trec, static_cast<int>(it), cluster_id,
-                                       nclusters);
-    return;
-  }
-  // ---- the last row's unit counts (the settle kernel takes it from here)
-  if (prev_row >= 0) {
-    const int par = static_cast<int>((it + 1) & 1);  // the last row's parity
+  // ---- settle the last two rows (rows 0 .. it-1 are complete; all but the
+  // last two are settled, and the x of row it-2 is on its way)
+  if (it >= 1) {
     ex.sync();
-    if (tid == 0 && rank == 0) {
-      int *hp = header(prev_row);
-      hp[2] = lcnt[par * 2 + 0];
-      hp[3] = lcnt[par * 2 + 1];
+    if (settler) {
+      prefetch_record<ADD, U>(p, slot(it - 1), prev_row, lane);
+      if (it >= 2) {
+        cp_async_wait<1>();
+        __syncwarp();
+        settle_record<T, INT4, NOUT, ADD, U>(p, slot(it - 2), prev2_row, lane);
+      }
+      cp_async_wait<0>();
+      __syncwarp();
+      settle_record<T, INT4, NOUT, ADD, U>(p, slot(it - 1), prev_row, lane);
     }
   }
-  // no CTA leaves while a peer may still touch its shared memory
-  if (CL) ex.sync();
+  // ---- the last CTA to finish returns the hand-out counters to zero (every
+  // CTA's tickets are taken before it counts itself done) and checks that
+  // every dynamic row was handed out exactly once and each CTA drew one empty
+  // ticket: counters that were not zero when the call started fail this
+  if (dyn && tid == 0) {
+    atomicAdd(p.sched + 2, ts->ndyn);
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+      __threadfence();
+      const int handed = atomicExch(p.sched, 0);
+      const int taken = atomicExch(p.sched + 2, 0);
+      atomicExch(p.sched + 1, 0);
+      const int64_t pool = p.rows - p.dyn_base;
+      if ((static_cast<int64_t>(taken) != pool ||
+           static_cast<int64_t>(handed) != pool + gridDim.x) &&
+          atomicCAS(p.status, 0, DEV_SCHED) == 0)
+        *reinterpret_cast<volatile int64_t *>(p.status + 2) = -1;
+    }
+  }
 }
 
+// At most 128 registers a thread (two 256-thread CTAs per SM), whatever the
+// launch bound allows.
 template <class T, bool INT4, int MODE, int UPT, int NOUT, bool ADD, bool CL>
-__global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT))
+__global__ void __launch_bounds__(max_threads_for(MODE, UPT, NOUT),
+                                  max_threads_for(MODE, UPT, NOUT) <= 256 ? 2 : 1)
     rows_kernel(const __grid_constant__ KParams p) {
   rows_body<T, INT4, MODE, UPT, NOUT, ADD, CL>(p);
 }

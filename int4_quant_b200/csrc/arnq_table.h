@@ -59,27 +59,7 @@ void fill_quarter(KernelFn *t) {
   fill_na<T, I4, 2, true, CL>(t);
 }
 
-// The settle kernels: by output count, add / no-add, and unit size (8: vector
-// and staged row kernels; 2: scalar).
-typedef void (*SettleFn)(KParams);
-constexpr int kSettleSize = 2 * 2 * 2;
-inline int settle_index(int nout, bool add, bool vec) {
-  return ((nout - 1) * 2 + (add ? 1 : 0)) * 2 + (vec ? 1 : 0);
-}
-template <class T, bool I4>
-void fill_settle(SettleFn *t) {
-  t[settle_index(1, false, false)] = settle_kernel<T, I4, 1, false, 2>;
-  t[settle_index(1, false, true)] = settle_kernel<T, I4, 1, false, 8>;
-  t[settle_index(1, true, false)] = settle_kernel<T, I4, 1, true, 2>;
-  t[settle_index(1, true, true)] = settle_kernel<T, I4, 1, true, 8>;
-  t[settle_index(2, false, false)] = settle_kernel<T, I4, 2, false, 2>;
-  t[settle_index(2, false, true)] = settle_kernel<T, I4, 2, false, 8>;
-  t[settle_index(2, true, false)] = settle_kernel<T, I4, 2, true, 2>;
-  t[settle_index(2, true, true)] = settle_kernel<T, I4, 2, true, 8>;
-}
-
-// Defined one per translation unit (arnq_k_<dtype>_<codes>[_cl].cu; the
-// settle kernels in the ones without _cl).
+// Defined one per translation unit (arnq_k_<dtype>_<codes>[_cl].cu).
 void fill_table_bf16_int8(KernelFn *t);
 void fill_table_bf16_int4(KernelFn *t);
 void fill_table_fp16_int8(KernelFn *t);
@@ -88,9 +68,5 @@ void fill_table_bf16_int8_cl(KernelFn *t);
 void fill_table_bf16_int4_cl(KernelFn *t);
 void fill_table_fp16_int8_cl(KernelFn *t);
 void fill_table_fp16_int4_cl(KernelFn *t);
-void fill_settle_bf16_int8(SettleFn *t);
-void fill_settle_bf16_int4(SettleFn *t);
-void fill_settle_fp16_int8(SettleFn *t);
-void fill_settle_fp16_int4(SettleFn *t);
 
 }  // namespace arnq

@@ -27,8 +27,18 @@ _LIB = os.path.join(_HERE, "libarnq_oracle.so")
 # The oracle's own status codes (see arnq_oracle.c).
 ORC_OK, ORC_BAD_MASK, ORC_EMPTY, ORC_BAD_SHAPE, ORC_NULL, ORC_BAD_ARG = range(6)
 DTYPES = {"bf16": 0, "fp16": 1}
-QDTYPES = {"int8": 0, "int4": 1}
-QMAX = {"int8": 127, "int4": 7}
+QDTYPES = {"int8": 0, "int4": 1, "int4_int32": 2}
+QMAX = {"int8": 127, "int4": 7, "int4_int32": 7}
+
+
+def _code_array(rows, n, qdtype):
+    """Output array of one quantized output: int8 [rows, n], packed uint8
+    [rows, n/2], or uint32 words [rows, n/8] of eight INT4 codes."""
+    if qdtype == "int8":
+        return np.zeros((rows, n), np.int8)
+    if qdtype == "int4_int32":
+        return np.zeros((rows, n // 8 if n % 8 == 0 else 0), np.uint32)
+    return np.zeros((rows, n // 2), np.uint8)
 
 
 def build(force: bool = False) -> str:
@@ -111,7 +121,8 @@ def add_rms_norm_dynamic_quant_v2(x1, x2, gamma, beta=None, smooth1=None, smooth
 
     Returns a dict with "status", and, when it is ORC_OK: "x_out" (uint16 bits),
     "y1"/"scale1" and "y2"/"scale2" (None when not produced; codes are int8
-    [rows, n] or packed uint8 [rows, n/2]), "clamp_hits", and with debug=True
+    [rows, n], packed uint8 [rows, n/2], or for qdtype "int4_int32" uint32
+    [rows, n/8] words of eight codes), "clamp_hits", and with debug=True
     the fp64 "in1"/"in2" arrays.
     """
     x1 = _u16(x1)
@@ -124,12 +135,10 @@ def add_rms_norm_dynamic_quant_v2(x1, x2, gamma, beta=None, smooth1=None, smooth
            "x_out": None, "in1": None, "in2": None, "clamp_hits": 0}
     if st != ORC_OK:
         return out
-    cb = n if qdtype == "int8" else n // 2
-    cdt = np.int8 if qdtype == "int8" else np.uint8
     x_out = np.zeros((rows, n), np.uint16)
-    y1 = np.zeros((rows, cb), cdt) if on1 else None
+    y1 = _code_array(rows, n, qdtype) if on1 else None
     s1 = np.zeros((rows,), np.float32) if on1 else None
-    y2 = np.zeros((rows, cb), cdt) if on2 else None
+    y2 = _code_array(rows, n, qdtype) if on2 else None
     s2 = np.zeros((rows,), np.float32) if on2 else None
     in1 = np.zeros((rows, n), np.float64) if debug else None
     in2 = np.zeros((rows, n), np.float64) if debug else None
@@ -150,8 +159,7 @@ def rms_norm_dynamic_quant(x, gamma, beta=None, smooth=None, *, eps: float,
     x = _u16(x)
     rows, n = x.shape if x.ndim == 2 else (0, 0)
     gamma, beta, smooth = _u16(gamma, (n,)), _u16(beta, (n,)), _u16(smooth, (n,))
-    cb = n if qdtype == "int8" else n // 2
-    y = np.zeros((rows, cb), np.int8 if qdtype == "int8" else np.uint8)
+    y = _code_array(rows, n, qdtype)
     scale = np.zeros((rows,), np.float32)
     dbg = np.zeros((rows, n), np.float64) if debug else None
     hits = ctypes.c_int64(0)

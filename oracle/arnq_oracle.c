@@ -27,7 +27,10 @@
  *     stored value; round() is round-half-to-even; codes are clamped to
  *     [-Q, Q] as a guard that the arithmetic never needs (hits are counted).
  *   - Q = 127 for INT8, 7 for INT4; INT4 codes are packed two per byte,
- *     two's-complement nibbles, the even index in the low nibble.
+ *     two's-complement nibbles, the even index in the low nibble.  The
+ *     alternate INT4 container (the page names no container) holds eight
+ *     codes per 32-bit word: code 8w + k of a row in bits 4k .. 4k+3 of word
+ *     w (two's-complement nibbles), for rows whose length is a multiple of 8.
  *   - a row whose scale is 0 (all inputs 0) yields scale 0 and all codes 0.
  *   - y2 is produced with the mask absent only when both smooth scales are
  *     given.
@@ -51,7 +54,7 @@
 #define ORC_OK 0
 #define ORC_BAD_MASK 1  /* a Constraints-section rule on outputMask / smooth scales */
 #define ORC_EMPTY 2     /* empty tensor: not supported (aclnnRmsNormDynamicQuant) */
-#define ORC_BAD_SHAPE 3 /* INT4 with an odd row length cannot be packed */
+#define ORC_BAD_SHAPE 3 /* INT4 with a row length its container cannot pack */
 #define ORC_NULL 4      /* a required input or a selected output is missing */
 #define ORC_BAD_ARG 5   /* unknown dtype / qdtype, negative or non-finite eps */
 
@@ -59,6 +62,7 @@
 #define ORC_FP16 1
 #define ORC_INT8 0
 #define ORC_INT4 1
+#define ORC_INT4_WORDS 2 /* INT4 codes, eight per 32-bit word */
 
 /* ------------------------------------------------------------------------- */
 /* 16-bit floating-point formats, written from their definitions.            */
@@ -194,10 +198,12 @@ int orc_selected_outputs(int mask, int has_s1, int has_s2, int *y1_on, int *y2_o
 /* Dynamic per-row symmetric quantization of one row of fp64 inputs:
  * scale = row_max(abs(input)) / Q rounded to binary32, code = round(input /
  * scale) with round-half-even, clamped to [-Q, Q] (guard; hits counted).
- * Writes n int8 codes, or n/2 packed INT4 bytes (even index in the low nibble). */
+ * Writes n int8 codes, n/2 packed INT4 bytes (even index in the low nibble),
+ * or n/8 32-bit words of eight INT4 codes (code k of a word in bits 4k..4k+3). */
 static void quantize_row(const double *in, int64_t n, int qdtype, uint8_t *codes_out,
                          float *scale_out, int64_t *clamp_hits) {
   double qmax = (qdtype == ORC_INT8) ? 127.0 : 7.0;
+  uint32_t *words = (uint32_t *)codes_out;
   double amax = 0.0;
   for (int64_t j = 0; j < n; ++j) {
     double a = fabs(in[j]);
@@ -215,6 +221,10 @@ static void quantize_row(const double *in, int64_t n, int qdtype, uint8_t *codes
     int code = (int)q;
     if (qdtype == ORC_INT8) {
       codes_out[j] = (uint8_t)(int8_t)code;
+    } else if (qdtype == ORC_INT4_WORDS) {
+      uint32_t nib = (uint32_t)code & 0xFu; /* two's-complement nibble */
+      if ((j % 8) == 0) words[j / 8] = 0u;
+      words[j / 8] |= nib << (4 * (j % 8));
     } else {
       uint8_t nib = (uint8_t)(code & 0xF); /* two's-complement nibble */
       if ((j & 1) == 0) {
@@ -228,10 +238,11 @@ static void quantize_row(const double *in, int64_t n, int qdtype, uint8_t *codes
 
 static int check_common(int64_t rows, int64_t n, int dtype, float eps, int qdtype) {
   if (dtype != ORC_BF16 && dtype != ORC_FP16) return ORC_BAD_ARG;
-  if (qdtype != ORC_INT8 && qdtype != ORC_INT4) return ORC_BAD_ARG;
+  if (qdtype != ORC_INT8 && qdtype != ORC_INT4 && qdtype != ORC_INT4_WORDS) return ORC_BAD_ARG;
   if (!(eps >= 0.0f) || !isfinite(eps)) return ORC_BAD_ARG;
   if (rows <= 0 || n <= 0) return ORC_EMPTY;
   if (qdtype == ORC_INT4 && (n % 2) != 0) return ORC_BAD_SHAPE;
+  if (qdtype == ORC_INT4_WORDS && (n % 8) != 0) return ORC_BAD_SHAPE;
   return ORC_OK;
 }
 
@@ -239,7 +250,8 @@ static int check_common(int64_t rows, int64_t n, int dtype, float eps, int qdtyp
 /* [V2] aclnnAddRmsNormDynamicQuantV2, "Formula" section, row by row.        */
 /* All tensors row-major ("ND"): x1, x2, x_out, in1_dbg, in2_dbg are         */
 /* [rows, n]; gamma, beta, smooth1, smooth2 are [n]; scale1/scale2 are       */
-/* [rows]; y1/y2 are [rows, n] int8 or [rows, n/2] packed INT4 bytes.        */
+/* [rows]; y1/y2 are [rows, n] int8, [rows, n/2] packed INT4 bytes, or      */
+/* [rows, n/8] 32-bit words of eight INT4 codes (4-byte aligned).            */
 /* in1_dbg / in2_dbg (optional) receive the fp64 input1 / input2 values.     */
 /* ------------------------------------------------------------------------- */
 int orc_add_rms_norm_dynamic_quant_v2(

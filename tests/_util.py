@@ -49,8 +49,22 @@ def unpack_int4(packed: np.ndarray) -> np.ndarray:
     return out
 
 
+def unpack_int4_words(words: np.ndarray) -> np.ndarray:
+    """32-bit words [..., n/8] -> signed codes [..., n]: code k of a word is its
+    bits 4k..4k+3, a two's-complement nibble (shifts on the word value, not a
+    reading of its bytes)."""
+    w = np.asarray(words).view(np.uint32).astype(np.int64)
+    out = np.empty(w.shape[:-1] + (w.shape[-1] * 8,), np.int16)
+    for k in range(8):
+        nib = (w >> (4 * k)) & 0xF
+        out[..., k::8] = np.where(nib >= 8, nib - 16, nib)
+    return out
+
+
 def codes(y, qdtype):
     """Signed integer codes of an output tensor (int8 as is; INT4 unpacked)."""
     if qdtype == "int8":
         return np.asarray(y).view(np.int8).astype(np.int16)
+    if qdtype == "int4_int32":
+        return unpack_int4_words(y)
     return unpack_int4(y)

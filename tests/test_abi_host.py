@@ -35,7 +35,7 @@ def test_exports_every_header_symbol():
 
 
 def test_status_strings():
-    for code in range(0, 12):
+    for code in range(0, 13):
         s = A.arnq_status_string(code)
         assert s.startswith("ARNQ_")
     assert "unknown" in A.arnq_status_string(99)
@@ -66,29 +66,28 @@ def test_selected_outputs_rejects_unknown_mask_bits():
     assert A.arnq_selected_outputs(-2, 0, 0)[0] == A.ARNQ_ERR_MASK
 
 
-def test_workspace_records_stay_aligned():
-    # per-row records hold a double: their size must keep every record 8-byte
-    # (here: 16-byte) aligned for any row length and output count
-    for n in list(range(2, 600, 2)) + [4096, 4098, 7168, 16384, 131072]:
-        for mask, s1, s2 in ((-1, 0, 0), (3, 1, 1)):
-            a = A.arnq_workspace_size(1, n, A.ARNQ_BF16, A.ARNQ_INT8, mask, s1, s2)[1]
-            b = A.arnq_workspace_size(2, n, A.ARNQ_BF16, A.ARNQ_INT8, mask, s1, s2)[1]
-            assert (b - a) % 16 == 0 and a % 16 == 0, (n, mask)
+def test_workspace_is_the_status_block_for_every_problem():
+    # the per-row bookkeeping stays on chip: the workspace is the 256-byte
+    # status block (status + row hand-out counters) whatever the shape, dtype,
+    # code type and outputs
+    for rows in (1, 2, 64, 8192, 16384, 2 ** 31 - 1):
+        for n in (2, 8, 1000, 4096, 7168, 16384, A.ARNQ_MAX_N):
+            for qdt in (A.ARNQ_INT8, A.ARNQ_INT4):
+                for mask, s1, s2 in ((-1, 0, 0), (1, 1, 0), (3, 1, 1), (-1, 1, 1)):
+                    st, nb = A.arnq_workspace_size(rows, n, A.ARNQ_BF16, qdt, mask, s1, s2)
+                    assert st == A.ARNQ_OK and nb == A.ARNQ_WORKSPACE_BYTES, (rows, n, qdt, mask)
 
 
 def test_workspace_size():
     st, nb = A.arnq_workspace_size(8192, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
-    assert st == A.ARNQ_OK and nb >= 16
-    # a status block plus one fixed-size record per row
-    st1, nb1 = A.arnq_workspace_size(1, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
-    st2, nb2 = A.arnq_workspace_size(2, 4096, A.ARNQ_BF16, A.ARNQ_INT8, 1, 1, 0)
-    assert st1 == st2 == A.ARNQ_OK and nb - nb1 == 8191 * (nb2 - nb1)
+    assert st == A.ARNQ_OK and nb == 256
     assert A.arnq_workspace_size(0, 4096, 0, 0, -1, 0, 0)[0] == A.ARNQ_ERR_EMPTY
     assert A.arnq_workspace_size(8, 0, 0, 0, -1, 0, 0)[0] == A.ARNQ_ERR_EMPTY
     assert A.arnq_workspace_size(8, 7, 0, A.ARNQ_INT4, -1, 0, 0)[0] == A.ARNQ_ERR_SHAPE
     assert A.arnq_workspace_size(8, A.ARNQ_MAX_N + 8, 0, 0, -1, 0, 0)[0] == A.ARNQ_ERR_SHAPE
     assert A.arnq_workspace_size(8, 64, 2, 0, -1, 0, 0)[0] == A.ARNQ_ERR_DTYPE
-    assert A.arnq_workspace_size(8, 64, 0, 2, -1, 0, 0)[0] == A.ARNQ_ERR_DTYPE
+    assert A.arnq_workspace_size(8, 64, 0, 3, -1, 0, 0)[0] == A.ARNQ_ERR_DTYPE
+    assert A.arnq_workspace_size(8, 60, 0, A.ARNQ_INT4_INT32, -1, 0, 0)[0] == A.ARNQ_ERR_SHAPE
     assert A.arnq_workspace_size(8, 64, 0, 0, 0, 0, 0)[0] == A.ARNQ_ERR_MASK
     assert A.arnq_workspace_size(-1, 64, 0, 0, -1, 0, 0)[0] == A.ARNQ_ERR_SHAPE
     L = A.lib()
@@ -122,8 +121,11 @@ def run(**kw):
     (dict(rows=-3), A.ARNQ_ERR_SHAPE),
     (dict(n=A.ARNQ_MAX_N + 2), A.ARNQ_ERR_SHAPE),
     (dict(n=63, qdt=A.ARNQ_INT4), A.ARNQ_ERR_SHAPE),
+    (dict(n=60, qdt=A.ARNQ_INT4_INT32), A.ARNQ_ERR_SHAPE),
+    (dict(qdt=A.ARNQ_INT4_INT32, y1=P["y1"] + 2), A.ARNQ_ERR_ALIGN),
     (dict(dt=5), A.ARNQ_ERR_DTYPE),
     (dict(qdt=-1), A.ARNQ_ERR_DTYPE),
+    (dict(qdt=3), A.ARNQ_ERR_DTYPE),
     (dict(eps=-1e-6), A.ARNQ_ERR_EPS),
     (dict(eps=math.nan), A.ARNQ_ERR_EPS),
     (dict(eps=math.inf), A.ARNQ_ERR_EPS),
@@ -168,7 +170,7 @@ def test_v1_and_no_add_entry_points_validate():
 
 
 def test_plan_struct_layout():
-    assert ctypes.sizeof(A.arnq_plan) == 32
+    assert ctypes.sizeof(A.arnq_plan) == 44
     assert ctypes.sizeof(A.arnq_workspace_status) == 16
 
 
@@ -182,11 +184,18 @@ def test_static_scratch_entry_validates_on_the_host():
     assert A.arnq_run_static_scratch(P["x1"], P["x2"], P["g"], None, None, P["s2"], 8, 64, 0, 1e-6,
                                      -1, 0, P["y1"], P["sc1"], None, None, None,
                                      None) == A.ARNQ_ERR_MASK
-    assert A.ARNQ_STATIC_SCRATCH_BYTES >= A.arnq_workspace_size(8, 64, 0, 0, -1, 0, 0)[1]
-    # a problem needing more than the static array is refused before any device work
-    big = 1
-    while A.arnq_workspace_size(big, 64, 0, 0, -1, 0, 0)[1] <= A.ARNQ_STATIC_SCRATCH_BYTES:
-        big *= 2
-    assert A.arnq_run_static_scratch(P["x1"], P["x2"], P["g"], None, None, None, big, 64, 0, 1e-6,
-                                     -1, 0, P["y1"], P["sc1"], None, None, None,
-                                     None) == A.ARNQ_ERR_WORKSPACE
+    # the static array covers the workspace of every valid problem, the largest too
+    assert A.ARNQ_STATIC_SCRATCH_BYTES >= A.arnq_workspace_size(2 ** 31 - 1, A.ARNQ_MAX_N, 0, 1,
+                                                                 3, 1, 1)[1]
+
+
+@pytest.mark.parametrize("field,value", [
+    ("schedule", 3), ("schedule", -1), ("test_hold_bytes", 65537), ("test_hold_bytes", -16),
+    ("wait_limit_us", -1), ("grid", -2), ("stages", -1), ("cluster", -4)])
+def test_plan_fields_out_of_range_are_refused_on_the_host(field, value):
+    p = A.arnq_plan()
+    setattr(p, field, value)
+    st = A.arnq_run_planned(P["x1"], P["x2"], P["g"], None, None, None, 16, 64, A.ARNQ_BF16, 1e-6,
+                            A.ARNQ_MASK_ABSENT, A.ARNQ_INT8, P["y1"], P["sc1"], None, None,
+                            P["xo"], P["ws"], 256, None, p)
+    assert st == A.ARNQ_ERR_PLAN

@@ -70,11 +70,22 @@ def test_bench_workload_floor():
 
 
 def test_launches_per_call():
+    # one kernel per call, whether a row has one CTA or a cluster
     class P:
         cluster = 1
     assert bench.launches_per_call(P) == 1
     P.cluster = 4
-    assert bench.launches_per_call(P) == 2
+    assert bench.launches_per_call(P) == 1
+
+
+def test_rotated_sets_cover_twice_the_l2():
+    class W:  # 64 x 1024 bf16, gamma only, one INT8 output: 461,056 bytes a call
+        rows, n, dtype, qdtype = 64, 1024, "bf16", "int8"
+        beta = smooth1 = smooth2 = None
+    assert bench.sets_for(W, True, False) == 3
+    k = bench.sets_for(W, True, False, min_bytes=300 << 20)
+    assert k == -(-(300 << 20) // 461_056) and k * 461_056 >= 300 << 20
+    assert bench.sets_for(W, True, False, min_bytes=1 << 40) == 2048
 
 
 def test_job_throughput_counts_every_rank():

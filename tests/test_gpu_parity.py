@@ -5,8 +5,9 @@ Acceptance (the operator's stated tolerance): xOut bit-exact; INT4 packing
 bit-exact (codes are compared after unpacking both sides with the same
 reader, and hand-worked rows compare raw bytes); scales within relative 1e-5;
 codes within +-1 with at most 1e-4 of them off by one.  Every run also checks
-that the workspace status block stayed clear and that outputs the call must
-not write kept their canary bytes.
+that the workspace status block stayed clear, that the row hand-out counters
+are back at zero, and that outputs the call must not write kept their canary
+bytes.
 """
 import numpy as np
 import pytest
@@ -25,7 +26,7 @@ OFF_BY_ONE_RATE = 1e-4
 CANARY = 0xA5
 
 DT = {"bf16": A.ARNQ_BF16, "fp16": A.ARNQ_FP16}
-QDT = {"int8": A.ARNQ_INT8, "int4": A.ARNQ_INT4}
+QDT = {"int8": A.ARNQ_INT8, "int4": A.ARNQ_INT4, "int4_int32": A.ARNQ_INT4_INT32}
 TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}
 
 
@@ -55,8 +56,8 @@ def canary_bytes(nbytes, offset=0):
 
 
 def workspace_for(rows, n):
-    """A workspace of the size arnq_workspace_size asks for with two outputs
-    (enough for any call on rows x n), status block zeroed."""
+    """A zeroed workspace of the size arnq_workspace_size asks for (the same
+    for every call: the status block and the row hand-out counters)."""
     st, nb = A.arnq_workspace_size(max(rows, 1), max(n, 2), A.ARNQ_BF16, A.ARNQ_INT8,
                                    A.ARNQ_MASK_Y1 | A.ARNQ_MASK_Y2, 1, 1)
     assert st == A.ARNQ_OK
@@ -91,8 +92,9 @@ def run_gpu(w, plan=None, offset=0, inplace=False, mask="use", smooth="use", str
         st = A.arnq_run_planned(*args, plan)
     assert st == A.ARNQ_OK, A.arnq_status_string(st)
     torch.cuda.synchronize()
-    wsh = ws[:16].cpu().numpy().view(np.int32)
+    wsh = ws[:32].cpu().numpy().view(np.int32)
     assert wsh[0] == 0, f"device status {wsh[0]}"
+    assert not wsh[4:7].any(), f"hand-out counters left at {wsh[4:7]}"
     out = {
         "y1": y1.cpu().numpy().reshape(rows, cb),
         "y2": y2.cpu().numpy().reshape(rows, cb),
@@ -215,9 +217,15 @@ PLAN_CASES = [
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=1, cluster=4),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=8, units=2),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=16),
-    # one CTA per row (settled in the row kernel's tail), also with few CTAs
-    # per SM: more rows per CTA, or a grid run in waves
+    # one CTA per row, also with few CTAs per SM (more rows per CTA), rows
+    # dealt out in turn or the last quarter handed out by the counter, and
+    # explicit grids (fewer CTAs than rows; more CTAs than rows)
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=1, grid=16),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=16),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=7, stages=2),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, grid=1000),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4, grid=12),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, units=2),
     dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=1),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, ctas_per_sm=1),
@@ -249,12 +257,13 @@ def test_scalar_plans(units, cluster):
 
 
 @pytest.mark.parametrize("rows,n", [(40000, 256), (300000, 64)])
-def test_many_rows_per_cta(rows, n):
-    # one resident CTA per SM: hundreds of rows per CTA, each CTA's records in
-    # its shared memory, settled after its last row; at 300000 rows one CTA
-    # cannot hold all its rows' records, so the grid grows (run in waves)
+@pytest.mark.parametrize("schedule", [1, 2])
+def test_many_rows_per_cta(rows, n, schedule):
+    # one resident CTA per SM: hundreds of rows per CTA, each settled one row
+    # behind from the two records in shared memory; with schedule 2 a quarter
+    # of the rows (tens of thousands) go through the hand-out counter
     w = wl.random_case(rows, n, seed=21, beta=True, smooth1=True)
-    p = plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1)
+    p = plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1, schedule=schedule)
     g, _ = run_gpu(w, plan=p)
     compare(g, run_oracle(w), "int8", f"{rows} rows")
 
@@ -313,8 +322,7 @@ def test_deterministic_rerun():
         assert np.array_equal(a[k].view(np.uint8), b[k].view(np.uint8)), k
 
 
-# one CTA per row (the row kernel settles its rows) or a cluster per row (the
-# settle kernel does)
+# one CTA per row, or a cluster per row (its first CTA holds the records)
 SETTLE_PLANS = [dict(cluster=1), dict(cluster=4)]
 
 
@@ -430,3 +438,109 @@ def test_non_default_stream():
     s = torch.cuda.Stream()
     g, _ = run_gpu(w, stream=s)
     compare(g, run_oracle(w), "int8", "side stream")
+
+
+# ------------------------------------------------------------------ device-side failure paths
+
+def _call_with_plan(w, p, ws, nb):
+    x1 = dev_bits(w.x1, w.dtype)
+    x2 = dev_bits(w.x2, w.dtype)
+    cb = w.n if w.qdtype == "int8" else w.n // 2
+    y1 = canary_bytes(w.rows * cb)
+    sc1 = canary_bytes(w.rows * 4).view(torch.float32)
+    xo = canary_bytes(w.rows * w.n * 2).view(torch.int16)
+    st = A.arnq_run_planned(x1, x2, dev_bits(w.gamma, w.dtype), dev_bits(w.beta, w.dtype),
+                            dev_bits(w.smooth1, w.dtype), None, w.rows, w.n, DT[w.dtype], w.eps,
+                            A.ARNQ_MASK_ABSENT, QDT[w.qdtype], y1, sc1, None, None, xo, ws, nb,
+                            None, p)
+    assert st == A.ARNQ_OK, A.arnq_status_string(st)
+    torch.cuda.synchronize()
+    h = ws[:32].cpu().numpy().view(np.int32)
+    return int(h[0]), int(h[2:4].view(np.int64)[0]), h[4:7].copy()
+
+
+@pytest.mark.parametrize("pk", [dict(cluster=1), dict(cluster=1, schedule=2, grid=64),
+                                dict(cluster=4, stages=2)],
+                         ids=["cta", "cta-handout", "cluster"])
+def test_a_device_wait_that_runs_out_is_reported(pk):
+    # Every CTA's first copy barrier expects 16 bytes more than its copies
+    # bring, so its bounded wait (2 ms here) runs out while every real copy
+    # still lands: the kernel records ARNQ_ERR_DEVICE_TIMEOUT and the row it
+    # did not finish, waits (bounded) for its copies, and returns.  The context
+    # stays usable: the next call on the same workspace, re-armed, is exact.
+    w = wl.random_case(600, 4096, seed=77, beta=True, smooth1=True)
+    ws, nb = workspace_for(w.rows, w.n)
+    p = plan(kernel=A.ARNQ_KERNEL_STAGED, wait_limit_us=2000, test_hold_bytes=16, **pk)
+    code, row, ctr = _call_with_plan(w, p, ws, nb)
+    assert code == A.ARNQ_ERR_DEVICE_TIMEOUT
+    assert 0 <= row < w.rows
+    assert not ctr.any()
+    ws.zero_()
+    g, _ = run_gpu(w, plan=plan(kernel=A.ARNQ_KERNEL_STAGED, **pk))
+    compare(g, run_oracle(w), "int8", "after a timeout")
+
+
+def test_hand_out_counters_not_at_zero_are_reported_and_cleared():
+    # A workspace whose counters were not zero-filled: the call hands out rows
+    # from the wrong place, and says so (ARNQ_ERR_WORKSPACE_STATE); it leaves
+    # the counters at zero, so the next call is exact.
+    w = wl.random_case(600, 4096, seed=78, beta=True, smooth1=True)
+    ws, nb = workspace_for(w.rows, w.n)
+    p = plan(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=64)
+    for garbage in (5, -3):
+        ws.zero_()
+        ws[16:20].view(torch.int32).fill_(garbage)
+        code, row, ctr = _call_with_plan(w, p, ws, nb)
+        assert code == A.ARNQ_ERR_WORKSPACE_STATE and row == -1, (garbage, code)
+        assert not ctr.any()
+    ws[:16].zero_()
+    code, _, ctr = _call_with_plan(w, p, ws, nb)
+    assert code == 0 and not ctr.any()
+
+
+# ------------------------------------------------------------------ the INT4 word container
+
+@pytest.mark.parametrize("pk", [dict(), dict(kernel=A.ARNQ_KERNEL_DIRECT),
+                                dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4),
+                                dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=2, units=1)],
+                         ids=["auto", "direct", "staged-cl4", "direct-cl2"])
+@pytest.mark.parametrize("rows,n,dt", [(211, 5120, "fp16"), (37, 1000, "bf16"),
+                                       (9, 8200, "bf16"), (3, 16384, "fp16")])
+def test_int4_word_container(rows, n, dt, pk):
+    # eight codes per 32-bit word: parity with the oracle's word packing, and
+    # the same bytes as the two-per-byte container on the same inputs and plan
+    w = wl.random_case(rows, n, dtype=dt, qdtype="int4_int32", seed=rows + n, beta=True,
+                       smooth1=True, smooth2=True, mask=(True, True))
+    p = plan(**pk) if pk else None
+    g, _ = run_gpu(w, plan=p)
+    o = run_oracle(w)
+    compare(g, o, "int4_int32", "word container")
+    w4 = wl.Workload(**{**w.__dict__, "qdtype": "int4"})
+    g4, _ = run_gpu(w4, plan=p)
+    for k in ("y1", "y2", "scale1", "scale2"):
+        assert np.array_equal(g[k].view(np.uint8), g4[k].view(np.uint8)), k
+
+
+def test_int4_word_container_no_add_and_alignment():
+    w = wl.random_case(64, 2048, seed=31, qdtype="int4_int32", beta=True, smooth1=True)
+    x = dev_bits(w.x1, "bf16")
+    y = torch.empty(w.rows * w.n // 8, dtype=torch.int32, device="cuda")
+    sc = torch.empty(w.rows, dtype=torch.float32, device="cuda")
+    ws, nb = workspace_for(w.rows, w.n)
+    gm, bt, sm = dev_bits(w.gamma, "bf16"), dev_bits(w.beta, "bf16"), dev_bits(w.smooth1, "bf16")
+    st = A.arnq_rms_norm_dynamic_quant(x, gm, bt, sm, w.rows, w.n, A.ARNQ_BF16, w.eps,
+                                       A.ARNQ_INT4_INT32, y, sc, ws, nb, None)
+    assert st == A.ARNQ_OK
+    torch.cuda.synchronize()
+    o = oracle.rms_norm_dynamic_quant(w.x1, w.gamma, w.beta, w.smooth1, eps=w.eps,
+                                      qdtype="int4_int32")
+    g = {"y1": y.cpu().numpy().reshape(w.rows, -1), "scale1": sc.cpu().numpy(),
+         "y2": np.full((w.rows, w.n // 2), CANARY, np.uint8),
+         "scale2": np.full(w.rows * 4, CANARY, np.uint8).view(np.float32)}
+    compare(g, {"y1": o["y"], "scale1": o["scale"], "y2": None}, "int4_int32", "no-add words",
+            xout=False)
+    # a word output that is not 4-byte aligned is refused before any launch
+    yb = torch.empty(w.rows * w.n // 2 + 2, dtype=torch.uint8, device="cuda")
+    st = A.arnq_rms_norm_dynamic_quant(x, gm, bt, sm, w.rows, w.n, A.ARNQ_BF16, w.eps,
+                                       A.ARNQ_INT4_INT32, yb.data_ptr() + 2, sc, ws, nb, None)
+    assert st == A.ARNQ_ERR_ALIGN

@@ -19,7 +19,7 @@ import torch
 
 import oracle
 from int4_quant_b200 import workloads as wl
-from tests._util import codes, f32_of_fraction, golden, unpack_int4
+from tests._util import codes, f32_of_fraction, golden, unpack_int4, unpack_int4_words
 
 
 def bits(values, dtype="bf16"):
@@ -52,6 +52,10 @@ def test_hand_worked_rows(case):
     if "expect_y1_packed" in case:
         assert r["y1"][0].tolist() == case["expect_y1_packed"]
         assert unpack_int4(r["y1"])[0].tolist() == case["expect_y1_codes"]
+    if "expect_y1_words" in case:
+        assert r["y1"].dtype == np.uint32
+        assert r["y1"][0].tolist() == case["expect_y1_words"]
+        assert unpack_int4_words(r["y1"])[0].tolist() == case["expect_y1_codes"]
     assert r["clamp_hits"] == 0
 
 
@@ -78,6 +82,23 @@ def test_mask_truth_table_drives_the_outputs():
             assert (r["y1"] is not None, r["y2"] is not None) == (y1, y2)
         else:
             assert r["status"] == oracle.ORC_BAD_MASK
+
+
+def test_int4_containers_hold_the_same_codes():
+    # the same row quantized into both INT4 containers: identical codes,
+    # identical scales; the word container needs n % 8 == 0
+    w = wl.random_case(5, 48, seed=9, beta=True, smooth1=True)
+    a = oracle.add_rms_norm_dynamic_quant_v2(w.x1, w.x2, w.gamma, w.beta, w.smooth1, eps=1e-6,
+                                             qdtype="int4")
+    b = oracle.add_rms_norm_dynamic_quant_v2(w.x1, w.x2, w.gamma, w.beta, w.smooth1, eps=1e-6,
+                                             qdtype="int4_int32")
+    assert a["status"] == b["status"] == oracle.ORC_OK
+    assert np.array_equal(a["scale1"], b["scale1"])
+    assert np.array_equal(unpack_int4(a["y1"]), unpack_int4_words(b["y1"]))
+    x = bits(np.ones((2, 12)))
+    r = oracle.add_rms_norm_dynamic_quant_v2(x, x, bits(np.ones(12)), eps=1e-6,
+                                             qdtype="int4_int32")
+    assert r["status"] == oracle.ORC_BAD_SHAPE
 
 
 def test_rejects_empty_and_odd_int4():

@@ -1,9 +1,13 @@
 """The no-allocation entry point arnq_run_static_scratch on a GPU.
 
-Its scratch is a file-scope device array inside the library; this checks that
-two calls in a row each give exactly what arnq_run (caller workspace) gives on
-the same inputs and plan, for INT8 with two outputs and for packed INT4.  The
-file name sorts last so the suite also runs it after every other GPU test.
+It serves callers that cannot allocate device memory at the point of the
+call; its scratch (the status block and the row hand-out counters) is a
+file-scope device array inside the library.  These tests check that two
+calls in a row each give exactly what arnq_run with a caller workspace gives
+on the same inputs and plan: INT8 with two outputs, packed INT4, rows shared
+by a thread-block cluster, and rows handed out through the array's counters.
+The file name sorts last so that a run stopping at the first failure has run
+every other GPU test first; it also passes alone in a fresh process.
 """
 import numpy as np
 import pytest
@@ -47,26 +51,78 @@ def _call(entry, w, ins, out, mask):
     torch.cuda.synchronize()
 
 
-@pytest.mark.parametrize("case", ["int8_two_outputs", "int4_fp16"])
-def test_static_scratch_equals_workspace_entry_on_two_calls(case):
-    if case == "int8_two_outputs":
+def _case(name):
+    if name == "int8_two_outputs":
         w = wl.random_case(300, 4096, seed=41, beta=True, smooth1=True, smooth2=True,
                            mask=(True, True))
-        mask, on2 = A.ARNQ_MASK_Y1 | A.ARNQ_MASK_Y2, True
-    else:
-        w = wl.random_case(257, 5120, dtype="fp16", qdtype="int4", seed=42, beta=True)
-        mask, on2 = A.ARNQ_MASK_ABSENT, False
-    ins = dict(x1=_dev(w.x1, w.dtype), x2=_dev(w.x2, w.dtype), g=_dev(w.gamma, w.dtype),
-               b=_dev(w.beta, w.dtype), s1=_dev(w.smooth1, w.dtype), s2=_dev(w.smooth2, w.dtype))
+        return w, A.ARNQ_MASK_Y1 | A.ARNQ_MASK_Y2, True
+    if name == "int4_fp16":
+        return wl.random_case(257, 5120, dtype="fp16", qdtype="int4", seed=42, beta=True), \
+            A.ARNQ_MASK_ABSENT, False
+    if name == "dual_16384":   # a cluster shares each row
+        w = wl.random_case(16, 16384, seed=43, beta=True, smooth1=True, smooth2=True,
+                           mask=(True, True))
+        return w, A.ARNQ_MASK_Y1 | A.ARNQ_MASK_Y2, True
+    if name.startswith("rows_16384_"):   # cluster plans, one row per cluster
+        rows = int(name.rsplit("_", 1)[1])
+        return wl.random_case(rows, 16384, seed=44 + rows, beta=True, smooth1=True), \
+            A.ARNQ_MASK_ABSENT, False
+    if name == "handout_2048x4096":   # rows handed out through the array's counters
+        return wl.random_case(2048, 4096, seed=45, x_sigma=(1.0, 0.5), beta=True, smooth1=True,
+                              mask=(True, False)), A.ARNQ_MASK_Y1, False
+    raise KeyError(name)
+
+
+def _inputs(w):
+    return dict(x1=_dev(w.x1, w.dtype), x2=_dev(w.x2, w.dtype), g=_dev(w.gamma, w.dtype),
+                b=_dev(w.beta, w.dtype), s1=_dev(w.smooth1, w.dtype), s2=_dev(w.smooth2, w.dtype))
+
+
+def _same(got, ref):
+    for k in ("y1", "s1", "y2", "s2", "xo"):
+        if ref[k] is None:
+            continue
+        assert torch.equal(got[k].view(torch.uint8), ref[k].view(torch.uint8)), k
+
+
+# Each case: the no-allocation entry point, twice in a row, against arnq_run
+# with a caller workspace (same inputs, same plan: identical bits).  The
+# cluster cases run right after a dual-output 16384-column call through the
+# same array, and the hand-out case right after the others, so each starts
+# from whatever the previous calls left in the array.
+CASES = ["int8_two_outputs", "int4_fp16", "dual_16384", "rows_16384_8", "rows_16384_128",
+         "handout_2048x4096"]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_static_scratch_equals_workspace_entry_on_two_calls(case):
+    w, mask, on2 = _case(case)
+    ins = _inputs(w)
     ref = _outputs(w, on2)
     _call("ws", w, ins, ref, mask)
+    if case.startswith("rows_16384_"):
+        # leave a dual-output cluster call's traces in the array first
+        wd, maskd, _ = _case("dual_16384")
+        _call("static", wd, _inputs(wd), _outputs(wd, True), maskd)
     for _ in range(2):  # two calls in a row through the static scratch
         got = _outputs(w, on2)
         _call("static", w, ins, got, mask)
-        for k in ("y1", "s1", "y2", "s2", "xo"):
-            if ref[k] is None:
-                continue
-            assert torch.equal(got[k].view(torch.uint8), ref[k].view(torch.uint8)), k
+        _same(got, ref)
+
+
+def test_static_scratch_sequence_in_one_process():
+    # the whole sequence again, back to back, with no test in between
+    results = {}
+    for case in CASES:
+        w, mask, on2 = _case(case)
+        ins = _inputs(w)
+        ref = _outputs(w, on2)
+        _call("ws", w, ins, ref, mask)
+        got = _outputs(w, on2)
+        _call("static", w, ins, got, mask)
+        _same(got, ref)
+        results[case] = True
+    assert all(results.values())
 
 
 def test_static_scratch_rejects_on_the_host_first():
