@@ -292,6 +292,18 @@ def job_gbs(bytes_per_step, steps, world, total_ms):
     return bytes_per_step * steps * world / (total_ms / 1e3) / 1e9
 
 
+# Device-side delay queued in front of a timed region (clock cycles, about
+# 2 ms at 1.9 GHz): the host enqueues the timed calls while the GPU waits, so
+# the first event does not also time the host's launch of the first calls.
+HOST_AHEAD_CYCLES = 4_000_000
+
+
+def hold_device(torch):
+    """Queues HOST_AHEAD_CYCLES of device-side delay on the current stream
+    (a torch kernel outside the timed region: it runs before the first event)."""
+    torch.cuda._sleep(HOST_AHEAD_CYCLES)
+
+
 def outputs_of(w):
     """(y1 produced, y2 produced) for a workload, by the outputMask rules."""
     on1 = w.mask is None or w.mask[0]
@@ -395,6 +407,7 @@ class DeviceRun:
         torch.cuda.synchronize(self.dev)
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
+        hold_device(torch)
         e0.record(self.stream)
         for i in range(steps):
             self.launch(i)
@@ -471,6 +484,8 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the other workloads' lines (the `workloads` object)")
     ap.add_argument("--sets", type=int, default=3, help="rotated buffer sets")
+    ap.add_argument("--repeats", type=int, default=5,
+                    help="further timed regions of K steps after the first (spread only)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -523,6 +538,7 @@ def main():
     clocks = ClockSampler(local, period=0.0005)
     clocks.start()
     barrier()
+    hold_device(torch)
     ev0.record(stream)
     for i in range(K):
         run.launch(i)
@@ -530,6 +546,21 @@ def main():
     barrier()
     clocks.stop()
     total_ms = ev0.elapsed_time(ev1)
+    # the same K steps timed again (spread of the figure; `value` is the first)
+    repeats = []
+    for _ in range(args.repeats):
+        for i in range(args.warmup):
+            run.launch(i)
+        barrier()
+        r0 = torch.cuda.Event(enable_timing=True)
+        r1 = torch.cuda.Event(enable_timing=True)
+        hold_device(torch)
+        r0.record(stream)
+        for i in range(K):
+            run.launch(i)
+        r1.record(stream)
+        barrier()
+        repeats.append(r0.elapsed_time(r1) / K)
     run.check_status()
     local_ms = total_ms
     total_ms = max_over_ranks(total_ms, dist, dev)
@@ -599,10 +630,20 @@ def main():
             if name == args.workload:
                 continue
             wr = DeviceRun(wl.CONFIGS[name](), dev, stream, nsets=3)
-            ms = wr.timed(steps=200, warmup=20)
+            ck = ClockSampler(local, period=0.002)
+            ck.start()
+            regions = [wr.timed(steps=200, warmup=20) for _ in range(5)]
+            ck.stop()
             wr.check_status()
-            workloads[name] = workload_entry(wr, ms, peak, "200 calls back to back, 3 sets")
-            workloads[name]["workload"] = wr.w.name
+            ms = statistics.median(regions)
+            e = workload_entry(wr, ms, peak, "200 calls back to back, 3 sets; median of 5 "
+                                             "timed regions")
+            e["us_per_call_min_max"] = [min(regions) * 1e3, max(regions) * 1e3]
+            e["clocks"] = ck.summary()
+            if e["clocks"]["sm_mhz"]:
+                e["us_x_ghz"] = ms * e["clocks"]["sm_mhz"]  # ms * MHz = us * GHz
+            e["workload"] = wr.w.name
+            workloads[name] = e
             del wr
             torch.cuda.empty_cache()
         for name in SMALL:
@@ -645,6 +686,9 @@ def main():
         "steps": K,
         "warmup": args.warmup,
         "ms_per_step": total_ms / K,
+        "ms_per_step_repeats": ({"median": statistics.median(repeats), "min": min(repeats),
+                                 "max": max(repeats), "regions": len(repeats),
+                                 "rank": "this rank (rank 0)"} if repeats else None),
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
@@ -656,6 +700,8 @@ def main():
             "smooth1": w.smooth1 is not None, "smooth2": w.smooth2 is not None, "eps": w.eps,
             "l2": f"{args.sets} rotated buffer sets, inputs {2 * w.rows * w.n * 2 / 1e6:.0f} MB "
                   f"per set (> 126 MB L2)",
+            "timing": f"CUDA events around the K calls, queued behind a "
+                      f"{HOST_AHEAD_CYCLES}-cycle device delay outside the timed region",
             "plan": headline_plan,
             "parallelism": f"replicas x{world} (rows independent; no collective)",
         },
@@ -670,8 +716,8 @@ def main():
             "frac": achieved / peak,
             "traffic": recorded_traffic(w.name, headline_plan),
             "peak_kind": peak_kind,
-            "kernel": "arnq::rows_kernel (one launch per arnq_run call; rows settled in the "
-                      "kernel, one row behind)",
+            "kernel": "arnq::rows_kernel (one launch per arnq_run call; each CTA settles "
+                      "its rows from their records after its last row)",
             "mean_call_us": mean_launch_ms * 1e3,
             "launches_per_call": launches_per_call(plan),
         },

@@ -227,10 +227,11 @@ typedef struct arnq_plan {
                             than its copies bring, so that wait runs out and
                             the call records ARNQ_ERR_DEVICE_TIMEOUT; at most
                             65536; 0 in normal use                           */
-  int32_t schedule;      /* 1: rows dealt out to CTAs in turn; 2: the last
-                            quarter of the rows handed out one at a time to
-                            whichever CTA is free (staged kernel, one CTA per
-                            row, at least two rows per CTA); 0 = choose      */
+  int32_t schedule;      /* 1: rows dealt out to CTAs in turn (the default);
+                            2: the last quarter of the rows handed out one at
+                            a time, by counters in the workspace, to whichever
+                            CTA is free (staged kernel, one CTA per row, at
+                            least two rows per CTA); 0 = choose (1)          */
 } arnq_plan;
 
 /* Fills *plan with the plan arnq_run would use for these arguments (pointers

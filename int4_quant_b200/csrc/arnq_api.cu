@@ -221,7 +221,7 @@ bool vector_ok(const Problem &P) {
 struct Launch {
   KernelFn fn;
   int smem, seg, units;
-  int rec_bytes;     // bytes of one row record (three live in shared memory)
+  int tail_rows, trec_bytes;  // row records per CTA (cluster) and their bytes
   int64_t dyn_base;  // first row handed out by the workspace counter (rows: none)
 };
 
@@ -230,12 +230,12 @@ int upt_candidate(int mode, int i) {
   return mode == arnq::LOAD_SCALAR ? sca[i] : vec[i];
 }
 
-// Shared memory of one CTA: the exchange slots, three row records, B_k of
-// 16-byte units, then (staged) the input ring.
+// Shared memory of one CTA: the exchange slots, `tail_rows` row records,
+// B_k of 16-byte units, then (staged) the input ring.
 int smem_bytes(int mode, int upt, int cl, int threads, int nout, int stages, int stage_bytes,
-               int rec_bytes) {
+               int tail_rows, int trec_bytes) {
   const arnq::Layout lay = arnq::make_layout(
-      cl * (threads / 32), nout, stages, rec_bytes,
+      cl * (threads / 32), nout, stages, tail_rows, trec_bytes,
       arnq::bsm_bytes_for(mode != arnq::LOAD_SCALAR, nout, upt, threads));
   return lay.ring + stages * stage_bytes;
 }
@@ -307,7 +307,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   const int seg = static_cast<int>(ceil_div(units, cl));
   if (seg > max_seg) return ARNQ_ERR_PLAN;
   const int stage_bytes = nin * seg * 16;
-  const int rec = arnq::rec_slot_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
+  const int trec = arnq::tail_rec_bytes(arnq::tie_cap(static_cast<int>(P.n), nout));
 
   // units per thread: of the variants whose threads hold a slice, the one with
   // the most CTAs (rows in flight) per SM, then the most units per thread
@@ -323,7 +323,7 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       KernelFn f = lookup(P.dt, P.qdt, nout, P.add, mode, c, cl);
       if (!f) continue;
       const int sm = smem_bytes(mode, c, cl, t, nout, mode == arnq::LOAD_STAGED ? 1 : 0,
-                                stage_bytes, rec);
+                                stage_bytes, 1, trec);
       if (sm > di.smem_per_block_optin) continue;
       st = prepare_kernel(f, dev, sm);
       if (st != ARNQ_OK) return st;
@@ -353,23 +353,28 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   if (!fn) return ARNQ_ERR_PLAN;
   const int upt = pl->units;
 
-  // Resident clusters (CTAs when cl == 1) and the grid for a ring depth
-  // `stages`: every resident slot gets a cluster (more rows in flight beat
+  // Resident clusters (CTAs when cl == 1), grid and records per cluster for a
+  // ring depth `stages`.  A cluster keeps one record per row it processes in
+  // its first CTA's shared memory, so shared memory grows with the rows per
+  // cluster.  Every resident slot gets a cluster (more rows in flight beat
   // equal row counts: on 8192 x 4096, 740 CTAs took 44.3 us a call, the 683
-  // that give every CTA 12 rows 46.2 us), no more clusters than rows.  A
-  // requested grid is kept.
+  // that give every CTA 12 rows 46.2 us), no more clusters than rows; while
+  // the records do not fit, fewer clusters per SM with more rows each; when
+  // not even one cluster can hold its rows' records, a grid run in waves with
+  // fewer rows per cluster.  A requested grid is kept.  With the counter
+  // hand-out (schedule 2) a CTA keeps two records more than its share: the
+  // rows handed out at the end go to whichever CTA is free.
   struct Eval {
-    int per_sm = 0, smem = 0;
+    int per_sm = 0, smem = 0, tail_rows = 0;
     int64_t nclusters = 0;
   };
-  auto evaluate = [&](int stages, Eval *e) -> arnq_status {
-    *e = Eval();
-    const int sm = smem_bytes(mode, upt, cl, pl->threads, nout, stages, stage_bytes, rec);
-    if (sm > di.smem_per_block_optin) return ARNQ_OK;
+  const int spare = (pl->schedule == 2 && cl == 1 && mode == arnq::LOAD_STAGED) ? 2 : 0;
+  // clusters resident at once with `sm` bytes of shared memory per CTA
+  auto resident = [&](int sm, int *per_sm, int64_t *slots) -> arnq_status {
+    *per_sm = 0;
+    *slots = 0;
     arnq_status s2 = prepare_kernel(fn, dev, sm);
     if (s2 != ARNQ_OK) return s2;
-    int64_t slots = 0;
-    int per_sm = 0;
     if (cl > 1) {
       cudaLaunchConfig_t cfg = {};
       cudaLaunchAttribute attr[1];
@@ -388,26 +393,76 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
       int64_t want =
           pl->ctas_per_sm != 0 ? static_cast<int64_t>(pl->ctas_per_sm) * di.sms / cl : nc;
       if (want < 1) want = 1;
-      slots = want < nc ? want : nc;
-      per_sm = static_cast<int>(ceil_div(slots * cl, di.sms));
-    } else {
-      s2 = occupancy(fn, pl->threads, sm, &per_sm);
-      if (s2 != ARNQ_OK) return s2;
-      if (per_sm < 1) return ARNQ_OK;
-      if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < per_sm) per_sm = pl->ctas_per_sm;
-      slots = static_cast<int64_t>(per_sm) * di.sms;
+      *slots = want < nc ? want : nc;
+      *per_sm = static_cast<int>(ceil_div(*slots * cl, di.sms));
+      return ARNQ_OK;
     }
-    int64_t nclusters;
-    if (pl->grid != 0) {
-      if (pl->grid % cl != 0) return ARNQ_ERR_PLAN;
-      nclusters = pl->grid / cl;
-    } else {
-      nclusters = P.rows < slots ? P.rows : slots;
-    }
-    e->per_sm = per_sm;
-    e->nclusters = nclusters;
-    e->smem = sm;
+    int ps = 0;
+    s2 = occupancy(fn, pl->threads, sm, &ps);
+    if (s2 != ARNQ_OK) return s2;
+    if (ps < 1) return ARNQ_OK;
+    if (pl->ctas_per_sm != 0 && pl->ctas_per_sm < ps) ps = pl->ctas_per_sm;
+    *per_sm = ps;
+    *slots = static_cast<int64_t>(ps) * di.sms;
     return ARNQ_OK;
+  };
+  // shared memory of a CTA holding `nrec` records; false if beyond the limit
+  auto smem_for = [&](int stages, int64_t nrec, int *sm) -> bool {
+    if (nrec * static_cast<int64_t>(trec) > di.smem_per_block_optin) return false;
+    *sm = smem_bytes(mode, upt, cl, pl->threads, nout, stages, stage_bytes,
+                     static_cast<int>(nrec), trec);
+    return *sm <= di.smem_per_block_optin;
+  };
+  auto evaluate = [&](int stages, Eval *e) -> arnq_status {
+    *e = Eval();
+    int sm = 0, per_sm = 0;
+    int64_t slots = 0;
+    if (!smem_for(stages, 1 + spare, &sm)) return ARNQ_OK;
+    arnq_status s2 = resident(sm, &per_sm, &slots);
+    if (s2 != ARNQ_OK) return s2;
+    if (slots < 1) return ARNQ_OK;
+    const bool fixed = pl->grid != 0;
+    if (fixed && pl->grid % cl != 0) return ARNQ_ERR_PLAN;
+    int64_t ncl = fixed ? pl->grid / cl : (P.rows < slots ? P.rows : slots);
+    for (int iter = 0; iter < 32; ++iter) {  // ncl only decreases
+      const int64_t nrec = ceil_div(P.rows, ncl) + spare;
+      int fps = 0;
+      int64_t fit = 0;
+      if (smem_for(stages, nrec, &sm)) {
+        s2 = resident(sm, &fps, &fit);
+        if (s2 != ARNQ_OK) return s2;
+      }
+      if (fit >= 1 && (fixed || fit >= ncl)) {
+        e->per_sm = fps;
+        e->nclusters = ncl;
+        e->tail_rows = static_cast<int>(nrec);
+        e->smem = sm;
+        return ARNQ_OK;
+      }
+      if (fixed || fit < 1) break;
+      ncl = fit;  // fewer clusters, more rows (records) each
+    }
+    if (fixed) return ARNQ_OK;
+    // not even one resident cluster holds its rows' records: fewer rows per
+    // cluster, a grid run in waves
+    int64_t rows_per = ceil_div(P.rows, slots);
+    while (true) {
+      int fps = 0;
+      int64_t fit = 0;
+      if (smem_for(stages, rows_per + spare, &sm)) {
+        s2 = resident(sm, &fps, &fit);
+        if (s2 != ARNQ_OK) return s2;
+      }
+      if (fit >= 1) {
+        e->per_sm = fps;
+        e->nclusters = ceil_div(P.rows, rows_per);
+        e->tail_rows = static_cast<int>(rows_per + spare);
+        e->smem = sm;
+        return ARNQ_OK;
+      }
+      if (rows_per == 1) return ARNQ_OK;
+      rows_per = ceil_div(rows_per, 2);
+    }
   };
 
   Eval best;
@@ -441,17 +496,22 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   const int64_t nclusters = best.nclusters;
   const int smem = best.smem;
   pl->grid = static_cast<int32_t>(nclusters * cl);
-  L->rec_bytes = rec;
-  // Row hand-out (staged kernel, one CTA per row, at least two rows per CTA):
-  // the first three quarters of each CTA's share dealt out in turn, the rest
-  // handed out by the workspace counter as CTAs become free (CTAs of one call
-  // run at different speeds: on 8192 x 4096, CTAs with the same eleven rows
-  // ended their loops anywhere from 32 to 40 us).
+  L->tail_rows = best.tail_rows;
+  L->trec_bytes = trec;
+  // Row hand-out.  Schedule 1 (the default): rows dealt out in turn.
+  // Schedule 2 (staged kernel, one CTA per row, at least two rows per CTA, on
+  // request): the first three quarters of each CTA's share dealt out in turn,
+  // the rest handed out by the workspace counter as CTAs become free.  The
+  // counter evens out the CTAs' loop ends, but then every CTA settles its
+  // records at the same time, with HBM idle; dealt out in turn, the CTAs that
+  // finish first settle while the others still stream, and on B200 that was
+  // faster on 8192 x 4096, 2048 x 16384 and 4096 x 7168 (and even on
+  // 16384 x 5120).
   L->dyn_base = P.rows;
   const bool can_dyn = mode == arnq::LOAD_STAGED && cl == 1 && P.rows >= 2 * nclusters &&
                        P.rows < (int64_t(1) << 30);
   if (pl->schedule == 2 && !can_dyn) return ARNQ_ERR_PLAN;
-  if (pl->schedule == 0) pl->schedule = can_dyn ? 2 : 1;
+  if (pl->schedule == 0) pl->schedule = 1;
   if (pl->schedule == 2) {
     int64_t per = 3 * P.rows / (4 * nclusters);
     if (per < 1) per = 1;
@@ -465,12 +525,13 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
 }
 
 // Plans depend on the device, the shape, the dtypes, the outputs, whether the
-// 16-byte path applies and the requested plan fields, not on the pointers:
+// 16-byte path applies, whether xOut is written and the requested plan
+// fields, not on the pointers:
 // cached per key, so that repeated calls skip the occupancy queries.
 struct PlanKey {
   int dev;
   int64_t rows, n;
-  int dt, qdt, nout, add, vec, beta;
+  int dt, qdt, nout, add, vec, beta, xout;
   arnq_plan req;
 };
 struct PlanEntry {
@@ -485,6 +546,17 @@ int g_plan_next = 0;
 
 bool same_key(const PlanKey &a, const PlanKey &b) { return std::memcmp(&a, &b, sizeof a) == 0; }
 
+// The last plan this thread used: a call with the same key (a decode loop
+// calls with one shape over and over) takes it without the lock.  Entries are
+// never invalidated: a plan depends only on its key.
+struct LastPlan {
+  bool used = false;
+  PlanKey key;
+  arnq_plan plan;
+  Launch L;
+};
+thread_local LastPlan t_last;
+
 arnq_status make_plan_cached(const Problem &P, arnq_plan *pl, Launch *L) {
   PlanKey key;
   std::memset(&key, 0, sizeof key);  // padding too: keys compare bytewise
@@ -497,18 +569,32 @@ arnq_status make_plan_cached(const Problem &P, arnq_plan *pl, Launch *L) {
   key.add = P.add ? 1 : 0;
   key.vec = vector_ok(P) ? 1 : 0;
   key.beta = P.beta ? 1 : 0;
+  key.xout = P.x_out ? 1 : 0;  // where the settling reads x back from
   key.req = *pl;
+  if (t_last.used && same_key(t_last.key, key)) {
+    *pl = t_last.plan;
+    *L = t_last.L;
+    return ARNQ_OK;
+  }
+  auto remember = [&]() {
+    t_last.used = true;
+    t_last.key = key;
+    t_last.plan = *pl;
+    t_last.L = *L;
+  };
   {
     std::lock_guard<std::mutex> lock(g_mu);
     for (int i = 0; i < kPlanCache; ++i)
       if (g_plans[i].used && same_key(g_plans[i].key, key)) {
         *pl = g_plans[i].plan;
         *L = g_plans[i].L;
+        remember();
         return ARNQ_OK;
       }
   }
   arnq_status st = make_plan(P, pl, L);
   if (st != ARNQ_OK) return st;
+  remember();
   std::lock_guard<std::mutex> lock(g_mu);
   PlanEntry &e = g_plans[g_plan_next];
   g_plan_next = (g_plan_next + 1) % kPlanCache;
@@ -547,7 +633,8 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   k.status = static_cast<int32_t *>(workspace);
   k.sched = static_cast<int32_t *>(workspace) + 4;
   k.tie_cap = arnq::tie_cap(static_cast<int>(P.n), (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0));
-  k.rec_bytes = L.rec_bytes;
+  k.tail_rows = L.tail_rows;
+  k.trec_bytes = L.trec_bytes;
   k.dyn_base = L.dyn_base;
   k.rows = P.rows;
   k.n = static_cast<int32_t>(P.n);

@@ -16,42 +16,36 @@
 // parameters G_k in registers (B_k of 16-byte units in shared memory, read
 // back by the thread that wrote it).  Persistent grid: a CTA takes rows c,
 // c + G, ... and then (staged kernel, one CTA per row) rows handed out one at
-// a time by a counter in the workspace.  Three barriers per row: after the
-// sum of squares, after the binary32 row maxima and after the exact row
-// maxima.  The kernel is launched as a programmatic dependent (it waits for
-// the preceding work before touching memory, and lets the next kernel start
-// its set-up after its last row).
+// a time by a counter in the workspace.  Two barriers per row: after the sum
+// of squares and after the row maximum.  The kernel is launched as a
+// programmatic dependent (it waits for the preceding work before touching
+// memory, and lets the next kernel start its set-up after its last row).
 //
-// The result is what an fp64 evaluation of the definition gives, with the
-// scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
-// code = RNE(input_k / scale_k).  Per row:
+// Arithmetic of the fast path, binary32 two lanes at a time with the sm_100
+// packed instructions (add/mul/fma.rn.f32x2):
 //   x = RN16(x1 + x2)            add.rn.{bf16,f16}x2 -- the correctly rounded
-//                                sum, which equals rounding the binary32 sum;
-//                                written as xOut and kept in registers
+//                                sum, which equals rounding the binary32 sum
 //   ss = sum x^2                 fp64 (each x^2 is exact)
 //   1/Rms                        binary32 from ss (within a few ulp)
-//   input_k = x*rinv*G_k + B_k   binary32, packed f32x2 (add/mul/fma.rn.f32x2);
-//                                G_k = gamma*smooth_k, B_k = beta*smooth_k,
-//                                exact products of two 16-bit values
-//   max_k                        binary32 row maximum, then exact: the threads
-//                                holding a candidate unit (an element within
-//                                the binary32 error bound of that maximum; the
-//                                true maximum is among them) evaluate its
-//                                elements in fp64, and the fp64 maxima meet
-//                                at the third barrier
-//   scale_k = RN32(max_k / Q)    exact
-//   code = RNE(input_k * RN32(1/scale_k))  binary32, rounded half to even by
-//                                adding 1.5*2^23; a code whose quotient lies
-//                                within tau of a half-way point (tau bounds the
-//                                binary32 error) is recomputed by its thread in
-//                                fp64 as input_k / scale_k (about 1e-3 of the
-//                                codes)
-// The fp64 inputs use 1/Rms from Newton steps (a few fp64 ulp): the decisions
-// they settle sit many orders of magnitude above fp64 rounding.  A row whose
-// ss/n + eps leaves the normal binary32 range is computed whole in fp64, in
-// the definition's order with IEEE divisions; one whose 1/scale is not a
-// normal binary32 number gets all its codes in fp64.  Every thread handles
-// its own elements: no global memory is read twice.
+//   input_k = x*rinv*G_k + B_k   G_k = gamma*smooth_k, B_k = beta*smooth_k, exact
+//                                products of two 16-bit values
+//   s~_k = max|input_k| / Q      approximate scale
+//   code = RNE(input_k / s~_k)   rounded half-to-even by adding 1.5*2^23
+// The result must be what an fp64 evaluation of the definition gives, with the
+// scale rounded to binary32: scale_k = RN32(max|input_k| / Q) and
+// code = RNE(input_k / scale_k).  The fast path writes its codes and, for
+// each row, a record of the few units it cannot settle (candidates for the
+// row maximum, codes near a half-way point; see the records below).  After
+// its last row the CTA (the cluster's first CTA) settles its rows from the
+// records: the exact scale RN32(max fp64 |input| over the candidates / Q),
+// then the near-tie codes, decided exactly from fp64 inputs (code_exact).
+// The records hold unit indices only; the settling reads those units' x back
+// from xOut (or the inputs) and the parameters from memory.  The fp64 inputs
+// use 1/Rms from Newton steps (a few fp64 ulp): the decisions they settle sit
+// many orders of magnitude above fp64 rounding.  A row whose record overflows
+// (many equal maxima, many exact ties) or whose sum of squares or scale leaves
+// the normal binary32 range is recomputed whole by its lanes, in fp64 with
+// IEEE divisions in the definition's order.
 // Nothing here is a contraction: no tensor cores.
 #pragma once
 
@@ -90,45 +84,44 @@ constexpr int kStatusBytes = 256;
 // Row records.  The binary32 fast path leaves a few units (8 or 2 elements)
 // per row that it cannot settle: candidate units, holding an element within
 // the binary32 error bound of the row maximum (the true maximum is among
-// them), and near-tie units, holding a code whose binary32 quotient lies
-// within tau of a half-way point.  The thread that holds such a unit appends
-// it to the row's record together with the unit's G_k and B_k; one row later
-// one warp (the settling warp) copies the recorded units' x from xOut (or
-// x1, x2) into the record with cp.async, and one row later again settles the
-// row from the record alone: the exact scale RN32(max fp64 |input| over the
-// candidates / Q), then the near-tie codes in fp64 -- with no load on its
-// critical path.  Three records live in the shared memory of the row's CTA
-// (of the cluster's first CTA): the row being processed, the one whose x is
-// on its way, and the one being settled.
-//   header (32 B): double ss; int cnt[2] (candidate, near-tie entries); int flags
-//   ue  [cap] ints: unit | output << 31, candidates first (cap = kCandCap + tie_cap)
-//   ent [cap][24] 32-bit words: x (16 bytes: eight 16-bit values, or x1 then
-//       x2 when xOut is not written; 32 bytes reserved), G_k (8 floats), B_k
-//       (8 floats); pair units (2 elements) use the first words of each part
-// A row whose near-tie list overflows (many exact ties) or whose arithmetic
-// leaves the normal binary32 range is recomputed whole, in fp64.
-constexpr int kCandCap = 4;
+// them), and near-tie units, holding a code whose binary32 quotient t lies
+// within tau of a half-way point (|t - t_exact| <= tau covers the binary32
+// error and the distance between s~ and the exact scale).  Each CTA (each
+// cluster: in its first CTA) keeps one record per row it processes in its
+// shared memory and settles them all after its last row, reading x back from
+// xOut (or the inputs) and the parameters from memory.  Record:
+//   header (32 B): double ss; int cnt[2] (candidate, near-tie units); int flags;
+//       int pad; int64 row
+//   ue [cap] ints: unit | output << 31, candidates first (cap = kCandCap + tie_cap)
+// (a record holds indices only: the records of a CTA's rows share the SM's
+// shared memory with the staging ring and B_k, and larger ones cost CTAs)
+// A near tie needs |t - RNE(t)| > 0.5 - tau, about 2 tau ~ 1e-3 of the codes
+// or fewer; tie_cap leaves several times that for a row of n columns and nout
+// outputs, so rows overflow (and go to the slow path) only by design: many
+// exact ties.
+constexpr int kCandCap = 4;     // candidate units per row
 __host__ __device__ inline int tie_cap(int n, int nout) { return 12 + (n * nout + 255) / 256; }
-struct RecHead {
+struct TailHead {
   double ss;
   int cnt[2];
   int flags;
-  int pad[3];
+  int pad;
+  int64_t row;
 };
-__host__ __device__ inline int rec_ue_bytes(int tcap) { return ((kCandCap + tcap) * 4 + 15) & ~15; }
-__host__ __device__ inline int rec_slot_bytes(int tcap) {
-  return static_cast<int>(sizeof(RecHead)) + rec_ue_bytes(tcap) + (kCandCap + tcap) * 96;
+// bytes of one record (a multiple of 16: the header's double stays aligned)
+__host__ __device__ inline int tail_rec_bytes(int tcap) {
+  return static_cast<int>(sizeof(TailHead)) + (((kCandCap + tcap) * 4 + 15) & ~15);
 }
 
 // Shared-memory layout, sized by the launch (the host computes the same):
-//   ss    [nslots] doubles: per-warp partial sums (also the exact path's reductions)
+//   ss    [nslots] doubles: per-warp partial sums
 //   wmax  [NOUT][nslots] floats: per-warp binary32 row maxima of |input_k|
 //   maxb  [NOUT][nslots] floats: set-up reduction of the bound on |B_k|
 //   flags [2] ints: RF_* of a row, by row parity
 //   bars  [stages] mbarriers
-//   recs  [3] row records of rec_bytes each (used in the cluster's first CTA)
 //   srow  [stages] int64: staged kernel, the row each stage holds (-1: none)
-//   take  16 bytes: the copy-issuing thread's row hand-out state (TakeState)
+//   take  32 bytes: the copy-issuing thread's row hand-out state (TakeState)
+//   trec  [tail_rows] row records of trec_bytes each (used in the cluster's first CTA)
 //   bsm   16-byte units: B_k = beta * smooth_k of every thread's units,
 //         [NOUT][UPT][2][threads] float4 (bsm_bytes_for)
 //   ring  [stages] rows of staged input
@@ -140,15 +133,18 @@ __host__ __device__ inline int bsm_bytes_for(bool vector_units, int nout, int up
   return vector_units ? nout * upt * threads * 32 : 0;
 }
 struct Layout {
-  int ss, wmax, maxb, flags, bars, srow, take, recs, bsm, ring;
+  int ss, wmax, maxb, flags, bars, srow, take, trec, bsm, ring;
 };
 struct TakeState {
   int64_t nxt;   // next row dealt out in turn
+  int64_t pend;  // the row of the next refill, taken before it is due
   int ndyn;      // rows taken from the counter
   int dry;       // the counter ran out: take nothing more
+  int taken;     // rows taken (at most tail_rows: one record each)
+  int pad;
 };
-__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int rec_bytes,
-                                              int bsm_bytes) {
+__host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int tail_rows,
+                                              int trec_bytes, int bsm_bytes) {
   Layout L;
   int off = 0;
   L.ss = off;    off += nslots * 8;
@@ -159,9 +155,9 @@ __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, 
   off = (off + 7) & ~7;
   L.bars = off;  off += stages * 8;
   L.srow = off;  off += stages * 8;
-  L.take = off;  off += 16;
+  L.take = off;  off += 32;
   off = (off + 15) & ~15;
-  L.recs = off;  off += 3 * rec_bytes;
+  L.trec = off;  off += tail_rows * trec_bytes;
   off = (off + 15) & ~15;
   L.bsm = off;   off += bsm_bytes;
   L.ring = (off + 127) & ~127;
@@ -179,14 +175,15 @@ struct KParams {
                               // (all zero between calls)
   int64_t dyn_base;           // staged, one CTA per row: rows from here on are handed
                               // out by the counter (rows = none)
+  int32_t tie_cap;            // near-tie units a record holds
   int64_t rows;
   int32_t n;                  // row length in elements
   int32_t units;              // units per row: ceil(n / U)
   int32_t seg_units;          // units per CTA of a cluster
   int32_t flags;
   int32_t stages;             // staged kernel: ring depth
-  int32_t tie_cap;            // near-tie entries a record holds
-  int32_t rec_bytes;          // bytes of one record (rec_slot_bytes)
+  int32_t tail_rows;          // records per CTA (cluster): rows it processes, at most
+  int32_t trec_bytes;         // bytes per record (tail_rec_bytes)
   float eps;
   double inv_n;               // 1 / n
   uint64_t wait_limit_ns;     // bounded waits give up after this long
@@ -307,20 +304,6 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
       : "memory");
 }
 
-// 16-byte copy global -> shared (cp.async, through L2 only); completes for
-// the issuing thread at cp.async.wait_group
-__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_addr(dst)), "l"(src)
-               : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-  asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-
 // L2 policy of the staged input copies: normal eviction (measured faster than
 // evict-first on the 8192 x 4096 workload, where x1, x2 and the outputs
 // together exceed L2).
@@ -348,6 +331,16 @@ __device__ __forceinline__ double warp_sum_d(double v) {
 __device__ __forceinline__ double warp_max_d(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+// sum / max over an aligned group of `width` lanes (a power of two up to 32;
+// mask: the group's lanes)
+__device__ __forceinline__ double group_sum_d(double v, unsigned mask, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(mask, v, o, width));
+  return v;
+}
+__device__ __forceinline__ double group_max_d(double v, unsigned mask, int width) {
+  for (int o = width >> 1; o > 0; o >>= 1) v = fmax(v, __shfl_xor_sync(mask, v, o, width));
   return v;
 }
 // max over lanes of non-negative floats (their bit patterns order as integers)
@@ -408,14 +401,6 @@ __device__ __forceinline__ double input_of(const KParams &p, int o, int c, float
   return y;
 }
 
-// round_half_even(input / scale) clamped to [-qmax, qmax]; 0 for a zero scale
-__device__ __forceinline__ int code_of(double in, float scale, int qmax) {
-  if (scale == 0.f) return 0;
-  return code_of_t(__ddiv_rn(in, static_cast<double>(scale)), qmax);
-}
-
-// ---------------------------------------------------------------- exact codes
-
 // RNE(in / sc) clamped to [-qmax, qmax], for an fp64 input `in`, a positive
 // normal binary32 scale sc and an approximation t of in / sc that is off by
 // less than 1/2: the only rounding boundary within reach is the half-integer
@@ -435,176 +420,10 @@ __device__ __forceinline__ int code_exact(double in, float sc, float t, int qmax
   return min(max(q, -qmax), qmax);
 }
 
-// ---------------------------------------------------------------- whole rows in fp64
-
-// x of column c of a row, read back from memory: xOut when written, else the
-// inputs (then unchanged: an in-place update always writes xOut).
-template <class T, bool ADD>
-__device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) {
-  using C = Cvt<T>;
-  const int64_t j = row * p.n + c;
-  if (!ADD) return C::f1(p.x1[j]);
-  if (p.flags & F_XOUT) return C::f1(p.x_out[j]);
-  return C::f2(C::add2(p.x1[j], p.x2[j])).x;
-}
-
-// Whole row in fp64, in the definition's order with IEEE divisions, by the 32
-// lanes of a warp, x read back from memory: the slow path for rows the fast
-// path cannot settle (a near-tie list that overflowed, or ss/n + eps or the
-// scale outside the normal binary32 range).  Called, not inlined: rare, and
-// its division sequences would take registers from the row loop.
-template <class T, bool INT4, int NOUT, bool ADD>
-__device__ __noinline__ void exact_row_warp(const KParams &p, int64_t row, int lane) {
-  constexpr int QI = INT4 ? 7 : 127;
-  const int n = p.n;
-  const int64_t base = row * n;
-  double ss = 0.0;
-  for (int c = lane; c < n; c += 32) {
-    const double a = x_reload<T, ADD>(p, row, c);
-    ss = __fma_rn(a, a, ss);
-  }
-  const double rms = rms_of(warp_sum_d(ss), n, p.eps);
-  for (int o = 0; o < NOUT; ++o) {
-    double m = 0.0;
-    for (int c = lane; c < n; c += 32)
-      m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
-    const float sc = __double2float_rn(__ddiv_rn(warp_max_d(m), static_cast<double>(QI)));
-    if (lane == 0) p.scale[o][row] = sc;
-    for (int c = 2 * lane; c < n; c += 64) {  // element pairs: an INT4 byte has one writer
-      const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
-      const int q1 =
-          c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
-                    : 0;
-      if (INT4) {
-        p.y[o][row * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
-      } else {
-        p.y[o][base + c] = static_cast<uint8_t>(q0);
-        if (c + 1 < n) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
-      }
-    }
-  }
-}
-
-// ---------------------------------------------------------------- settling a record
-
-__device__ __forceinline__ int *rec_ue(RecHead *h) { return reinterpret_cast<int *>(h + 1); }
-__device__ __forceinline__ uint32_t *rec_ent(RecHead *h, int tcap, int ent) {
-  return reinterpret_cast<uint32_t *>(reinterpret_cast<unsigned char *>(h + 1) +
-                                      rec_ue_bytes(tcap)) + ent * 24;
-}
-
-// Copies the recorded units' x of row r into the record h (16-byte units:
-// cp.async, one commit group per call, waited for by the same warp at the
-// row's settle).  Rows the slow path takes need nothing.
-template <bool ADD, int U>
-__device__ __forceinline__ void prefetch_record(const KParams &p, RecHead *h, int64_t r, int lane) {
-  if (U == 8) {
-    const int nc = min(h->cnt[0], kCandCap), nt = min(h->cnt[1], p.tie_cap);
-    const int *ue = rec_ue(h);
-    for (int q = lane; q < kCandCap + nt; q += 32) {
-      if (q >= nc && q < kCandCap) continue;
-      const int u = static_cast<int>(static_cast<uint32_t>(ue[q]) & 0x7FFFFFFFu);
-      const int64_t j = r * p.n + static_cast<int64_t>(u) * 8;
-      uint32_t *dst = rec_ent(h, p.tie_cap, q);
-      if (!ADD) {
-        cp_async16(dst, p.x1 + j);
-      } else if (p.flags & F_XOUT) {
-        cp_async16(dst, p.x_out + j);
-      } else {
-        cp_async16(dst, p.x1 + j);
-        cp_async16(dst + 4, p.x2 + j);
-      }
-    }
-  }
-  cp_async_commit();
-}
-
-// Settles row r from its record h (in this CTA's shared memory, or the
-// cluster's first CTA's) with one warp, then clears the record's counters.
-// The record holds every value needed (x copied in by prefetch_record, whose
-// group the caller has waited for; G_k and B_k from the recording threads):
-// the candidates' fp64 maximum gives the exact scale RN32(max / Q); each
-// near-tie unit's codes are then decided exactly from their fp64 inputs
-// (code_exact).  Pair units (U == 2: misaligned or ragged rows) read x from
-// memory here.
-template <class T, bool INT4, int NOUT, bool ADD, int U>
-__device__ __forceinline__ void settle_record(const KParams &p, RecHead *h, int64_t r, int lane) {
-  using C = Cvt<T>;
-  constexpr int QI = INT4 ? 7 : 127;
-  constexpr int PAIRS = U / 2;
-  const int n = p.n;
-  const int nc = h->cnt[0], nt = h->cnt[1];
-  if ((h->flags & RF_REDO) || nc > kCandCap || nt > p.tie_cap) {
-    exact_row_warp<T, INT4, NOUT, ADD>(p, r, lane);
-  } else {
-    const int *ue = rec_ue(h);
-    const double ri = rsqrt64(__fma_rn(h->ss, p.inv_n, static_cast<double>(p.eps)));
-    // fp64 input of element e of entry ent (column c)
-    auto in64 = [&](int ent, int e, int c) -> double {
-      const uint32_t *v = rec_ent(h, p.tie_cap, ent);
-      float x;
-      if (U == 8) {
-        const int wd = e >> 1;
-        const float2 a = C::f2(ADD && !(p.flags & F_XOUT) ? C::add2(v[wd], v[4 + wd]) : v[wd]);
-        x = (e & 1) ? a.y : a.x;
-      } else {
-        x = x_reload<T, ADD>(p, r, c);
-      }
-      return __fma_rn(__dmul_rn(static_cast<double>(x), ri),
-                      static_cast<double>(__uint_as_float(v[8 + e])),
-                      static_cast<double>(__uint_as_float(v[16 + e])));
-    };
-    // exact scales: fp64 maximum over the candidate elements (one a lane)
-    double m0 = 0.0, m1 = 0.0;
-    if (lane < nc * U) {
-      const int ent = lane / U, e = lane % U;
-      const uint32_t hd = static_cast<uint32_t>(ue[ent]);
-      const int c = U * static_cast<int>(hd & 0x7FFFFFFFu) + e;
-      if (c < n) {
-        const double v = fabs(in64(ent, e, c));
-        if ((hd >> 31) == 0) m0 = v; else m1 = v;
-      }
-    }
-    float sc[2], r32[2];
-    sc[0] = __double2float_rn(__dmul_rn(warp_max_d(m0), 1.0 / static_cast<double>(QI)));
-    sc[1] = NOUT == 2 ? __double2float_rn(__dmul_rn(warp_max_d(m1), 1.0 / static_cast<double>(QI)))
-                      : 0.f;
-#pragma unroll
-    for (int o = 0; o < 2; ++o) r32[o] = sc[o] >= 1.1754943508222875e-38f ? __frcp_rn(sc[o]) : 0.f;
-    if (lane == 0) {
-      p.scale[0][r] = sc[0];
-      if (NOUT == 2) p.scale[1][r] = sc[1];
-    }
-    // near-tie codes, one element pair (one INT4 byte) a lane
-    for (int q = lane; q < nt * PAIRS; q += 32) {
-      const int ent = kCandCap + q / PAIRS;
-      const uint32_t hd = static_cast<uint32_t>(ue[ent]);
-      const int o = static_cast<int>(hd >> 31);
-      const int e = 2 * (q % PAIRS);
-      const int c = U * static_cast<int>(hd & 0x7FFFFFFFu) + e;
-      const float so = o ? sc[1] : sc[0], ro = o ? r32[1] : r32[0];
-      int q2[2] = {0, 0};
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        if (so != 0.f && c + h2 < n) {
-          const double v = in64(ent, e + h2, c + h2);
-          q2[h2] = ro != 0.f ? code_exact(v, so, __double2float_rn(v) * ro, QI) : code_of(v, so, QI);
-        }
-      }
-      if (INT4) {
-        p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q2[0] & 0xF) | ((q2[1] & 0xF) << 4));
-      } else {
-        p.y[o][r * n + c] = static_cast<uint8_t>(q2[0]);
-        if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q2[1]);
-      }
-    }
-  }
-  __syncwarp();
-  if (lane == 0) {
-    h->cnt[0] = 0;
-    h->cnt[1] = 0;
-    h->flags = 0;
-  }
+// round_half_even(input / scale) clamped to [-qmax, qmax]; 0 for a zero scale
+__device__ __forceinline__ int code_of(double in, float scale, int qmax) {
+  if (scale == 0.f) return 0;
+  return code_of_t(__ddiv_rn(in, static_cast<double>(scale)), qmax);
 }
 
 // ---------------------------------------------------------------- exchange
@@ -649,6 +468,210 @@ struct Exchange {
   }
 };
 
+// x of column c of a row, read back from memory: xOut when written, else the
+// inputs (then unchanged: an in-place update always writes xOut).
+template <class T, bool ADD>
+__device__ __forceinline__ float x_reload(const KParams &p, int64_t row, int c) {
+  using C = Cvt<T>;
+  const int64_t j = row * p.n + c;
+  if (!ADD) return C::f1(p.x1[j]);
+  if (p.flags & F_XOUT) return C::f1(p.x_out[j]);
+  return C::f2(C::add2(p.x1[j], p.x2[j])).x;
+}
+
+// Whole row in fp64, in the definition's order, by an aligned group of
+// `width` lanes (lane = 0 .. width-1, mask: the group's lanes), x read back
+// from memory: the slow path for rows the fast path cannot settle.
+template <class T, bool INT4, int NOUT, bool ADD>
+__device__ __forceinline__ void exact_row_lanes(const KParams &p, int64_t row, int lane, int width,
+                                                unsigned mask) {
+  constexpr int QI = INT4 ? 7 : 127;
+  const int n = p.n;
+  const int64_t base = row * n;
+  double ss = 0.0;
+  for (int c = lane; c < n; c += width) {
+    const double a = x_reload<T, ADD>(p, row, c);
+    ss = __fma_rn(a, a, ss);
+  }
+  const double rms = rms_of(group_sum_d(ss, mask, width), n, p.eps);
+#pragma unroll
+  for (int o = 0; o < NOUT; ++o) {
+    double m = 0.0;
+    for (int c = lane; c < n; c += width)
+      m = fmax(m, fabs(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms)));
+    const float sc =
+        __double2float_rn(__ddiv_rn(group_max_d(m, mask, width), static_cast<double>(QI)));
+    if (lane == 0) p.scale[o][row] = sc;
+    for (int c = 2 * lane; c < n; c += 2 * width) {  // element pairs: an INT4 byte has one writer
+      const int q0 = code_of(input_of<T>(p, o, c, x_reload<T, ADD>(p, row, c), rms), sc, QI);
+      const int q1 =
+          c + 1 < n ? code_of(input_of<T>(p, o, c + 1, x_reload<T, ADD>(p, row, c + 1), rms), sc, QI)
+                    : 0;
+      if (INT4) {
+        p.y[o][row * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+      } else {
+        p.y[o][base + c] = static_cast<uint8_t>(q0);
+        if (c + 1 < n) p.y[o][base + c + 1] = static_cast<uint8_t>(q1);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- in-kernel settling
+
+// Settles one row from its record with an aligned group of g lanes (lane l of
+// g >= 8, gmask: the group's lanes): the exact scales from the candidate
+// units, then the near-tie units' codes, in fp64 from x read back from memory
+// and the parameters (the same arithmetic as settle_kernel).  The loads of the
+// common case (every candidate element, and each lane's first two element
+// pairs of near-tie units) are issued before any arithmetic.
+template <class T, bool INT4, int NOUT, bool ADD, int U>
+__device__ __forceinline__ void settle_row_group(const KParams &p, int64_t r, double ss, int nc,
+                                                 int nt, const int *ent, int l, int g,
+                                                 unsigned gmask) {
+  using C = Cvt<T>;
+  constexpr int QI = INT4 ? 7 : 127;
+  constexpr int PAIRS = U / 2;           // element pairs per unit
+  constexpr int CE = kCandCap * U / 8;   // candidate elements per lane, at most (g >= 8)
+  const int n = p.n;
+  struct Elem { float x, g, b; };
+  const Elem zero = {0.f, 0.f, 0.f};
+  auto load = [&](int q, int o, int c) -> Elem {
+    (void)q;
+    Elem e;
+    e.x = x_reload<T, ADD>(p, r, c);
+    const float sm = p.smooth[o] ? C::f1(__ldg(p.smooth[o] + c)) : 1.f;
+    e.g = C::f1(__ldg(p.gamma + c)) * sm;  // exact: two 16-bit significands
+    e.b = (p.flags & F_BETA) ? C::f1(__ldg(p.beta + c)) * sm : 0.f;
+    return e;
+  };
+  auto unit_of = [](uint32_t hd) { return static_cast<int>(hd & 0x7FFFFFFFu); };
+  auto out_of = [](uint32_t hd) { return static_cast<int>(hd >> 31); };
+
+  // candidate elements e = l, l + g, ... of the nc * U
+  Elem ce[CE];
+  int co[CE];
+  bool cv[CE];
+#pragma unroll
+  for (int k = 0; k < CE; ++k) {
+    const int e = l + k * g;
+    ce[k] = zero;
+    co[k] = 0;
+    cv[k] = false;
+    if (e < nc * U) {
+      const uint32_t hd = static_cast<uint32_t>(ent[e / U]);
+      const int c = U * unit_of(hd) + e % U;
+      if (c < n) {
+        co[k] = out_of(hd);
+        cv[k] = true;
+        ce[k] = load(e / U, co[k], c);
+      }
+    }
+  }
+  // near-tie element pairs q = l, l + g, ...: the first two now
+  Elem ta[2], tb[2];
+  uint32_t th[2];
+  int tc[2];
+  bool tv[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int q = l + k * g;
+    ta[k] = tb[k] = zero;
+    th[k] = 0u;
+    tc[k] = 0;
+    tv[k] = q < nt * PAIRS;
+    if (tv[k]) {
+      th[k] = static_cast<uint32_t>(ent[kCandCap + q / PAIRS]);
+      tc[k] = U * unit_of(th[k]) + 2 * (q % PAIRS);
+      tv[k] = tc[k] < n;  // (always: a unit of the row)
+    }
+    if (tv[k]) {
+      ta[k] = load(kCandCap + q / PAIRS, out_of(th[k]), tc[k]);
+      if (tc[k] + 1 < n) tb[k] = load(kCandCap + q / PAIRS, out_of(th[k]), tc[k] + 1);
+    }
+  }
+
+  const double ri = rsqrt64(__fma_rn(ss, p.inv_n, static_cast<double>(p.eps)));
+  auto input64 = [&](const Elem &e) -> double {
+    return __fma_rn(__dmul_rn(static_cast<double>(e.x), ri), static_cast<double>(e.g),
+                    static_cast<double>(e.b));
+  };
+  // exact scales: fp64 maximum over the candidate elements
+  double m0 = 0.0, m1 = 0.0;
+#pragma unroll
+  for (int k = 0; k < CE; ++k) {
+    if (cv[k]) {
+      const double v = fabs(input64(ce[k]));
+      if (co[k] == 0) m0 = fmax(m0, v); else m1 = fmax(m1, v);
+    }
+  }
+  const double inv_q = 1.0 / static_cast<double>(QI);
+  float sc[2] = {0.f, 0.f};
+  sc[0] = __double2float_rn(__dmul_rn(group_max_d(m0, gmask, g), inv_q));
+  if (NOUT == 2) sc[1] = __double2float_rn(__dmul_rn(group_max_d(m1, gmask, g), inv_q));
+  if (l == 0) {
+    p.scale[0][r] = sc[0];
+    if (NOUT == 2) p.scale[1][r] = sc[1];
+  }
+  // near-tie codes in fp64, one element pair (one INT4 byte) at a time
+  auto put = [&](uint32_t hd, int c, const Elem &e0, const Elem &e1) {
+    const int o = out_of(hd);
+    const float so = o == 0 ? sc[0] : sc[1];
+    // exact decisions: code_exact with the binary32 quotient as its guide
+    // (a normal scale), else an IEEE division
+    auto code = [&](const Elem &el) -> int {
+      const double v = input64(el);
+      if (so >= 1.1754943508222875e-38f) return code_exact(v, so, __double2float_rn(v) * __frcp_rn(so), QI);
+      return code_of(v, so, QI);
+    };
+    const int q0 = so == 0.f ? 0 : code(e0);
+    const int q1 = (so == 0.f || c + 1 >= n) ? 0 : code(e1);
+    if (INT4) {
+      p.y[o][r * (n / 2) + c / 2] = static_cast<uint8_t>((q0 & 0xF) | ((q1 & 0xF) << 4));
+    } else {
+      p.y[o][r * n + c] = static_cast<uint8_t>(q0);
+      if (c + 1 < n) p.y[o][r * n + c + 1] = static_cast<uint8_t>(q1);
+    }
+  };
+#pragma unroll
+  for (int k = 0; k < 2; ++k)
+    if (tv[k]) put(th[k], tc[k], ta[k], tb[k]);
+  for (int q = l + 2 * g; q < nt * PAIRS; q += g) {  // more than two pairs per lane
+    const uint32_t hd = static_cast<uint32_t>(ent[kCandCap + q / PAIRS]);
+    const int c = U * unit_of(hd) + 2 * (q % PAIRS);
+    if (c >= n) continue;  // (always in the row)
+    const Elem e0 = load(kCandCap + q / PAIRS, out_of(hd), c);
+    const Elem e1 = c + 1 < n ? load(kCandCap + q / PAIRS, out_of(hd), c + 1) : zero;
+    put(hd, c, e0, e1);
+  }
+}
+
+// The CTA (the first CTA of a cluster) settles its rows (records 0 ..
+// nrows-1, each naming its row) from the records in its shared memory, after
+// its last row: a group of lanes per row (32, 16 or 8: as many rows at once as
+// the CTA's threads allow).  Rows whose record overflowed, or that the fast
+// path flagged, are recomputed whole in fp64 by their group.
+template <class T, bool INT4, int NOUT, bool ADD, int U>
+__device__ __forceinline__ void tail_settle(const KParams &p, const unsigned char *trec, int nrows) {
+  const int nthreads = static_cast<int>(blockDim.x);
+  int g = 32;
+  while (g > 8 && nthreads / g < nrows) g >>= 1;
+  const int groups = nthreads / g;
+  const int wl = static_cast<int>(threadIdx.x) & 31;
+  const int l = wl & (g - 1);
+  const unsigned gmask = g == 32 ? 0xFFFFFFFFu : ((1u << g) - 1u) << (wl & ~(g - 1));
+  for (int i = static_cast<int>(threadIdx.x) / g; i < nrows; i += groups) {
+    const TailHead *h = reinterpret_cast<const TailHead *>(trec + static_cast<size_t>(i) * p.trec_bytes);
+    const int *ent = reinterpret_cast<const int *>(h + 1);
+    const int64_t r = h->row;
+    const int nc = h->cnt[0], nt = h->cnt[1];
+    if ((h->flags & RF_REDO) || nc > kCandCap || nt > p.tie_cap)
+      exact_row_lanes<T, INT4, NOUT, ADD>(p, r, l, g, gmask);
+    else
+      settle_row_group<T, INT4, NOUT, ADD, U>(p, r, h->ss, nc, nt, ent, l, g, gmask);
+  }
+}
+
 // ---------------------------------------------------------------- row kernel
 
 // The row kernel's body; the __global__ entry points below differ only in
@@ -689,7 +712,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   extern __shared__ __align__(128) unsigned char smem[];
   // 16-byte units keep B_k in shared memory (registers go to x and G_k)
   constexpr bool BSM = (W == 4);
-  const Layout lay = make_layout(nslots, NOUT, ring_depth, p.rec_bytes,
+  const Layout lay = make_layout(nslots, NOUT, ring_depth, p.tail_rows, p.trec_bytes,
                                  bsm_bytes_for(BSM, NOUT, UPT, static_cast<int>(blockDim.x)));
   float4 *bsm = reinterpret_cast<float4 *>(smem + lay.bsm);
   auto bsm_at = [&](int o, int k, int j) -> float4 & {
@@ -708,8 +731,8 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   // the barriers only after the set-up exchange below.
   // staged: row `row` goes to stage s, x1 then x2; the barrier expects `hold`
   // bytes more than the copies bring (testing only: then the wait runs out)
-  uint64_t policy = 0;
   auto issue = [&](int64_t row, int s, uint32_t hold) {
+    const uint64_t policy = policy_evict_normal();
     const uint32_t bar = smem_addr(&bars[s]);
     const uint32_t dst = smem_addr(ring + static_cast<size_t>(s) * stage_bytes);
     const int64_t off = row * n + static_cast<int64_t>(seg_begin) * 8;
@@ -725,18 +748,25 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   // copies sees them: rows below p.dyn_base are dealt out in turn (c, c + G,
   // ...); the others are handed out one at a time by the workspace counter,
   // so that CTAs that run faster take more of them.  A ticket is fetched one
-  // take ahead: its latency overlaps a row.  -1: no more rows.
-  // The hand-out state lives in shared memory (registers are scarce), all but
-  // the prefetched ticket, whose load is waited for only at the next take.
+  // take ahead: its latency overlaps a row.  -1: no more rows.  The hand-out
+  // state lives in shared memory (registers are scarce), all but the
+  // prefetched ticket, whose load is waited for only at the next take.
   const bool dyn = MODE == LOAD_STAGED && !CL && p.dyn_base < p.rows;
   TakeState *ts = reinterpret_cast<TakeState *>(smem + lay.take);
   int ticket = 0;
+  // A ticket is drawn only while the CTA has a record left for its row: a
+  // ticket drawn and never used would be a row nobody processes.
   auto take = [&]() -> int64_t {
+    if (ts->taken >= p.tail_rows) return -1;  // every record in use
     const int64_t nx = ts->nxt;
     if (nx < p.dyn_base) {
       ts->nxt = nx + nclusters;
-      if (dyn && nx + nclusters >= p.dyn_base) ticket = atomicAdd(p.sched, 1);  // the first ticket
-      return nx < p.rows ? nx : -1;
+      if (nx >= p.rows) return -1;
+      ts->taken += 1;
+      // the first ticket, with the last row dealt out in turn
+      if (dyn && nx + nclusters >= p.dyn_base && ts->taken < p.tail_rows)
+        ticket = atomicAdd(p.sched, 1);
+      return nx;
     }
     if (!dyn || ts->dry) return -1;
     const int64_t r = p.dyn_base + ticket;
@@ -744,15 +774,16 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       ts->dry = 1;
       return -1;
     }
-    ticket = atomicAdd(p.sched, 1);
     ts->ndyn += 1;
+    ts->taken += 1;
+    if (ts->taken < p.tail_rows) ticket = atomicAdd(p.sched, 1);
     return r;
   };
   if (MODE == LOAD_STAGED && tid == 0) {
     ts->nxt = cluster_id;
     ts->ndyn = 0;
     ts->dry = 0;
-    policy = policy_evict_normal();
+    ts->taken = 0;
     for (int s = 0; s < stages; ++s) {
       const int64_t row = take();
       srow[s] = row;
@@ -848,16 +879,19 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     if (lane == 0) ex.publish(maxb_slots, o * nslots + my_slot, v);
   }
   if (tid < 2) rflags[tid] = 0;
-  // the record of row iteration i: slot i % 3, in the shared memory of the
-  // cluster's first CTA
-  unsigned char *const recs = ex.first_cta(smem + lay.recs);
-  auto slot = [&](int64_t i) -> RecHead * {
-    return reinterpret_cast<RecHead *>(recs + static_cast<int>(i % 3) * p.rec_bytes);
+  // the records: one per row this CTA (cluster) processes, in the shared
+  // memory of the cluster's first CTA
+  unsigned char *const trec = ex.first_cta(smem + lay.trec);
+  auto thead = [&](int64_t i) -> TailHead * {
+    return reinterpret_cast<TailHead *>(trec + static_cast<size_t>(i) * p.trec_bytes);
   };
-  if (rank == 0 && tid < 3) {
-    RecHead *h = reinterpret_cast<RecHead *>(smem + lay.recs + tid * p.rec_bytes);
-    h->cnt[0] = h->cnt[1] = 0;
-    h->flags = 0;
+  if (rank == 0) {
+    for (int i = tid; i < p.tail_rows; i += blockDim.x) {
+      TailHead *th = reinterpret_cast<TailHead *>(smem + lay.trec +
+                                                  static_cast<size_t>(i) * p.trec_bytes);
+      th->cnt[0] = th->cnt[1] = 0;
+      th->flags = 0;
+    }
   }
   ex.sync();
   float maxBg[NOUT];  // bound on |B_k| over the whole row
@@ -868,68 +902,19 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     maxBg[o] = warp_max_nonneg(m);
   }
 
-  // the codes of unit u (8 or 2 elements, low bits of bits[]) of row `row`
-  auto store_codes = [&](uint8_t *y, int64_t row, int u, const uint32_t (&bits)[2 * W]) {
-    if (MODE != LOAD_SCALAR) {
-      if (INT4) {  // 8 codes -> 4 bytes, even column in the low nibble
-        uint32_t w = 0;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) w |= (bits[e] & 0xFu) << (4 * e);
-        __stcs(reinterpret_cast<unsigned int *>(y + row * (n / 2) + static_cast<int64_t>(u) * 4),
-               w);
-      } else {     // 8 codes -> 8 bytes
-        const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
-                                        __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
-        const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
-                                        __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
-        __stcs(reinterpret_cast<uint2 *>(y + row * n + static_cast<int64_t>(u) * 8),
-               make_uint2(lo, hi));
-      }
-    } else {
-      if (INT4) {
-        y[row * (n / 2) + u] = static_cast<uint8_t>((bits[0] & 0xFu) | ((bits[1] & 0xFu) << 4));
-      } else {
-        const int64_t j = row * n + 2 * static_cast<int64_t>(u);
-        y[j] = static_cast<uint8_t>(bits[0] & 0xFFu);
-        if (2 * u + 1 < n) y[j + 1] = static_cast<uint8_t>(bits[1] & 0xFFu);
-      }
-    }
-  };
-
-  // ---- row records: unit u of output o on list l (0 candidate, 1 near tie) of
-  // the current row, with its G_k and B_k; an overflowing list only counts,
-  // and the row goes to the slow path
+  // ---- row records: record unit u of output o on list l (0 candidate, 1
+  // near tie) of the current row; an overflowing list only counts, and the
+  // row goes to the slow path.
   int64_t it = 0;          // rows this CTA (cluster) has processed
-  auto record = [&](int l, int u, int o, const float2 (&gk)[W], const float2 (&bk)[W]) {
-    RecHead *h = slot(it);
-    const int k = atomicAdd(&h->cnt[l], 1);
-    if (k >= (l == 0 ? kCandCap : p.tie_cap)) return;
-    const int ent = l == 0 ? k : kCandCap + k;
-    rec_ue(h)[ent] = static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
-    float *v = reinterpret_cast<float *>(rec_ent(h, p.tie_cap, ent));
-    if (W == 4) {
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        reinterpret_cast<float4 *>(v + 8)[j] = make_float4(gk[2 * j].x, gk[2 * j].y,
-                                                           gk[2 * j + 1].x, gk[2 * j + 1].y);
-        reinterpret_cast<float4 *>(v + 16)[j] = make_float4(bk[2 * j].x, bk[2 * j].y,
-                                                            bk[2 * j + 1].x, bk[2 * j + 1].y);
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < W; ++i) {
-        reinterpret_cast<float2 *>(v + 8)[i] = gk[i];
-        reinterpret_cast<float2 *>(v + 16)[i] = bk[i];
-      }
-    }
+  auto record = [&](int l, int u, int o) {
+    TailHead *th = thead(it);
+    const int k = atomicAdd(&th->cnt[l], 1);
+    if (k < (l == 0 ? kCandCap : p.tie_cap))
+      reinterpret_cast<int *>(th + 1)[l == 0 ? k : kCandCap + k] =
+          static_cast<int>(static_cast<uint32_t>(u) | (static_cast<uint32_t>(o) << 31));
   };
-  // the settling warp: the last warp of the cluster's first CTA
-  const bool settler = rank == 0 && warp == nwarps - 1;
-
-  int stage = 0;           // staged: it % stages, kept incrementally
-  uint32_t phase = 0;      // staged: (it / stages) & 1, the mbarrier phase to wait for
-  int64_t prev_row = -1;   // the row of the previous iteration
-  int64_t prev2_row = -1;  // and of the one before
+  int stage = 0;          // staged: it % stages, kept incrementally
+  uint32_t phase = 0;     // staged: (it / stages) & 1, the mbarrier phase to wait for
   for (;; ++it) {
     int64_t row;
     if (MODE == LOAD_STAGED) {
@@ -941,6 +926,12 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     }
     const int par = static_cast<int>(it & 1);
     bool timed_out = false;
+    if (MODE == LOAD_STAGED && tid == 0) {
+      // while this row's data is on its way: the row of this iteration's
+      // refill (issued after the first barrier, when the stage is free), so
+      // that the refill itself is one shared-memory load and the copy
+      ts->pend = take();
+    }
     if (MODE == LOAD_STAGED && seg_len > 0) {
       timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), phase, p.wait_limit_ns);
     }
@@ -1038,7 +1029,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       }
       // every thread has read this stage (and its row): refill it
       if (tid == 0) {
-        const int64_t nrow = take();
+        const int64_t nrow = ts->pend;
         srow[stage] = nrow;
         if (nrow >= 0 && seg_len > 0) issue(nrow, stage, 0u);
       }
@@ -1051,7 +1042,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       for (int i = lane; i < nslots; i += 32) ss_row = __dadd_rn(ss_row, ss_slots[i]);
       ss_row = warp_sum_d(ss_row);
     }
-    // v = ss/n + eps; 1/sqrt(v) in binary32 for the bulk
+    // v = ss/n + eps; 1/sqrt(v) in binary32 for the bulk, in fp64 when needed
     const double v64 = __fma_rn(ss_row, p.inv_n, static_cast<double>(p.eps));
     const float v32 = __double2float_rn(v64);
     float2 rinv2;
@@ -1059,12 +1050,13 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       const float r = rsqrt_refined(v32);
       rinv2 = make_float2(r, r);
     }
-    // the record: this row's sum of squares and flags (outside the normal
-    // binary32 range the bulk arithmetic is not trusted: the slow path)
+    // the record: this row, its sum of squares and flags (outside the normal
+    // binary32 range the bulk arithmetic is not trusted)
     if (tid == 0 && rank == 0) {
-      RecHead *h = slot(it);
-      h->ss = ss_row;
-      h->flags = (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
+      TailHead *th = thead(it);
+      th->row = row;
+      th->ss = ss_row;
+      th->flags = (v32 >= 1.1754943508222875e-38f && v32 <= 3.4028234663852886e+38f) ? 0 : RF_REDO;
     }
 
     // ---- pass 2: binary32 maxima of |input_k|, per unit and over the row
@@ -1094,8 +1086,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     if (tid == 0) rflags[par ^ 1] = 0;
 
     // ---- pass 3: quantize with the approximate scale s~ = max / Q (rounded half
-    // to even via the 1.5*2^23 trick); record the candidate units and the
-    // units with a code near a half-way point
+    // to even via the 1.5*2^23 trick); queue the codes near a half-way point
 #pragma unroll
     for (int o = 0; o < NOUT; ++o) {
       float gm = 0.f;
@@ -1105,12 +1096,19 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       const float sa = gm * (1.f / QF);
       const bool normal = sa >= 1.1754943508222875e-38f;
       // 1/s~ would overflow: the slow path
-      if (sa != 0.f && !normal && tid == 0 && rank == 0) slot(it)->flags = RF_REDO;
+      if (sa != 0.f && !normal && tid == 0 && rank == 0) {
+        thead(it)->flags = RF_REDO;
+      }
       const float r32 = normal ? __frcp_rn(sa) : 0.f;
-      // candidates for the row maximum: every binary32 input is within
-      // 3u|input| + 12u max|B| of its value scaled by the row's common 1/Rms
-      // error: the true maximum's unit is at or above thr
-      const float thr = gm - 12.f * kUnit * gm - 24.f * kUnit * maxBg[o];
+      // candidates for the row maximum: within the binary32 error of it
+      const float thr = gm - 12.f * kUnit * (gm + maxBg[o]);
+      if (gm > 0.f) {  // about one unit per row
+#pragma unroll
+        for (int k = 0; k < UPT; ++k) {
+          const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
+          if (mu[o][k] >= thr && u < seg_end) record(0, u, o);
+        }
+      }
       // |t - t_exact| <= tau: the binary32 error of t (12u(Q + |B| r) + 2uQ) plus
       // the distance between s~ and the exact scale (10uQ + 6u maxB r)
       const float tau = 24.f * kUnit * QF + 18.f * kUnit * maxBg[o] * r32;
@@ -1121,11 +1119,6 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
       for (int k = 0; k < UPT; ++k) {
         const int u = seg_begin + tid + k * static_cast<int>(blockDim.x);
         if (u >= seg_end) continue;
-        if (gm > 0.f && mu[o][k] >= thr) {  // about one unit a row
-          float2 bk[W];
-          b_of(o, k, bk);
-          record(0, u, o, G[o][k], bk);
-        }
         uint32_t bits[2 * W];  // low bits: the code (two's complement)
         float dmax = 0.f;      // largest |t - RNE(t)| of the unit
         float2 bk[W];
@@ -1145,67 +1138,64 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
           bits[2 * i + 1] = __float_as_uint(m.y);
           dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
         }
-        store_codes(y, row, u, bits);
-        // some code of the unit is near a half-way point (rare): record the unit
-        if (dmax > lim) {
-          if (NOUT == 1) b_of(o, k, bk);
-          record(1, u, o, G[o][k], bk);
+        if (MODE != LOAD_SCALAR) {
+          if (INT4) {  // 8 codes -> 4 bytes, even column in the low nibble
+            uint32_t w = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w |= (bits[e] & 0xFu) << (4 * e);
+            __stcs(reinterpret_cast<unsigned int *>(y + row * (n / 2) +
+                                                    static_cast<int64_t>(u) * 4), w);
+          } else {     // 8 codes -> 8 bytes
+            const uint32_t lo = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040),
+                                            __byte_perm(bits[2], bits[3], 0x0040), 0x5410);
+            const uint32_t hi = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040),
+                                            __byte_perm(bits[6], bits[7], 0x0040), 0x5410);
+            __stcs(reinterpret_cast<uint2 *>(y + row * n + static_cast<int64_t>(u) * 8),
+                   make_uint2(lo, hi));
+          }
+        } else {
+          if (INT4) {
+            y[row * (n / 2) + u] =
+                static_cast<uint8_t>((bits[0] & 0xFu) | ((bits[1] & 0xFu) << 4));
+          } else {
+            const int64_t j = row * n + 2 * static_cast<int64_t>(u);
+            y[j] = static_cast<uint8_t>(bits[0] & 0xFFu);
+            if (2 * u + 1 < n) y[j + 1] = static_cast<uint8_t>(bits[1] & 0xFFu);
+          }
         }
+        // some code of the unit is near a half-way point (rare): record the unit
+        if (dmax > lim) record(1, u, o);
       }
     }
     if (MODE == LOAD_STAGED && ++stage == stages) {
       stage = 0;
       phase ^= 1u;
     }
-    // ---- the settling warp, while the next row's copy is in flight: the
-    // previous row's record is complete (two barriers have passed since):
-    // fetch its units' x; the row before that has its x in place: settle it
-    if (settler) {
-      if (it >= 1) prefetch_record<ADD, U>(p, slot(it - 1), prev_row, lane);
-      if (it >= 2) {
-        cp_async_wait<1>();
-        __syncwarp();
-        settle_record<T, INT4, NOUT, ADD, U>(p, slot(it - 2), prev2_row, lane);
-      }
-    }
-    prev2_row = prev_row;
-    prev_row = row;
   }
 
   // the next kernel on the stream may start its set-up (it waits for this
   // grid's completion before it reads anything)
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  // ---- settle the last two rows (rows 0 .. it-1 are complete; all but the
-  // last two are settled, and the x of row it-2 is on its way)
+  // ---- settle this CTA's (cluster's) rows from their records, once the last
+  // row's record is complete.  After the barrier no CTA touches a peer's
+  // shared memory.
   if (it >= 1) {
     ex.sync();
-    if (settler) {
-      prefetch_record<ADD, U>(p, slot(it - 1), prev_row, lane);
-      if (it >= 2) {
-        cp_async_wait<1>();
-        __syncwarp();
-        settle_record<T, INT4, NOUT, ADD, U>(p, slot(it - 2), prev2_row, lane);
-      }
-      cp_async_wait<0>();
-      __syncwarp();
-      settle_record<T, INT4, NOUT, ADD, U>(p, slot(it - 1), prev_row, lane);
-    }
+    if (rank == 0) tail_settle<T, INT4, NOUT, ADD, U>(p, smem + lay.trec, static_cast<int>(it));
   }
   // ---- the last CTA to finish returns the hand-out counters to zero (every
   // CTA's tickets are taken before it counts itself done) and checks that
-  // every dynamic row was handed out exactly once and each CTA drew one empty
-  // ticket: counters that were not zero when the call started fail this
+  // the rows handed out were exactly the dynamic rows: counters that were not
+  // zero when the call started fail this
   if (dyn && tid == 0) {
     atomicAdd(p.sched + 2, ts->ndyn);
     __threadfence();
     if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
       __threadfence();
-      const int handed = atomicExch(p.sched, 0);
+      atomicExch(p.sched, 0);
       const int taken = atomicExch(p.sched + 2, 0);
       atomicExch(p.sched + 1, 0);
-      const int64_t pool = p.rows - p.dyn_base;
-      if ((static_cast<int64_t>(taken) != pool ||
-           static_cast<int64_t>(handed) != pool + gridDim.x) &&
+      if (static_cast<int64_t>(taken) != p.rows - p.dyn_base &&
           atomicCAS(p.status, 0, DEV_SCHED) == 0)
         *reinterpret_cast<volatile int64_t *>(p.status + 2) = -1;
     }

@@ -259,9 +259,10 @@ def test_scalar_plans(units, cluster):
 @pytest.mark.parametrize("rows,n", [(40000, 256), (300000, 64)])
 @pytest.mark.parametrize("schedule", [1, 2])
 def test_many_rows_per_cta(rows, n, schedule):
-    # one resident CTA per SM: hundreds of rows per CTA, each settled one row
-    # behind from the two records in shared memory; with schedule 2 a quarter
-    # of the rows (tens of thousands) go through the hand-out counter
+    # one resident CTA per SM: hundreds of rows per CTA (or, where their
+    # records do not fit in shared memory, a grid run in waves), settled from
+    # the records after each CTA's last row; with schedule 2 a quarter of the
+    # rows (tens of thousands) go through the hand-out counter
     w = wl.random_case(rows, n, seed=21, beta=True, smooth1=True)
     p = plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1, schedule=schedule)
     g, _ = run_gpu(w, plan=p)
@@ -442,7 +443,7 @@ def test_non_default_stream():
 
 # ------------------------------------------------------------------ device-side failure paths
 
-def _call_with_plan(w, p, ws, nb):
+def _call_with_plan(w, p, ws, nb, outputs=False):
     x1 = dev_bits(w.x1, w.dtype)
     x2 = dev_bits(w.x2, w.dtype)
     cb = w.n if w.qdtype == "int8" else w.n // 2
@@ -456,7 +457,14 @@ def _call_with_plan(w, p, ws, nb):
     assert st == A.ARNQ_OK, A.arnq_status_string(st)
     torch.cuda.synchronize()
     h = ws[:32].cpu().numpy().view(np.int32)
-    return int(h[0]), int(h[2:4].view(np.int64)[0]), h[4:7].copy()
+    res = (int(h[0]), int(h[2:4].view(np.int64)[0]), h[4:7].copy())
+    if outputs:
+        g = {"y1": y1.cpu().numpy().reshape(w.rows, cb), "scale1": sc1.cpu().numpy(),
+             "x_out": xo.cpu().numpy().view(np.uint16).reshape(w.rows, w.n),
+             "y2": np.full((w.rows, cb), CANARY, np.uint8),
+             "scale2": np.full(w.rows * 4, CANARY, np.uint8).view(np.float32)}
+        return res + (g,)
+    return res
 
 
 @pytest.mark.parametrize("pk", [dict(cluster=1), dict(cluster=1, schedule=2, grid=64),
@@ -481,66 +489,30 @@ def test_a_device_wait_that_runs_out_is_reported(pk):
 
 
 def test_hand_out_counters_not_at_zero_are_reported_and_cleared():
-    # A workspace whose counters were not zero-filled: the call hands out rows
-    # from the wrong place, and says so (ARNQ_ERR_WORKSPACE_STATE); it leaves
-    # the counters at zero, so the next call is exact.
+    # A workspace whose counters were not zero-filled.  Starting above zero,
+    # the call skips the rows below the start and says so
+    # (ARNQ_ERR_WORKSPACE_STATE); starting below zero, the CTAs that draw the
+    # negative tickets stop early, and the call either hands every row out
+    # (exact results) or says so.  Either way it leaves the counters at zero,
+    # so the next call is exact.
     w = wl.random_case(600, 4096, seed=78, beta=True, smooth1=True)
+    o = run_oracle(w)
     ws, nb = workspace_for(w.rows, w.n)
     p = plan(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=64)
-    for garbage in (5, -3):
-        ws.zero_()
-        ws[16:20].view(torch.int32).fill_(garbage)
-        code, row, ctr = _call_with_plan(w, p, ws, nb)
-        assert code == A.ARNQ_ERR_WORKSPACE_STATE and row == -1, (garbage, code)
-        assert not ctr.any()
+    ws.zero_()
+    ws[16:20].view(torch.int32).fill_(5)
+    code, row, ctr = _call_with_plan(w, p, ws, nb)
+    assert code == A.ARNQ_ERR_WORKSPACE_STATE and row == -1, code
+    assert not ctr.any()
+    ws.zero_()
+    ws[16:20].view(torch.int32).fill_(-3)
+    code, row, ctr, g = _call_with_plan(w, p, ws, nb, outputs=True)
+    assert not ctr.any()
+    if code == 0:
+        compare(g, o, "int8", "negative start")
+    else:
+        assert code == A.ARNQ_ERR_WORKSPACE_STATE and row == -1, code
     ws[:16].zero_()
-    code, _, ctr = _call_with_plan(w, p, ws, nb)
+    code, _, ctr, g = _call_with_plan(w, p, ws, nb, outputs=True)
     assert code == 0 and not ctr.any()
-
-
-# ------------------------------------------------------------------ the INT4 word container
-
-@pytest.mark.parametrize("pk", [dict(), dict(kernel=A.ARNQ_KERNEL_DIRECT),
-                                dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4),
-                                dict(kernel=A.ARNQ_KERNEL_DIRECT, cluster=2, units=1)],
-                         ids=["auto", "direct", "staged-cl4", "direct-cl2"])
-@pytest.mark.parametrize("rows,n,dt", [(211, 5120, "fp16"), (37, 1000, "bf16"),
-                                       (9, 8200, "bf16"), (3, 16384, "fp16")])
-def test_int4_word_container(rows, n, dt, pk):
-    # eight codes per 32-bit word: parity with the oracle's word packing, and
-    # the same bytes as the two-per-byte container on the same inputs and plan
-    w = wl.random_case(rows, n, dtype=dt, qdtype="int4_int32", seed=rows + n, beta=True,
-                       smooth1=True, smooth2=True, mask=(True, True))
-    p = plan(**pk) if pk else None
-    g, _ = run_gpu(w, plan=p)
-    o = run_oracle(w)
-    compare(g, o, "int4_int32", "word container")
-    w4 = wl.Workload(**{**w.__dict__, "qdtype": "int4"})
-    g4, _ = run_gpu(w4, plan=p)
-    for k in ("y1", "y2", "scale1", "scale2"):
-        assert np.array_equal(g[k].view(np.uint8), g4[k].view(np.uint8)), k
-
-
-def test_int4_word_container_no_add_and_alignment():
-    w = wl.random_case(64, 2048, seed=31, qdtype="int4_int32", beta=True, smooth1=True)
-    x = dev_bits(w.x1, "bf16")
-    y = torch.empty(w.rows * w.n // 8, dtype=torch.int32, device="cuda")
-    sc = torch.empty(w.rows, dtype=torch.float32, device="cuda")
-    ws, nb = workspace_for(w.rows, w.n)
-    gm, bt, sm = dev_bits(w.gamma, "bf16"), dev_bits(w.beta, "bf16"), dev_bits(w.smooth1, "bf16")
-    st = A.arnq_rms_norm_dynamic_quant(x, gm, bt, sm, w.rows, w.n, A.ARNQ_BF16, w.eps,
-                                       A.ARNQ_INT4_INT32, y, sc, ws, nb, None)
-    assert st == A.ARNQ_OK
-    torch.cuda.synchronize()
-    o = oracle.rms_norm_dynamic_quant(w.x1, w.gamma, w.beta, w.smooth1, eps=w.eps,
-                                      qdtype="int4_int32")
-    g = {"y1": y.cpu().numpy().reshape(w.rows, -1), "scale1": sc.cpu().numpy(),
-         "y2": np.full((w.rows, w.n // 2), CANARY, np.uint8),
-         "scale2": np.full(w.rows * 4, CANARY, np.uint8).view(np.float32)}
-    compare(g, {"y1": o["y"], "scale1": o["scale"], "y2": None}, "int4_int32", "no-add words",
-            xout=False)
-    # a word output that is not 4-byte aligned is refused before any launch
-    yb = torch.empty(w.rows * w.n // 2 + 2, dtype=torch.uint8, device="cuda")
-    st = A.arnq_rms_norm_dynamic_quant(x, gm, bt, sm, w.rows, w.n, A.ARNQ_BF16, w.eps,
-                                       A.ARNQ_INT4_INT32, yb.data_ptr() + 2, sc, ws, nb, None)
-    assert st == A.ARNQ_ERR_ALIGN
+    compare(g, o, "int8", "after the counters were cleared")
