@@ -92,8 +92,7 @@ typedef enum arnq_status {
   ARNQ_ERR_WORKSPACE = 8,       /* workspace NULL or smaller than arnq_workspace_size()    */
   ARNQ_ERR_CUDA = 9,            /* a CUDA call failed (launch, attribute, device query)    */
   ARNQ_ERR_PLAN = 10,           /* an explicit plan that cannot run this problem           */
-  ARNQ_ERR_DEVICE_TIMEOUT = 11, /* reported through the workspace status block only        */
-  ARNQ_ERR_WORKSPACE_STATE = 12 /* status block only: the workspace was not zero-filled    */
+  ARNQ_ERR_DEVICE_TIMEOUT = 11  /* reported through the workspace status block only        */
 } arnq_status;
 
 typedef enum arnq_dtype { ARNQ_BF16 = 0, ARNQ_FP16 = 1 } arnq_dtype;
@@ -137,15 +136,12 @@ ARNQ_API arnq_status arnq_selected_outputs(int out_mask, int has_smooth1, int ha
 /* Workspace bytes arnq_run needs for this problem (first phase of the pages'
  * two-phase call, "aclnnAddRmsNormDynamicQuantV2GetWorkspaceSize"): 256 for
  * every valid problem.  The workspace holds the status block (bytes 0-15, see
- * arnq_workspace_status), which the kernels write only on error, and three
- * row hand-out counters (bytes 16-27) that every call leaves at zero; the
- * per-row bookkeeping of the exact scales stays in on-chip shared memory.
- * The caller allocates it on the device (8-byte aligned) and zero-fills all
- * 256 bytes once; it may then be reused for any number of calls on one
- * stream (not by calls that overlap).  A call that finds the counters not at
- * zero records ARNQ_ERR_WORKSPACE_STATE in the status block (its outputs are
- * then unreliable) and leaves them at zero.  Validates the same arguments as
- * arnq_run (except pointers).  Host only. */
+ * arnq_workspace_status), which the kernels write only on error; the rest is
+ * reserved.  The per-row bookkeeping of the exact scales stays in on-chip
+ * shared memory.  The caller allocates it on the device (8-byte aligned) and
+ * zero-fills its status block once; it may then be reused for any number of
+ * calls on one stream (not by calls that overlap).  Validates the same
+ * arguments as arnq_run (except pointers).  Host only. */
 ARNQ_API arnq_status arnq_workspace_size(int64_t rows, int64_t n, arnq_dtype dt, arnq_qdtype qdt,
                                 int out_mask, int has_smooth1, int has_smooth2, size_t *bytes);
 
@@ -188,7 +184,7 @@ ARNQ_API arnq_status arnq_rms_norm_dynamic_quant(const void *x, const void *gamm
                                         void *stream);
 
 /* Status block at the start of the workspace.  code is 0 (ARNQ_OK) until a
- * kernel records an error (ARNQ_ERR_DEVICE_TIMEOUT, ARNQ_ERR_WORKSPACE_STATE);
+ * kernel records an error (ARNQ_ERR_DEVICE_TIMEOUT);
  * the library never clears it.  row is the first row the failing kernel did
  * not finish (-1 when no row applies).  Read it with a device-to-host copy
  * after synchronizing the stream; zero it to re-arm. */
@@ -227,11 +223,7 @@ typedef struct arnq_plan {
                             than its copies bring, so that wait runs out and
                             the call records ARNQ_ERR_DEVICE_TIMEOUT; at most
                             65536; 0 in normal use                           */
-  int32_t schedule;      /* 1: rows dealt out to CTAs in turn (the default);
-                            2: the last quarter of the rows handed out one at
-                            a time, by counters in the workspace, to whichever
-                            CTA is free (staged kernel, one CTA per row, at
-                            least two rows per CTA); 0 = choose (1)          */
+  int32_t reserved;      /* must be 0                                          */
 } arnq_plan;
 
 /* Fills *plan with the plan arnq_run would use for these arguments (pointers

@@ -32,7 +32,6 @@ ARNQ_ERR_WORKSPACE = 8
 ARNQ_ERR_CUDA = 9
 ARNQ_ERR_PLAN = 10
 ARNQ_ERR_DEVICE_TIMEOUT = 11
-ARNQ_ERR_WORKSPACE_STATE = 12
 
 ARNQ_BF16, ARNQ_FP16 = 0, 1
 ARNQ_INT8, ARNQ_INT4, ARNQ_INT4_INT32 = 0, 1, 2
@@ -48,7 +47,7 @@ ARNQ_WORKSPACE_BYTES = 256
 class arnq_plan(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in
                 ("kernel", "cluster", "threads", "units", "stages", "ctas_per_sm", "grid",
-                 "vector", "wait_limit_us", "test_hold_bytes", "schedule")]
+                 "vector", "wait_limit_us", "test_hold_bytes", "reserved")]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

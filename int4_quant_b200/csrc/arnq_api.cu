@@ -222,7 +222,6 @@ struct Launch {
   KernelFn fn;
   int smem, seg, units;
   int tail_rows, trec_bytes;  // row records per CTA (cluster) and their bytes
-  int64_t dyn_base;  // first row handed out by the workspace counter (rows: none)
 };
 
 int upt_candidate(int mode, int i) {
@@ -251,7 +250,7 @@ arnq_status occupancy(KernelFn fn, int threads, int smem, int *per_sm) {
 // Requested plan fields that no plan can take (checked before any device query).
 arnq_status check_plan_fields(const arnq_plan &q) {
   if (q.wait_limit_us < 0 || q.test_hold_bytes < 0 || q.test_hold_bytes > 65536 || q.grid < 0 ||
-      q.ctas_per_sm < 0 || q.schedule < 0 || q.schedule > 2 || q.stages < 0 || q.threads < 0 ||
+      q.ctas_per_sm < 0 || q.reserved != 0 || q.stages < 0 || q.threads < 0 ||
       q.units < 0 || q.cluster < 0)
     return ARNQ_ERR_PLAN;
   return ARNQ_OK;
@@ -361,14 +360,12 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   // that give every CTA 12 rows 46.2 us), no more clusters than rows; while
   // the records do not fit, fewer clusters per SM with more rows each; when
   // not even one cluster can hold its rows' records, a grid run in waves with
-  // fewer rows per cluster.  A requested grid is kept.  With the counter
-  // hand-out (schedule 2) a CTA keeps two records more than its share: the
-  // rows handed out at the end go to whichever CTA is free.
+  // fewer rows per cluster.  A requested grid is kept.
   struct Eval {
     int per_sm = 0, smem = 0, tail_rows = 0;
     int64_t nclusters = 0;
   };
-  const int spare = (pl->schedule == 2 && cl == 1 && mode == arnq::LOAD_STAGED) ? 2 : 0;
+  const int spare = 0;
   // clusters resident at once with `sm` bytes of shared memory per CTA
   auto resident = [&](int sm, int *per_sm, int64_t *slots) -> arnq_status {
     *per_sm = 0;
@@ -498,25 +495,6 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   pl->grid = static_cast<int32_t>(nclusters * cl);
   L->tail_rows = best.tail_rows;
   L->trec_bytes = trec;
-  // Row hand-out.  Schedule 1 (the default): rows dealt out in turn.
-  // Schedule 2 (staged kernel, one CTA per row, at least two rows per CTA, on
-  // request): the first three quarters of each CTA's share dealt out in turn,
-  // the rest handed out by the workspace counter as CTAs become free.  The
-  // counter evens out the CTAs' loop ends, but then every CTA settles its
-  // records at the same time, with HBM idle; dealt out in turn, the CTAs that
-  // finish first settle while the others still stream, and on B200 that was
-  // faster on 8192 x 4096, 2048 x 16384 and 4096 x 7168 (and even on
-  // 16384 x 5120).
-  L->dyn_base = P.rows;
-  const bool can_dyn = mode == arnq::LOAD_STAGED && cl == 1 && P.rows >= 2 * nclusters &&
-                       P.rows < (int64_t(1) << 30);
-  if (pl->schedule == 2 && !can_dyn) return ARNQ_ERR_PLAN;
-  if (pl->schedule == 0) pl->schedule = 1;
-  if (pl->schedule == 2) {
-    int64_t per = 3 * P.rows / (4 * nclusters);
-    if (per < 1) per = 1;
-    L->dyn_base = per * nclusters;
-  }
   L->fn = fn;
   L->smem = smem;
   L->seg = seg;
@@ -631,11 +609,9 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   }
   k.x_out = static_cast<uint16_t *>(P.x_out);
   k.status = static_cast<int32_t *>(workspace);
-  k.sched = static_cast<int32_t *>(workspace) + 4;
   k.tie_cap = arnq::tie_cap(static_cast<int>(P.n), (P.on1 ? 1 : 0) + (P.on2 ? 1 : 0));
   k.tail_rows = L.tail_rows;
   k.trec_bytes = L.trec_bytes;
-  k.dyn_base = L.dyn_base;
   k.rows = P.rows;
   k.n = static_cast<int32_t>(P.n);
   k.units = L.units;
@@ -737,8 +713,6 @@ const char *arnq_status_string(arnq_status s) {
     case ARNQ_ERR_CUDA: return "ARNQ_ERR_CUDA: a CUDA call failed";
     case ARNQ_ERR_PLAN: return "ARNQ_ERR_PLAN: the launch plan cannot run this problem";
     case ARNQ_ERR_DEVICE_TIMEOUT: return "ARNQ_ERR_DEVICE_TIMEOUT: a kernel gave up waiting for a copy";
-    case ARNQ_ERR_WORKSPACE_STATE:
-      return "ARNQ_ERR_WORKSPACE_STATE: the workspace was not zero-filled before its first call";
   }
   return "ARNQ: unknown status";
 }

@@ -14,10 +14,9 @@
 // thread-block cluster of CTAs sharing a row through distributed shared memory)
 // takes one row at a time; each thread keeps its elements of x and its folded
 // parameters G_k in registers (B_k of 16-byte units in shared memory, read
-// back by the thread that wrote it).  Persistent grid: a CTA takes rows c,
-// c + G, ... and then (staged kernel, one CTA per row) rows handed out one at
-// a time by a counter in the workspace.  Two barriers per row: after the sum
-// of squares and after the row maximum.  The kernel is launched as a
+// back by the thread that wrote it).  Persistent grid: a CTA (cluster) takes
+// rows c, c + G, ...  Two barriers per row: after the sum of squares and
+// after the row maximum.  The kernel is launched as a
 // programmatic dependent (it waits for the preceding work before touching
 // memory, and lets the next kernel start its set-up after its last row).
 //
@@ -66,8 +65,7 @@ enum : int { LOAD_VEC = 0, LOAD_SCALAR = 1, LOAD_STAGED = 2 };
 
 // status codes the kernels record in the workspace status block
 enum : int {
-  DEV_TIMEOUT = 11,   // a bounded wait ran out
-  DEV_SCHED = 12      // the row hand-out counters were not zero when the call started
+  DEV_TIMEOUT = 11    // a bounded wait ran out
 };
 
 // A bounded wait gives up after this long (nanoseconds of %globaltimer)
@@ -77,8 +75,8 @@ constexpr unsigned long long kWaitLimitNs = 1000000000ull;
 // row flags exchanged at the first barrier of the next row
 enum : int { RF_REDO = 1, RF_ABORT = 2 };
 
-// The workspace holds only the status block (kStatusBytes: the status at
-// bytes 0-15, the row hand-out counters at 16-27).
+// The workspace holds only the status block (kStatusBytes; the status code
+// and a row at bytes 0-15, the rest reserved).
 constexpr int kStatusBytes = 256;
 
 // Row records.  The binary32 fast path leaves a few units (8 or 2 elements)
@@ -119,8 +117,6 @@ __host__ __device__ inline int tail_rec_bytes(int tcap) {
 //   maxb  [NOUT][nslots] floats: set-up reduction of the bound on |B_k|
 //   flags [2] ints: RF_* of a row, by row parity
 //   bars  [stages] mbarriers
-//   srow  [stages] int64: staged kernel, the row each stage holds (-1: none)
-//   take  32 bytes: the copy-issuing thread's row hand-out state (TakeState)
 //   trec  [tail_rows] row records of trec_bytes each (used in the cluster's first CTA)
 //   bsm   16-byte units: B_k = beta * smooth_k of every thread's units,
 //         [NOUT][UPT][2][threads] float4 (bsm_bytes_for)
@@ -133,15 +129,7 @@ __host__ __device__ inline int bsm_bytes_for(bool vector_units, int nout, int up
   return vector_units ? nout * upt * threads * 32 : 0;
 }
 struct Layout {
-  int ss, wmax, maxb, flags, bars, srow, take, trec, bsm, ring;
-};
-struct TakeState {
-  int64_t nxt;   // next row dealt out in turn
-  int64_t pend;  // the row of the next refill, taken before it is due
-  int ndyn;      // rows taken from the counter
-  int dry;       // the counter ran out: take nothing more
-  int taken;     // rows taken (at most tail_rows: one record each)
-  int pad;
+  int ss, wmax, maxb, flags, bars, trec, bsm, ring;
 };
 __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, int tail_rows,
                                               int trec_bytes, int bsm_bytes) {
@@ -154,8 +142,6 @@ __host__ __device__ inline Layout make_layout(int nslots, int nout, int stages, 
   L.flags = off; off += 2 * 4;
   off = (off + 7) & ~7;
   L.bars = off;  off += stages * 8;
-  L.srow = off;  off += stages * 8;
-  L.take = off;  off += 32;
   off = (off + 15) & ~15;
   L.trec = off;  off += tail_rows * trec_bytes;
   off = (off + 15) & ~15;
@@ -171,10 +157,6 @@ struct KParams {
   float *scale[2];            // per output slot
   uint16_t *x_out;
   int32_t *status;            // workspace status block
-  int32_t *sched;             // workspace: tickets handed out, CTAs done, rows handed out
-                              // (all zero between calls)
-  int64_t dyn_base;           // staged, one CTA per row: rows from here on are handed
-                              // out by the counter (rows = none)
   int32_t tie_cap;            // near-tie units a record holds
   int64_t rows;
   int32_t n;                  // row length in elements
@@ -723,7 +705,6 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   float *maxb_slots = reinterpret_cast<float *>(smem + lay.maxb);    // [NOUT][nslots]
   int *rflags = reinterpret_cast<int *>(smem + lay.flags);           // [2]
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + lay.bars);
-  int64_t *srow = reinterpret_cast<int64_t *>(smem + lay.srow);
   unsigned char *ring = smem + lay.ring;
 
   // ---- the first rows' copies go out before anything else (the parameter
@@ -743,51 +724,9 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   if (MODE == LOAD_STAGED && tid == 0) {
     for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  // The rows a CTA (cluster) takes, in order, as the thread that issues the
-  // copies sees them: rows below p.dyn_base are dealt out in turn (c, c + G,
-  // ...); the others are handed out one at a time by the workspace counter,
-  // so that CTAs that run faster take more of them.  A ticket is fetched one
-  // take ahead: its latency overlaps a row.  -1: no more rows.  The hand-out
-  // state lives in shared memory (registers are scarce), all but the
-  // prefetched ticket, whose load is waited for only at the next take.
-  const bool dyn = MODE == LOAD_STAGED && !CL && p.dyn_base < p.rows;
-  TakeState *ts = reinterpret_cast<TakeState *>(smem + lay.take);
-  int ticket = 0;
-  // A ticket is drawn only while the CTA has a record left for its row: a
-  // ticket drawn and never used would be a row nobody processes.
-  auto take = [&]() -> int64_t {
-    if (ts->taken >= p.tail_rows) return -1;  // every record in use
-    const int64_t nx = ts->nxt;
-    if (nx < p.dyn_base) {
-      ts->nxt = nx + nclusters;
-      if (nx >= p.rows) return -1;
-      ts->taken += 1;
-      // the first ticket, with the last row dealt out in turn
-      if (dyn && nx + nclusters >= p.dyn_base && ts->taken < p.tail_rows)
-        ticket = atomicAdd(p.sched, 1);
-      return nx;
-    }
-    if (!dyn || ts->dry) return -1;
-    const int64_t r = p.dyn_base + ticket;
-    if (r >= p.rows || r < p.dyn_base) {
-      ts->dry = 1;
-      return -1;
-    }
-    ts->ndyn += 1;
-    ts->taken += 1;
-    if (ts->taken < p.tail_rows) ticket = atomicAdd(p.sched, 1);
-    return r;
-  };
-  if (MODE == LOAD_STAGED && tid == 0) {
-    ts->nxt = cluster_id;
-    ts->ndyn = 0;
-    ts->dry = 0;
-    ts->taken = 0;
     for (int s = 0; s < stages; ++s) {
-      const int64_t row = take();
-      srow[s] = row;
-      if (row >= 0 && seg_len > 0) issue(row, s, s == 0 ? p.test_hold_tx : 0u);
+      const int64_t row = cluster_id + s * nclusters;
+      if (row < p.rows && seg_len > 0) issue(row, s, s == 0 ? p.test_hold_tx : 0u);
     }
   }
 
@@ -915,23 +854,9 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   };
   int stage = 0;          // staged: it % stages, kept incrementally
   uint32_t phase = 0;     // staged: (it / stages) & 1, the mbarrier phase to wait for
-  for (;; ++it) {
-    int64_t row;
-    if (MODE == LOAD_STAGED) {
-      row = srow[stage];
-      if (row < 0) break;
-    } else {
-      row = cluster_id + it * nclusters;
-      if (row >= p.rows) break;
-    }
+  for (int64_t row = cluster_id; row < p.rows; row += nclusters, ++it) {
     const int par = static_cast<int>(it & 1);
     bool timed_out = false;
-    if (MODE == LOAD_STAGED && tid == 0) {
-      // while this row's data is on its way: the row of this iteration's
-      // refill (issued after the first barrier, when the stage is free), so
-      // that the refill itself is one shared-memory load and the copy
-      ts->pend = take();
-    }
     if (MODE == LOAD_STAGED && seg_len > 0) {
       timed_out = !mbar_wait_bounded(smem_addr(&bars[stage]), phase, p.wait_limit_ns);
     }
@@ -1019,7 +944,7 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
           if (seg_len > 0) {
             for (int s = 0; s < stages; ++s) {
               const int64_t it2 = it + s;  // the ring's outstanding iterations
-              if (srow[it2 % stages] < 0) break;
+              if (cluster_id + it2 * nclusters >= p.rows) break;
               mbar_wait_bounded(smem_addr(&bars[it2 % stages]),
                                 static_cast<uint32_t>((it2 / stages) & 1), p.wait_limit_ns);
             }
@@ -1027,11 +952,10 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
         }
         break;
       }
-      // every thread has read this stage (and its row): refill it
-      if (tid == 0) {
-        const int64_t nrow = ts->pend;
-        srow[stage] = nrow;
-        if (nrow >= 0 && seg_len > 0) issue(nrow, stage, 0u);
+      // every thread has read this stage: refill it
+      if (tid == 0 && seg_len > 0) {
+        const int64_t nrow = row + static_cast<int64_t>(stages) * nclusters;
+        if (nrow < p.rows) issue(nrow, stage, 0u);
       }
     }
 
@@ -1182,23 +1106,6 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   if (it >= 1) {
     ex.sync();
     if (rank == 0) tail_settle<T, INT4, NOUT, ADD, U>(p, smem + lay.trec, static_cast<int>(it));
-  }
-  // ---- the last CTA to finish returns the hand-out counters to zero (every
-  // CTA's tickets are taken before it counts itself done) and checks that
-  // the rows handed out were exactly the dynamic rows: counters that were not
-  // zero when the call started fail this
-  if (dyn && tid == 0) {
-    atomicAdd(p.sched + 2, ts->ndyn);
-    __threadfence();
-    if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
-      __threadfence();
-      atomicExch(p.sched, 0);
-      const int taken = atomicExch(p.sched + 2, 0);
-      atomicExch(p.sched + 1, 0);
-      if (static_cast<int64_t>(taken) != p.rows - p.dyn_base &&
-          atomicCAS(p.status, 0, DEV_SCHED) == 0)
-        *reinterpret_cast<volatile int64_t *>(p.status + 2) = -1;
-    }
   }
 }
 

@@ -35,7 +35,7 @@ def test_exports_every_header_symbol():
 
 
 def test_status_strings():
-    for code in range(0, 13):
+    for code in range(0, 12):
         s = A.arnq_status_string(code)
         assert s.startswith("ARNQ_")
     assert "unknown" in A.arnq_status_string(99)
@@ -68,8 +68,7 @@ def test_selected_outputs_rejects_unknown_mask_bits():
 
 def test_workspace_is_the_status_block_for_every_problem():
     # the per-row bookkeeping stays on chip: the workspace is the 256-byte
-    # status block (status + row hand-out counters) whatever the shape, dtype,
-    # code type and outputs
+    # status block whatever the shape, dtype, code type and outputs
     for rows in (1, 2, 64, 8192, 16384, 2 ** 31 - 1):
         for n in (2, 8, 1000, 4096, 7168, 16384, A.ARNQ_MAX_N):
             for qdt in (A.ARNQ_INT8, A.ARNQ_INT4):
@@ -190,7 +189,7 @@ def test_static_scratch_entry_validates_on_the_host():
 
 
 @pytest.mark.parametrize("field,value", [
-    ("schedule", 3), ("schedule", -1), ("test_hold_bytes", 65537), ("test_hold_bytes", -16),
+    ("reserved", 1), ("reserved", -1), ("test_hold_bytes", 65537), ("test_hold_bytes", -16),
     ("wait_limit_us", -1), ("grid", -2), ("stages", -1), ("cluster", -4)])
 def test_plan_fields_out_of_range_are_refused_on_the_host(field, value):
     p = A.arnq_plan()

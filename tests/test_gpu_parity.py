@@ -5,9 +5,8 @@ Acceptance (the operator's stated tolerance): xOut bit-exact; INT4 packing
 bit-exact (codes are compared after unpacking both sides with the same
 reader, and hand-worked rows compare raw bytes); scales within relative 1e-5;
 codes within +-1 with at most 1e-4 of them off by one.  Every run also checks
-that the workspace status block stayed clear, that the row hand-out counters
-are back at zero, and that outputs the call must not write kept their canary
-bytes.
+that the workspace status block stayed clear (its reserved bytes untouched)
+and that outputs the call must not write kept their canary bytes.
 """
 import numpy as np
 import pytest
@@ -57,7 +56,7 @@ def canary_bytes(nbytes, offset=0):
 
 def workspace_for(rows, n):
     """A zeroed workspace of the size arnq_workspace_size asks for (the same
-    for every call: the status block and the row hand-out counters)."""
+    for every call: the status block)."""
     st, nb = A.arnq_workspace_size(max(rows, 1), max(n, 2), A.ARNQ_BF16, A.ARNQ_INT8,
                                    A.ARNQ_MASK_Y1 | A.ARNQ_MASK_Y2, 1, 1)
     assert st == A.ARNQ_OK
@@ -94,7 +93,7 @@ def run_gpu(w, plan=None, offset=0, inplace=False, mask="use", smooth="use", str
     torch.cuda.synchronize()
     wsh = ws[:32].cpu().numpy().view(np.int32)
     assert wsh[0] == 0, f"device status {wsh[0]}"
-    assert not wsh[4:7].any(), f"hand-out counters left at {wsh[4:7]}"
+    assert not wsh[4:7].any(), f"reserved workspace bytes written: {wsh[4:7]}"
     out = {
         "y1": y1.cpu().numpy().reshape(rows, cb),
         "y2": y2.cpu().numpy().reshape(rows, cb),
@@ -217,13 +216,11 @@ PLAN_CASES = [
     dict(kernel=A.ARNQ_KERNEL_STAGED, stages=1, cluster=4),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=8, units=2),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=16),
-    # one CTA per row, also with few CTAs per SM (more rows per CTA), rows
-    # dealt out in turn or the last quarter handed out by the counter, and
+    # one CTA per row, also with few CTAs per SM (more rows per CTA) and
     # explicit grids (fewer CTAs than rows; more CTAs than rows)
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=1, grid=16),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=16),
-    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=7, stages=2),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, grid=16),
+    dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, grid=7, stages=2),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, grid=1000),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4, grid=12),
     dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, units=2),
@@ -257,14 +254,13 @@ def test_scalar_plans(units, cluster):
 
 
 @pytest.mark.parametrize("rows,n", [(40000, 256), (300000, 64)])
-@pytest.mark.parametrize("schedule", [1, 2])
-def test_many_rows_per_cta(rows, n, schedule):
+@pytest.mark.parametrize("kernel", [A.ARNQ_KERNEL_STAGED, A.ARNQ_KERNEL_DIRECT])
+def test_many_rows_per_cta(rows, n, kernel):
     # one resident CTA per SM: hundreds of rows per CTA (or, where their
     # records do not fit in shared memory, a grid run in waves), settled from
-    # the records after each CTA's last row; with schedule 2 a quarter of the
-    # rows (tens of thousands) go through the hand-out counter
+    # the records after each CTA's last row
     w = wl.random_case(rows, n, seed=21, beta=True, smooth1=True)
-    p = plan(kernel=A.ARNQ_KERNEL_STAGED, ctas_per_sm=1, schedule=schedule)
+    p = plan(kernel=kernel, ctas_per_sm=1)
     g, _ = run_gpu(w, plan=p)
     compare(g, run_oracle(w), "int8", f"{rows} rows")
 
@@ -467,9 +463,9 @@ def _call_with_plan(w, p, ws, nb, outputs=False):
     return res
 
 
-@pytest.mark.parametrize("pk", [dict(cluster=1), dict(cluster=1, schedule=2, grid=64),
+@pytest.mark.parametrize("pk", [dict(cluster=1), dict(cluster=1, grid=64, stages=2),
                                 dict(cluster=4, stages=2)],
-                         ids=["cta", "cta-handout", "cluster"])
+                         ids=["cta", "cta-two-stages", "cluster"])
 def test_a_device_wait_that_runs_out_is_reported(pk):
     # Every CTA's first copy barrier expects 16 bytes more than its copies
     # bring, so its bounded wait (2 ms here) runs out while every real copy
@@ -486,33 +482,3 @@ def test_a_device_wait_that_runs_out_is_reported(pk):
     ws.zero_()
     g, _ = run_gpu(w, plan=plan(kernel=A.ARNQ_KERNEL_STAGED, **pk))
     compare(g, run_oracle(w), "int8", "after a timeout")
-
-
-def test_hand_out_counters_not_at_zero_are_reported_and_cleared():
-    # A workspace whose counters were not zero-filled.  Starting above zero,
-    # the call skips the rows below the start and says so
-    # (ARNQ_ERR_WORKSPACE_STATE); starting below zero, the CTAs that draw the
-    # negative tickets stop early, and the call either hands every row out
-    # (exact results) or says so.  Either way it leaves the counters at zero,
-    # so the next call is exact.
-    w = wl.random_case(600, 4096, seed=78, beta=True, smooth1=True)
-    o = run_oracle(w)
-    ws, nb = workspace_for(w.rows, w.n)
-    p = plan(kernel=A.ARNQ_KERNEL_STAGED, cluster=1, schedule=2, grid=64)
-    ws.zero_()
-    ws[16:20].view(torch.int32).fill_(5)
-    code, row, ctr = _call_with_plan(w, p, ws, nb)
-    assert code == A.ARNQ_ERR_WORKSPACE_STATE and row == -1, code
-    assert not ctr.any()
-    ws.zero_()
-    ws[16:20].view(torch.int32).fill_(-3)
-    code, row, ctr, g = _call_with_plan(w, p, ws, nb, outputs=True)
-    assert not ctr.any()
-    if code == 0:
-        compare(g, o, "int8", "negative start")
-    else:
-        assert code == A.ARNQ_ERR_WORKSPACE_STATE and row == -1, code
-    ws[:16].zero_()
-    code, _, ctr, g = _call_with_plan(w, p, ws, nb, outputs=True)
-    assert code == 0 and not ctr.any()
-    compare(g, o, "int8", "after the counters were cleared")

@@ -1,11 +1,11 @@
 """The no-allocation entry point arnq_run_static_scratch on a GPU.
 
 It serves callers that cannot allocate device memory at the point of the
-call; its scratch (the status block and the row hand-out counters) is a
-file-scope device array inside the library.  These tests check that two
-calls in a row each give exactly what arnq_run with a caller workspace gives
-on the same inputs and plan: INT8 with two outputs, packed INT4, rows shared
-by a thread-block cluster, and rows handed out through the array's counters.
+call; its scratch (the status block) is a file-scope device array inside
+the library.  These tests check that two calls in a row each give exactly
+what arnq_run with a caller workspace gives on the same inputs and plan:
+INT8 with two outputs, packed INT4, rows shared by a thread-block cluster,
+and a large row count.
 The file name sorts last so that a run stopping at the first failure has run
 every other GPU test first; it also passes alone in a fresh process.
 """
@@ -67,7 +67,7 @@ def _case(name):
         rows = int(name.rsplit("_", 1)[1])
         return wl.random_case(rows, 16384, seed=44 + rows, beta=True, smooth1=True), \
             A.ARNQ_MASK_ABSENT, False
-    if name == "handout_2048x4096":   # rows handed out through the array's counters
+    if name == "rows_2048x4096":   # several rows per CTA
         return wl.random_case(2048, 4096, seed=45, x_sigma=(1.0, 0.5), beta=True, smooth1=True,
                               mask=(True, False)), A.ARNQ_MASK_Y1, False
     raise KeyError(name)
@@ -88,10 +88,10 @@ def _same(got, ref):
 # Each case: the no-allocation entry point, twice in a row, against arnq_run
 # with a caller workspace (same inputs, same plan: identical bits).  The
 # cluster cases run right after a dual-output 16384-column call through the
-# same array, and the hand-out case right after the others, so each starts
-# from whatever the previous calls left in the array.
+# same array, and the last case right after the others, so each starts from
+# whatever the previous calls left in the array.
 CASES = ["int8_two_outputs", "int4_fp16", "dual_16384", "rows_16384_8", "rows_16384_128",
-         "handout_2048x4096"]
+         "rows_2048x4096"]
 
 
 @pytest.mark.parametrize("case", CASES)
