@@ -287,8 +287,12 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   if (max_seg == 0) return ARNQ_ERR_PLAN;
 
   // cluster: enough CTAs per row that one CTA's slice fits in registers (and,
-  // staged, one stage of it and its B_k in shared memory), then more CTAs per
-  // row while the rows are too few to fill the SMs
+  // staged, one stage of it and its B_k in shared memory).  No more: with
+  // fewer rows than SMs, a cluster spreading each row over more SMs measured
+  // slower than one CTA per row with more threads (B200, device time per
+  // call, L2-cold: 64 x 1024 4.4 us with one 128-thread CTA per row, 8.6 us
+  // as 2-CTA clusters; 128 x 16384 9.7 vs 12.8 us; 1 x 16384 7.4 vs 10.1 us
+  // as a 16-CTA cluster)
   if (pl->cluster == 0) {
     int cl = 1;
     auto too_big = [&](int c) {
@@ -298,7 +302,6 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
              nin * seg * 16 + nout * seg * 32 + 8192 > di.smem_per_block_optin;
     };
     while (cl < kMaxCluster && too_big(cl)) cl *= 2;
-    while (cl < kMaxCluster && P.rows * cl < di.sms && ceil_div(units, 2 * cl) >= 64) cl *= 2;
     pl->cluster = cl;
   }
   const int cl = pl->cluster;
@@ -311,7 +314,17 @@ arnq_status make_plan(const Problem &P, arnq_plan *pl, Launch *L) {
   // units per thread: of the variants whose threads hold a slice, the one with
   // the most CTAs (rows in flight) per SM, then the most units per thread
   // (fewer threads share a row: cheaper reductions); measured best on
-  // 4096..16384-column rows
+  // 4096..16384-column rows.  With fewer rows than SMs (each row has an SM
+  // to itself, latency rules): the fewest units per thread, i.e. the most
+  // threads on a row (64 x 1024: 4.4 us with 1 unit per thread, 5.8 us with 4)
+  if (pl->units == 0 && P.rows < di.sms) {
+    for (int i = 0; i < 3 && pl->units == 0; ++i) {
+      const int c = upt_candidate(mode, i);
+      const int t = round_up(static_cast<int>(ceil_div(seg, c)), 32);
+      if (t <= arnq::max_threads_for(mode, c, nout) && lookup(P.dt, P.qdt, nout, P.add, mode, c, cl))
+        pl->units = c;
+    }
+  }
   if (pl->units == 0) {
     int best = 0, best_ctas = -1;
     for (int i = 0; i < 3; ++i) {
