@@ -381,6 +381,20 @@ class DeviceRun:
                 p(s["s1"]), p(s["y2"]), p(s["s2"]), p(s["xo"]), p(self.ws), self.ws_bytes,
                 A._stream(stream))
 
+    def with_plan(self, **fields):
+        """The same buffers, launched through arnq_run_planned with a plan whose
+        given fields are set (the library chooses the others)."""
+        import copy
+        import ctypes
+        other = copy.copy(self)
+        pl = self.A.arnq_plan()
+        for k, v in fields.items():
+            setattr(pl, k, v)
+        other.plan_request = pl  # the struct the marshalled pointer refers to
+        other.fn = self.A.lib().arnq_run_planned
+        other.args = [tuple(a) + (ctypes.addressof(pl),) for a in self.args]
+        return other
+
     def launch(self, i, args=None):
         st = self.fn(*(args or self.args)[i % len(self.sets)])
         if st:
@@ -562,6 +576,24 @@ def main():
         barrier()
         repeats.append(r0.elapsed_time(r1) / K)
     run.check_status()
+    # the same K steps with the parameters promised constant (plan
+    # early_params; an opt-in, reported beside the default path's figure)
+    early_ms = []
+    er = run.with_plan(early_params=1)
+    for _ in range(max(1, args.repeats)):
+        for i in range(args.warmup):
+            er.launch(i)
+        barrier()
+        r0 = torch.cuda.Event(enable_timing=True)
+        r1 = torch.cuda.Event(enable_timing=True)
+        hold_device(torch)
+        r0.record(stream)
+        for i in range(K):
+            er.launch(i)
+        r1.record(stream)
+        barrier()
+        early_ms.append(r0.elapsed_time(r1) / K)
+    er.check_status()
     local_ms = total_ms
     total_ms = max_over_ranks(total_ms, dist, dev)
 
@@ -642,6 +674,12 @@ def main():
             e["clocks"] = ck.summary()
             if e["clocks"]["sm_mhz"]:
                 e["us_x_ghz"] = ms * e["clocks"]["sm_mhz"]  # ms * MHz = us * GHz
+            # the same calls with the parameters promised constant (plan
+            # early_params: loaded before the wait for the preceding call)
+            ep = wr.with_plan(early_params=1)
+            e["early_params_us_per_call"] = statistics.median(
+                [ep.timed(steps=200, warmup=20) for _ in range(3)]) * 1e3
+            ep.check_status()
             e["workload"] = wr.w.name
             workloads[name] = e
             del wr
@@ -705,6 +743,11 @@ def main():
             "plan": headline_plan,
             "parallelism": f"replicas x{world} (rows independent; no collective)",
         },
+        "early_params": {"ms_per_step": statistics.median(early_ms), "regions": len(early_ms),
+                         "gbs": nbytes / (statistics.median(early_ms) / 1e3) / 1e9,
+                         "note": "opt-in (plan early_params / constant_params=True): gamma, "
+                                 "beta and smooth loaded before the wait for the preceding "
+                                 "call; valid when that work does not write them"},
         "rows_per_s": rows_per_s,
         "bytes_per_step": nbytes,
         "frac_of_nominal_hbm": value / world / NOMINAL_HBM_GBS,

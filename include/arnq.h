@@ -223,7 +223,13 @@ typedef struct arnq_plan {
                             than its copies bring, so that wait runs out and
                             the call records ARNQ_ERR_DEVICE_TIMEOUT; at most
                             65536; 0 in normal use                           */
-  int32_t reserved;      /* must be 0                                          */
+  int32_t early_params;  /* 1: the kernel loads gamma, beta and the smooth
+                            scales before it waits for the preceding work on
+                            the stream (it is launched as a programmatic
+                            dependent), so those loads overlap that work's
+                            end.  Only correct when the preceding work does
+                            not write them (weights that stay constant, as in
+                            inference); 0 (the default): it waits first.     */
 } arnq_plan;
 
 /* Fills *plan with the plan arnq_run would use for these arguments (pointers

@@ -76,7 +76,8 @@ def _check(t, name, dtype=None):
 
 def add_rms_norm_dynamic_quant(x1, x2, gamma, beta=None, smooth1=None, smooth2=None, *,
                                eps: float = 1e-6, output_mask=None, qdtype: str = "int8",
-                               stream=None, out: Optional[dict] = None):
+                               stream=None, out: Optional[dict] = None,
+                               constant_params: bool = False):
     """aclnnAddRmsNormDynamicQuantV2 on CUDA tensors.
 
     x1, x2: [..., n] bf16 or fp16; gamma, beta, smooth1, smooth2: [n] same dtype.
@@ -85,7 +86,10 @@ def add_rms_norm_dynamic_quant(x1, x2, gamma, beta=None, smooth1=None, smooth2=N
     two codes per byte (even column in the low nibble); for
     qdtype="int4_int32", int32 [..., n/8] holding eight codes per word (column
     8w + k in bits 4k..4k+3).  `out` may pass preallocated tensors under the
-    same keys.
+    same keys.  constant_params=True promises that the work queued before
+    this call on the stream does not write gamma, beta or the smooth scales
+    (weights, as in inference): the kernel then loads them before it waits
+    for that work (the plan's early_params).
     """
     import torch
     _check(x1, "x1")
@@ -124,8 +128,14 @@ def add_rms_norm_dynamic_quant(x1, x2, gamma, beta=None, smooth1=None, smooth2=N
     if stream is None:
         stream = torch.cuda.current_stream(x1.device)
     ws = workspace(x1.device, nbytes, stream)
-    st = _abi.arnq_run(x1, x2, gamma, beta, smooth1, smooth2, rows, n, _DT[str(dt)], eps, mc,
-                       _QDT[qdtype], y1, s1, y2, s2, xo, ws, ws.numel(), stream)
+    args = (x1, x2, gamma, beta, smooth1, smooth2, rows, n, _DT[str(dt)], eps, mc, _QDT[qdtype],
+            y1, s1, y2, s2, xo, ws, ws.numel(), stream)
+    if constant_params:
+        plan = _abi.arnq_plan()
+        plan.early_params = 1
+        st = _abi.arnq_run_planned(*args, plan)
+    else:
+        st = _abi.arnq_run(*args)
     if st != _abi.ARNQ_OK:
         raise ArnqError(st, "arnq_run")
     return y1, s1, y2, s2, xo

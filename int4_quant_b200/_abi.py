@@ -47,7 +47,7 @@ ARNQ_WORKSPACE_BYTES = 256
 class arnq_plan(ctypes.Structure):
     _fields_ = [(name, ctypes.c_int32) for name in
                 ("kernel", "cluster", "threads", "units", "stages", "ctas_per_sm", "grid",
-                 "vector", "wait_limit_us", "test_hold_bytes", "reserved")]
+                 "vector", "wait_limit_us", "test_hold_bytes", "early_params")]
 
     def as_dict(self):
         return {f: getattr(self, f) for f, _ in self._fields_}

@@ -250,7 +250,8 @@ arnq_status occupancy(KernelFn fn, int threads, int smem, int *per_sm) {
 // Requested plan fields that no plan can take (checked before any device query).
 arnq_status check_plan_fields(const arnq_plan &q) {
   if (q.wait_limit_us < 0 || q.test_hold_bytes < 0 || q.test_hold_bytes > 65536 || q.grid < 0 ||
-      q.ctas_per_sm < 0 || q.reserved != 0 || q.stages < 0 || q.threads < 0 ||
+      q.ctas_per_sm < 0 || q.early_params < 0 || q.early_params > 1 || q.stages < 0 ||
+      q.threads < 0 ||
       q.units < 0 || q.cluster < 0)
     return ARNQ_ERR_PLAN;
   return ARNQ_OK;
@@ -629,7 +630,8 @@ arnq_status launch(const Problem &P, arnq_plan plan, void *workspace, cudaStream
   k.n = static_cast<int32_t>(P.n);
   k.units = L.units;
   k.seg_units = L.seg;
-  k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0);
+  k.flags = (P.beta ? arnq::F_BETA : 0) | (P.add && P.x_out ? arnq::F_XOUT : 0) |
+            (plan.early_params ? arnq::F_EARLY : 0);
   k.stages = plan.stages;
   k.eps = P.eps;
   k.inv_n = 1.0 / static_cast<double>(P.n);

@@ -59,7 +59,8 @@ namespace cg = cooperative_groups;
 
 enum : int {
   F_BETA = 1,   // beta given
-  F_XOUT = 2    // xOut written
+  F_XOUT = 2,   // xOut written
+  F_EARLY = 4   // parameters read before the wait for the preceding work
 };
 enum : int { LOAD_VEC = 0, LOAD_SCALAR = 1, LOAD_STAGED = 2 };
 
@@ -668,8 +669,14 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   constexpr int NIN = ADD ? 2 : 1;                  // staged inputs per row
 
   // Launched as a programmatic dependent: everything before this kernel on
-  // the stream is complete, and its memory visible, only from here on.
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  // the stream is complete, and its memory visible, only after
+  // griddepcontrol.wait.  Normally that is the first thing the kernel does.
+  // With F_EARLY (the caller's promise that the preceding work does not write
+  // gamma, beta or the smooth scales) the parameter loads and the set-up
+  // exchange come first, overlapping the preceding work's end, and the wait
+  // comes right before the first row's copies.
+  const bool early = (p.flags & F_EARLY) != 0;
+  if (!early) asm volatile("griddepcontrol.wait;" ::: "memory");
   Exchange<CL> ex;
   const int tid = threadIdx.x;
   const int lane = tid & 31;
@@ -708,7 +715,8 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
   unsigned char *ring = smem + lay.ring;
 
   // ---- the first rows' copies go out before anything else (the parameter
-  // loads and the set-up exchange overlap them).  The other threads wait on
+  // loads and the set-up exchange overlap them), unless the parameters were
+  // read before the wait (then right after it).  The other threads wait on
   // the barriers only after the set-up exchange below.
   // staged: row `row` goes to stage s, x1 then x2; the barrier expects `hold`
   // bytes more than the copies bring (testing only: then the wait runs out)
@@ -721,13 +729,16 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     bulk_g2s(dst, p.x1 + off, seg_bytes, bar, policy);
     if (ADD) bulk_g2s(dst + seg_bytes, p.x2 + off, seg_bytes, bar, policy);
   };
-  if (MODE == LOAD_STAGED && tid == 0) {
-    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  auto first_copies = [&]() {
     for (int s = 0; s < stages; ++s) {
       const int64_t row = cluster_id + s * nclusters;
       if (row < p.rows && seg_len > 0) issue(row, s, s == 0 ? p.test_hold_tx : 0u);
     }
+  };
+  if (MODE == LOAD_STAGED && tid == 0) {
+    for (int s = 0; s < stages; ++s) mbar_init(smem_addr(&bars[s]), 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!early) first_copies();
   }
 
   // ---- folded parameters for this thread's units: input_k = x*rinv*G_k + B_k
@@ -833,6 +844,10 @@ __device__ __forceinline__ void rows_body(const KParams &p) {
     }
   }
   ex.sync();
+  if (early) {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    if (MODE == LOAD_STAGED && tid == 0) first_copies();
+  }
   float maxBg[NOUT];  // bound on |B_k| over the whole row
 #pragma unroll
   for (int o = 0; o < NOUT; ++o) {

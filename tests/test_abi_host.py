@@ -189,7 +189,7 @@ def test_static_scratch_entry_validates_on_the_host():
 
 
 @pytest.mark.parametrize("field,value", [
-    ("reserved", 1), ("reserved", -1), ("test_hold_bytes", 65537), ("test_hold_bytes", -16),
+    ("early_params", 2), ("early_params", -1), ("test_hold_bytes", 65537), ("test_hold_bytes", -16),
     ("wait_limit_us", -1), ("grid", -2), ("stages", -1), ("cluster", -4)])
 def test_plan_fields_out_of_range_are_refused_on_the_host(field, value):
     p = A.arnq_plan()

@@ -253,6 +253,20 @@ def test_scalar_plans(units, cluster):
     compare(g, run_oracle(w), "int8", f"scalar u{units} c{cluster}")
 
 
+@pytest.mark.parametrize("pk", [dict(), dict(kernel=A.ARNQ_KERNEL_STAGED, cluster=4),
+                                dict(kernel=A.ARNQ_KERNEL_DIRECT), dict(kernel=A.ARNQ_KERNEL_STAGED,
+                                                                        stages=2)],
+                         ids=["auto", "cluster", "direct", "two-stages"])
+def test_parameters_read_before_the_wait(pk):
+    # early_params: gamma, beta and the smooth scales are loaded before the
+    # kernel waits for the preceding work on the stream (nothing before it
+    # writes them here); same results as the default order
+    w = wl.random_case(1000, 4096, seed=97, beta=True, smooth1=True, smooth2=True,
+                       mask=(True, True), outlier_frac=0.01)
+    g, _ = run_gpu(w, plan=plan(early_params=1, **pk))
+    compare(g, run_oracle(w), "int8", f"early params {pk}")
+
+
 @pytest.mark.parametrize("rows,n", [(40000, 256), (300000, 64)])
 @pytest.mark.parametrize("kernel", [A.ARNQ_KERNEL_STAGED, A.ARNQ_KERNEL_DIRECT])
 def test_many_rows_per_cta(rows, n, kernel):
@@ -428,6 +442,12 @@ def test_torch_facing_call_matches_the_abi():
     assert np.array_equal(y1.cpu().numpy().view(np.uint8), g["y1"])
     assert np.array_equal(s1.cpu().numpy(), g["scale1"])
     assert np.array_equal(xo.view(torch.int16).cpu().numpy().view(np.uint16), g["x_out"])
+    # the same call with the parameters promised constant (read before the
+    # kernel waits for the preceding work): the same bits
+    e1, t1, _, _, eo = q.add_rms_norm_dynamic_quant(x1, x2, dev_bits(w.gamma, "bf16"),
+                                                    eps=w.eps, constant_params=True)
+    torch.cuda.synchronize()
+    assert torch.equal(e1, y1) and torch.equal(t1, s1) and torch.equal(eo, xo)
 
 
 def test_non_default_stream():
