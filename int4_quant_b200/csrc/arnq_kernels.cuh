@@ -10,15 +10,15 @@
 //                memory with cp.async.bulk (1-D bulk copies completing on an
 //                mbarrier); a ring of `stages` rows keeps HBM reads in flight
 //                while the threads work on the current row.
-// A CTA (or, for rows too long for one CTA or too few rows to fill the SMs, a
-// thread-block cluster of CTAs sharing a row through distributed shared memory)
-// takes one row at a time; each thread keeps its elements of x and its folded
+// A CTA (or, for rows too long for one CTA, a thread-block cluster of CTAs
+// sharing a row through distributed shared memory) takes one row at a time; each thread keeps its elements of x and its folded
 // parameters G_k in registers (B_k of 16-byte units in shared memory, read
 // back by the thread that wrote it).  Persistent grid: a CTA (cluster) takes
 // rows c, c + G, ...  Two barriers per row: after the sum of squares and
-// after the row maximum.  The kernel is launched as a
-// programmatic dependent (it waits for the preceding work before touching
-// memory, and lets the next kernel start its set-up after its last row).
+// after the row maximum.  The kernel is launched as a programmatic dependent
+// (it waits for the preceding work before touching memory, or, when the
+// caller promises constant parameters, before touching anything but them;
+// and it lets the next kernel start its set-up after its last row).
 //
 // Arithmetic of the fast path, binary32 two lanes at a time with the sm_100
 // packed instructions (add/mul/fma.rn.f32x2):
@@ -505,7 +505,7 @@ __device__ __forceinline__ void exact_row_lanes(const KParams &p, int64_t row, i
 // Settles one row from its record with an aligned group of g lanes (lane l of
 // g >= 8, gmask: the group's lanes): the exact scales from the candidate
 // units, then the near-tie units' codes, in fp64 from x read back from memory
-// and the parameters (the same arithmetic as settle_kernel).  The loads of the
+// and the parameters.  The loads of the
 // common case (every candidate element, and each lane's first two element
 // pairs of near-tie units) are issued before any arithmetic.
 template <class T, bool INT4, int NOUT, bool ADD, int U>
