@@ -457,6 +457,53 @@ def test_non_default_stream():
     compare(g, run_oracle(w), "int8", "side stream")
 
 
+@pytest.mark.parametrize("rows,n", [(64, 1024), (8, 16384), (1000, 4096)])
+def test_calls_captured_in_a_cuda_graph(rows, n):
+    # arnq_run allocates nothing and never synchronises, so a decode loop can
+    # capture it in a CUDA graph: three calls on three buffer sets, captured
+    # once and replayed twice, give the oracle's results (the programmatic
+    # dependent launches become graph edges)
+    import int4_quant_b200 as q
+    ws_list, outs, ins = [], [], []
+    cases = [wl.random_case(rows, n, seed=300 + i, beta=True, smooth1=True) for i in range(3)]
+    side = torch.cuda.Stream()
+    for w in cases:
+        ins.append((dev_bits(w.x1, "bf16"), dev_bits(w.x2, "bf16"), dev_bits(w.gamma, "bf16"),
+                    dev_bits(w.beta, "bf16"), dev_bits(w.smooth1, "bf16")))
+        outs.append({"y1": torch.empty((rows, n), dtype=torch.int8, device="cuda"),
+                     "scale1": torch.empty(rows, dtype=torch.float32, device="cuda"),
+                     "x_out": torch.empty((rows, n), dtype=torch.bfloat16, device="cuda")})
+    ws, nb = workspace_for(rows, n)
+
+    def calls():
+        for (x1, x2, g, b, s1), o in zip(ins, outs):
+            st = A.arnq_run(x1, x2, g, b, s1, None, rows, n, A.ARNQ_BF16, 1e-6,
+                            A.ARNQ_MASK_ABSENT, A.ARNQ_INT8, o["y1"], o["scale1"], None, None,
+                            o["x_out"], ws, nb, side)
+            assert st == A.ARNQ_OK
+
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        calls()  # plans made and kernels loaded before the capture
+    torch.cuda.synchronize()
+    for o in outs:
+        for t in o.values():
+            t.zero_()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=side):
+        calls()
+    for _ in range(2):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    for w, o in zip(cases, outs):
+        g = {"y1": o["y1"].cpu().numpy().view(np.uint8), "scale1": o["scale1"].cpu().numpy(),
+             "x_out": o["x_out"].view(torch.int16).cpu().numpy().view(np.uint16),
+             "y2": np.full((rows, n), CANARY, np.uint8),  # not selected: not compared
+             "scale2": np.full(rows * 4, CANARY, np.uint8).view(np.float32)}
+        compare(g, run_oracle(w), "int8", f"graph {rows}x{n}")
+
+
 # ------------------------------------------------------------------ device-side failure paths
 
 def _call_with_plan(w, p, ws, nb, outputs=False):
