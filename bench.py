@@ -474,6 +474,65 @@ class DeviceRun:
         return (t1 - t0) / calls * 1e6
 
 
+def time_no_add(w, dev, stream, peak, calls=200, regions=5):
+    """The no-add operator (arnq_rms_norm_dynamic_quant: x normalised as given,
+    one output, no xOut) on workload w's x1, gamma, beta and smooth1: device
+    time per call of `calls` calls back to back on 3 rotated L2-cold sets."""
+    import ctypes
+    import torch
+    from int4_quant_b200 import _abi as A
+    TDT = {"bf16": torch.bfloat16, "fp16": torch.float16}[w.dtype]
+    dt = A.ARNQ_BF16 if w.dtype == "bf16" else A.ARNQ_FP16
+    qd = A.ARNQ_INT8 if w.qdtype == "int8" else A.ARNQ_INT4
+
+    def to_dev(bits):
+        if bits is None:
+            return None
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(TDT)
+
+    cb = w.n if w.qdtype == "int8" else w.n // 2
+    x0 = to_dev(w.x1)
+    g, b, s1 = to_dev(w.gamma), to_dev(w.beta), to_dev(w.smooth1)
+    sets = [dict(x=x0 if i == 0 else x0.clone(),
+                 y=torch.empty((w.rows, cb), dtype=torch.uint8, device=dev),
+                 s=torch.empty((w.rows,), dtype=torch.float32, device=dev)) for i in range(3)]
+    st, nb = A.arnq_workspace_size(w.rows, w.n, dt, qd, A.ARNQ_MASK_ABSENT, s1 is not None, False)
+    if st != A.ARNQ_OK:
+        raise A.ArnqError(st, "arnq_workspace_size")
+    ws = torch.zeros(nb, dtype=torch.uint8, device=dev)
+    fn = A.lib().arnq_rms_norm_dynamic_quant
+    P = A._ptr
+    args = [(P(t["x"]), P(g), P(b), P(s1), w.rows, w.n, dt, ctypes.c_float(w.eps), qd, P(t["y"]),
+             P(t["s"]), P(ws), nb, A._stream(stream)) for t in sets]
+    out = []
+    for _ in range(regions):
+        for i in range(20):
+            fn(*args[i % 3])
+        torch.cuda.synchronize(dev)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        hold_device(torch)
+        e0.record(stream)
+        for i in range(calls):
+            if fn(*args[i % 3]):
+                raise RuntimeError("arnq_rms_norm_dynamic_quant failed")
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        out.append(e0.elapsed_time(e1) / calls)
+    if int(ws[:4].view(torch.int32).item()) != 0:
+        raise RuntimeError("no-add run: device status set")
+    ms = statistics.median(out)
+    nbytes = algorithmic_bytes(w.rows, w.n, w.dtype, w.qdtype, w.beta is not None,
+                               w.smooth1 is not None, False, True, False, has_x2=False,
+                               x_out=False)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"us_per_call": ms * 1e3, "us_per_call_min_max": [min(out) * 1e3, max(out) * 1e3],
+            "gbs": gbs, "frac": gbs / peak, "bytes_per_call": nbytes,
+            "rows_per_s": w.rows / (ms / 1e3),
+            "timing": f"{calls} calls back to back, 3 sets; median of {regions} timed regions",
+            "workload": "rms_norm_dynquant_" + w.name.split("add_rmsnorm_dynquant_", 1)[-1]}
+
+
 def workload_entry(run, ms, peak, how):
     """One line of the `workloads` object: a call's time, throughput, roofline."""
     gbs = run.bytes / (ms / 1e3) / 1e9
@@ -709,6 +768,9 @@ def main():
             workloads[name] = e
             del wr
             torch.cuda.empty_cache()
+        # the no-add operator on the 8192 x 4096 workload's x1 and parameters
+        workloads["c2_no_add"] = time_no_add(wl.CONFIGS["c2"](), dev, stream, peak)
+        torch.cuda.empty_cache()
         for name in SMALL:
             ww = wl.CONFIGS[name]()
             o1, o2 = outputs_of(ww)

@@ -69,6 +69,16 @@ def test_bench_workload_floor():
     assert abs(nbytes / 6554.6e9 * 1e6 - 35.84) < 0.01
 
 
+def test_algorithmic_bytes_of_the_no_add_operator():
+    # rms_norm_dynamic_quant on the 8192 x 4096 workload's x1 and parameters:
+    # per row x read (2 B/element), INT8 codes written (1 B/element) and one
+    # fp32 scale; no x2, no xOut; gamma, beta, smooth1 read once
+    per_row = 4096 * 2 + 4096 + 4
+    assert bench.algorithmic_bytes(8192, 4096, "bf16", "int8", True, True, False, True, False,
+                                   has_x2=False, x_out=False) == 8192 * per_row + 3 * 4096 * 2
+    assert 8192 * per_row + 3 * 4096 * 2 == 100_720_640
+
+
 def test_launches_per_call():
     # one kernel per call, whether a row has one CTA or a cluster
     class P:
