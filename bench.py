@@ -18,16 +18,22 @@ so there is no data-path collective) and the time is the maximum over ranks.
 
 Also printed, on the same JSON line: rows/s, the roofline of the kernel
 (achieved GB/s from the mean per-launch CUDA-event duration against the
-measured copy bandwidth), the end-to-end figure through the public call with
-host buffers (H2D copies, the call, D2H of the outputs, all inside the timed
-region), SM clocks sampled by NVML during the timed region, and the CPU
+measured copy bandwidth, and the DRAM traffic per launch recorded by ncu for
+this kernel source), five more timed regions of K calls (the figure's
+spread), the same K calls with the opt-in early parameter loads, the
+end-to-end figure through the public call with host buffers (every step's
+H2D copies, the call and the D2H copy of its outputs inside the timed region;
+two buffer sets so that one step's copy-in overlaps the previous step's
+copy-out), SM clocks sampled by NVML during the timed region, and the CPU
 oracle's throughput on a bounded sample (rank 0, one GPU only).  The
 `workloads` object carries the other configurations measured in the same
-run: the large ones (>= 80 % roofline class) as device time per call of calls
-back to back, the small, latency-bound ones as device time per call from a
-CUDA graph of back-to-back calls (L2-cold and L2-hot) and as host time per
-call.  The timed loops call arnq_run through ctypes with arguments marshalled
-once, so that the host keeps ahead of the device.
+run: the large ones as device time per call of calls back to back (median of
+five regions, with the early-parameter figure), the no-add operator on the
+8192 x 4096 inputs, and the small, latency-bound ones as device time per call
+from a CUDA graph of back-to-back calls (L2-cold and L2-hot) and as host time
+per call.  The timed loops call arnq_run through ctypes with arguments
+marshalled once, and each timed region is queued behind a short device-side
+delay, so that the host's launches are not what is timed.
 
 --impl reference times the CPU oracle (the only other implementation of the
 operator; there is no runnable reference library) on the host cores.
